@@ -1,0 +1,185 @@
+"""Seeded synthetic workloads for exact attention.
+
+This module only draws random inputs and describes problem sizes.  It contains no
+attention arithmetic, and both the CUDA path's tests/bench and the CPU oracle's tests
+take their inputs from here, so the two sides always see identical 16-bit values.
+
+Recipe (identical for every workload):
+  * a CPU ``torch.Generator`` seeded with the workload's seed;
+  * ``torch.randn`` in float32 drawn in the order Q, K, V, dO (standard normal, the
+    i.i.d. N(0, 1) inputs the workloads call for);
+  * optional multiplication of Q and K by ``qk_mult`` (the "peaky softmax" stress case);
+  * a cast to the workload dtype (bf16 or fp16) on the CPU.
+The exact 16-bit tensors are what the GPU receives; their float64 upcast is what the
+oracle receives.
+
+Varlen lengths for the 64-sequence case are drawn with
+``numpy.random.default_rng(3).integers(64, 4097, size=64)`` (uniform on [64, 4096]).
+
+Problem sizes follow the shapes the pages use: the A100 table of the page
+"FlashAttention实战：如何在A100上实现3倍加速的Transformer训练" §6 (B=8, H=16, d=64,
+N=1K..4K), the Llama-style head and 16K benchmark of "FlashAttention-2的核心设计原理"
+(B=4/2, H=32, d=128) and its varlen example (lengths 128/256/512, cu_seqlens
+[0, 128, 384, 896]).
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Optional
+
+import numpy as np
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    H: int
+    d: int
+    dtype: str                       # "bf16" | "fp16"
+    causal: bool
+    seed: int
+    B: int = 0                       # dense only
+    N: int = 0                       # dense only
+    seqlens: Optional[tuple] = None  # varlen only
+    qk_mult: float = 1.0
+    scale: Optional[float] = None    # default 1/sqrt(d)
+
+    @property
+    def varlen(self) -> bool:
+        return self.seqlens is not None
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float16
+
+    @property
+    def total(self) -> int:
+        return int(sum(self.seqlens)) if self.varlen else self.B * self.N
+
+    def cu_seqlens(self) -> np.ndarray:
+        assert self.varlen
+        return np.concatenate([[0], np.cumsum(self.seqlens)]).astype(np.int32)
+
+    def fwd_flops(self) -> float:
+        """4·B·H·N²·d forward FLOPs, halved when causal; varlen sums per sequence."""
+        if self.varlen:
+            f = sum(4.0 * self.H * L * L * self.d for L in self.seqlens)
+        else:
+            f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+    def bwd_flops(self) -> float:
+        return 2.5 * self.fwd_flops()
+
+    def shape(self):
+        if self.varlen:
+            return (self.total, self.H, self.d)
+        return (self.B, self.N, self.H, self.d)
+
+    def describe(self) -> dict:
+        out = {"workload": self.name, "H": self.H, "d": self.d, "dtype": self.dtype,
+               "causal": self.causal, "seed": self.seed, "scale": self.softmax_scale}
+        if self.varlen:
+            out.update(num_seqs=len(self.seqlens), total_tokens=self.total,
+                       max_seqlen=int(max(self.seqlens)))
+        else:
+            out.update(B=self.B, N=self.N)
+        if self.qk_mult != 1.0:
+            out["qk_mult"] = self.qk_mult
+        return out
+
+
+def varlen_lengths_64(seed: int = 3) -> tuple:
+    rng = np.random.default_rng(seed)
+    return tuple(int(x) for x in rng.integers(64, 4097, size=64))
+
+
+def _registry():
+    w = {}
+
+    def add(x: Workload):
+        w[x.name] = x
+
+    for causal in (False, True):
+        c = "causal" if causal else "noncausal"
+        add(Workload(f"tiny_{c}", B=1, H=2, N=128, d=64, dtype="bf16", causal=causal, seed=0,
+                     scale=1.0 / 8.0))
+    for N in (1024, 2048, 4096):
+        add(Workload(f"a100table_N{N}", B=8, H=16, N=N, d=64, dtype="bf16", causal=True,
+                     seed=1, scale=1.0 / 8.0))
+    for causal in (False, True):
+        c = "causal" if causal else "noncausal"
+        add(Workload(f"llama_{c}", B=4, H=32, N=4096, d=128, dtype="fp16", causal=causal,
+                     seed=2))
+    add(Workload("varlen3", H=32, d=128, dtype="bf16", causal=True, seed=3,
+                 seqlens=(128, 256, 512)))
+    add(Workload("varlen64", H=32, d=128, dtype="bf16", causal=True, seed=3,
+                 seqlens=varlen_lengths_64(3)))
+    for causal in (False, True):
+        c = "causal" if causal else "noncausal"
+        add(Workload(f"long_{c}", B=2, H=32, N=16384, d=128, dtype="bf16", causal=causal,
+                     seed=4))
+        add(Workload(f"long_peaky_{c}", B=2, H=32, N=16384, d=128, dtype="bf16",
+                     causal=causal, seed=4, qk_mult=4.0))
+    return w
+
+
+WORKLOADS = _registry()
+
+
+def get(name: str) -> Workload:
+    return WORKLOADS[name]
+
+
+def custom(name="custom", *, B=1, N=128, H=1, d=64, dtype="bf16", causal=False, seed=0,
+           seqlens=None, qk_mult=1.0, scale=None) -> Workload:
+    """An ad-hoc workload (ragged sizes, edge cases) built with the same recipe."""
+    if seqlens is not None:
+        return Workload(name, H=H, d=d, dtype=dtype, causal=causal, seed=seed,
+                        seqlens=tuple(int(x) for x in seqlens), qk_mult=qk_mult, scale=scale)
+    return Workload(name, B=B, N=N, H=H, d=d, dtype=dtype, causal=causal, seed=seed,
+                    qk_mult=qk_mult, scale=scale)
+
+
+def generate(w: Workload, with_grad_out: bool = True):
+    """Return dict of CPU 16-bit tensors q, k, v (and do) with the workload's shape."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    shape = w.shape()
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    out = {}
+    if w.qk_mult != 1.0:
+        q = q * w.qk_mult
+        k = k * w.qk_mult
+    out["q"] = q.to(w.torch_dtype)
+    out["k"] = k.to(w.torch_dtype)
+    out["v"] = v.to(w.torch_dtype)
+    if with_grad_out:
+        out["do"] = torch.randn(shape, generator=g, dtype=torch.float32).to(w.torch_dtype)
+    if w.varlen:
+        out["cu_seqlens"] = torch.from_numpy(w.cu_seqlens())
+    return out
+
+
+def sample_rows(n_rows: int, k: int, seed: int) -> np.ndarray:
+    """Sorted seeded subset of query/key rows, always containing the tile and causal
+    boundaries 0, 1, 127, 128 and n_rows-1 (when they exist)."""
+    rng = np.random.default_rng(seed)
+    base = {0, 1, 127, 128, n_rows - 1}
+    base = {r for r in base if 0 <= r < n_rows}
+    k = min(k, n_rows)
+    pick = set(int(x) for x in rng.choice(n_rows, size=k, replace=False))
+    return np.array(sorted(pick | base), dtype=np.int64)
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.to(torch.float64).numpy()

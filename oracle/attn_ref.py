@@ -1,0 +1,242 @@
+"""fp64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or run this
+module: only the tests, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` use it.  It shares no code, constants or
+helpers with the CUDA library.
+
+What it computes is the plain definition of attention given as "standard attention"
+on the page "FlashAttention-2的核心设计原理" (yunthe.com), section
+"FlashAttention-2与标准注意力的计算对比": scores = Q Kᵀ / sqrt(d), a softmax over the
+keys, output = weights · V.  It is generalised to
+
+* an explicit ``scale`` (the pages pass softmax_scale = 1/sqrt(head_dim): page
+  "FlashAttention实战：如何在A100上实现3倍加速的Transformer训练" (jsqmd.com/news/620004)
+  section 4.1; any value, zero and negative included, is accepted here),
+* causal masking (the ``causal=True`` flag used on both pages) read bottom-right aligned:
+  key j is allowed for query i iff j <= i + (Lk - Lq); identical to the usual
+  top-left rule whenever Lq == Lk,
+* the log-sum-exp of each row in natural-log, scaled-score units,
+  LSE_i = ln sum_j exp(scale * q_i . k_j), the O(N) statistic the backward pass keeps
+  (page "Flash Attention V3：大模型训练加速与显存优化技术解析" (jsqmd.com/news/1204652)
+  section 3.2: O(N) storage, recomputation in the backward pass),
+* the analytic backward of O = softmax(scale Q Kᵀ) V (chain rule; the pages only say
+  that the backward pass recomputes the forward: "FlashAttention-2的核心设计原理",
+  section "FlashAttention-2反向传播与多GPU训练").
+
+Fully masked rows (possible only when Lk < Lq under the bottom-right rule, or when
+Lk == 0) give O = 0 and LSE = +inf, and contribute nothing to any gradient.
+
+Every number is float64.  Large problems are evaluated one block of at most
+``ROW_BLOCK`` query rows at a time: each block materialises its full row of scores
+against every key, so this is still the definition (each row of a softmax is
+independent of every other row), not an online or tiled reformulation.
+
+Parity status: every function here is pinned by tests/test_oracle_pins.py (closed
+forms, invariants, brute force, finite differences, a hand-worked golden example).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+ROW_BLOCK = 1024
+
+
+def allowed_mask(rows: np.ndarray, Lq: int, Lk: int, causal: bool) -> np.ndarray:
+    """Boolean [len(rows), Lk]: which keys each listed query row may attend to.
+
+    Causal reading (bottom-right): key j is allowed for query i iff j <= i + (Lk - Lq).
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    keys = np.arange(Lk, dtype=np.int64)
+    if not causal:
+        return np.ones((rows.shape[0], Lk), dtype=bool)
+    return keys[None, :] <= (rows[:, None] + (Lk - Lq))
+
+
+def _scores(q_rows: np.ndarray, k: np.ndarray, scale: float, mask: np.ndarray) -> np.ndarray:
+    """S = scale * Q_rows Kᵀ with disallowed entries set to -inf."""
+    s = scale * (q_rows @ k.T)
+    return np.where(mask, s, -np.inf)
+
+
+def _row_softmax_stats(s: np.ndarray):
+    """Row max m, row sum l = sum exp(S - m) and LSE = m + ln l of a score block.
+
+    Rows with no allowed key get m = -inf, l = 0, LSE = +inf.
+    """
+    m = s.max(axis=1) if s.shape[1] > 0 else np.full(s.shape[0], -np.inf)
+    dead = ~np.isfinite(m)
+    m_safe = np.where(dead, 0.0, m)
+    e = np.exp(s - m_safe[:, None])  # exp(-inf) = 0 for masked entries
+    l = e.sum(axis=1)
+    with np.errstate(divide="ignore"):
+        lse = np.where(dead, np.inf, m_safe + np.log(np.where(dead, 1.0, l)))
+    return m_safe, l, lse, e, dead
+
+
+def softmax_probs(q, k, scale, causal, rows=None):
+    """P = softmax(scale Q Kᵀ) for the listed query rows: [len(rows), Lk] float64.
+
+    Fully masked rows are all zero.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    Lq, Lk = q.shape[0], k.shape[0]
+    rows = np.arange(Lq) if rows is None else np.asarray(rows, dtype=np.int64)
+    s = _scores(q[rows], k, scale, allowed_mask(rows, Lq, Lk, causal))
+    _, l, _, e, dead = _row_softmax_stats(s)
+    return e / np.where(dead, 1.0, l)[:, None]
+
+
+def attention_forward(q, k, v, scale, causal, rows=None):
+    """O and LSE of one (batch, head) or one packed segment.
+
+    q: [Lq, d], k: [Lk, d], v: [Lk, dv] (any float dtype; upcast to float64).
+    rows: optional sorted query-row indices; only those rows are evaluated.
+    Returns (O [n_rows, dv], LSE [n_rows]) in float64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    Lq, Lk = q.shape[0], k.shape[0]
+    rows = np.arange(Lq) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.zeros((rows.shape[0], v.shape[1]), dtype=np.float64)
+    lse = np.zeros(rows.shape[0], dtype=np.float64)
+    for b0 in range(0, rows.shape[0], ROW_BLOCK):
+        r = rows[b0:b0 + ROW_BLOCK]
+        s = _scores(q[r], k, scale, allowed_mask(r, Lq, Lk, causal))
+        _, l, blk_lse, e, dead = _row_softmax_stats(s)
+        p = e / np.where(dead, 1.0, l)[:, None]
+        out[b0:b0 + r.shape[0]] = p @ v
+        lse[b0:b0 + r.shape[0]] = blk_lse
+    return out, lse
+
+
+def attention_backward(q, k, v, do, scale, causal, dq_rows=None, dkv_rows=None):
+    """Analytic gradients of O = softmax(scale Q Kᵀ) V for one (batch, head) / segment.
+
+    With P the softmax weights and D_i = sum_c dO_ic O_ic (O from this oracle, float64):
+      dV = Pᵀ dO,  dP = dO Vᵀ,  dS = P ∘ (dP − D),  dQ = scale dS K,  dK = scale dSᵀ Q.
+
+    dq_rows: query rows whose dQ is wanted (default: all).
+    dkv_rows: key rows whose dK, dV are wanted (default: all).
+    Returns (dQ [len(dq_rows), d], dK [len(dkv_rows), d], dV [len(dkv_rows), dv]).
+
+    Every entry of P used here is exp(S_ij − LSE_i) with LSE from the full row of
+    scores, i.e. the softmax definition itself; dK/dV rows need the statistics of
+    every query row, which are computed block by block.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    Lq, Lk = q.shape[0], k.shape[0]
+    dq_rows = np.arange(Lq) if dq_rows is None else np.asarray(dq_rows, dtype=np.int64)
+    dkv_rows = np.arange(Lk) if dkv_rows is None else np.asarray(dkv_rows, dtype=np.int64)
+
+    # dQ rows: each needs its own full row of P and dP.
+    dq = np.zeros((dq_rows.shape[0], q.shape[1]), dtype=np.float64)
+    for b0 in range(0, dq_rows.shape[0], ROW_BLOCK):
+        r = dq_rows[b0:b0 + ROW_BLOCK]
+        p = softmax_probs(q, k, scale, causal, rows=r)
+        o = p @ v
+        d_row = (do[r] * o).sum(axis=1)
+        dp = do[r] @ v.T
+        ds = p * (dp - d_row[:, None])
+        dq[b0:b0 + r.shape[0]] = scale * (ds @ k)
+
+    # dK / dV rows: need P[:, keys] for every query row, hence every row's LSE and D.
+    dk = np.zeros((dkv_rows.shape[0], k.shape[1]), dtype=np.float64)
+    dv = np.zeros((dkv_rows.shape[0], v.shape[1]), dtype=np.float64)
+    if dkv_rows.shape[0] > 0 and Lq > 0:
+        for b0 in range(0, Lq, ROW_BLOCK):
+            r = np.arange(b0, min(Lq, b0 + ROW_BLOCK))
+            mask = allowed_mask(r, Lq, Lk, causal)
+            s_full = _scores(q[r], k, scale, mask)
+            _, l, lse, e, dead = _row_softmax_stats(s_full)
+            p_full = e / np.where(dead, 1.0, l)[:, None]
+            o = p_full @ v
+            d_row = (do[r] * o).sum(axis=1)
+            p = p_full[:, dkv_rows]
+            dp = do[r] @ v[dkv_rows].T
+            ds = p * (dp - d_row[:, None])
+            dv += p.T @ do[r]
+            dk += scale * (ds.T @ q[r])
+    return dq, dk, dv
+
+
+def attention_forward_bhsd(q, k, v, scale, causal):
+    """Dense batched forward over the pages' [batch, seqlen, heads, head_dim] layout.
+
+    Returns O [B, N, H, d] and LSE [B, H, N] (float64).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, N, H, _ = q.shape
+    out = np.zeros(q.shape[:3] + (v.shape[3],), dtype=np.float64)
+    lse = np.zeros((B, H, N), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            o, l = attention_forward(q[b, :, h], k[b, :, h], v[b, :, h], scale, causal)
+            out[b, :, h] = o
+            lse[b, h] = l
+    return out, lse
+
+
+def attention_backward_bhsd(q, k, v, do, scale, causal):
+    """Dense batched backward over [batch, seqlen, heads, head_dim]: (dQ, dK, dV)."""
+    q = np.asarray(q, dtype=np.float64)
+    B, _, H, _ = q.shape
+    dq = np.zeros(q.shape, dtype=np.float64)
+    dk = np.zeros(np.shape(k), dtype=np.float64)
+    dv = np.zeros(np.shape(v), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            a, bb, c = attention_backward(q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h],
+                                          scale, causal)
+            dq[b, :, h], dk[b, :, h], dv[b, :, h] = a, bb, c
+    return dq, dk, dv
+
+
+def varlen_attention_forward(q, k, v, cu_seqlens_q, cu_seqlens_k, scale, causal):
+    """Packed variable-length forward: [total, H, d] tensors, one segment per sequence.
+
+    Segment s holds query rows cu_seqlens_q[s]:cu_seqlens_q[s+1] and key/value rows
+    cu_seqlens_k[s]:cu_seqlens_k[s+1] (flash_attn_varlen_func usage on the page
+    "FlashAttention-2的核心设计原理", section "变长序列处理与flash_attn_varlen_func").  No key outside a query's own
+    segment takes part.  Returns O [total_q, H, dv] and LSE [H, total_q].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    total_q, H, _ = q.shape
+    out = np.zeros((total_q, H, v.shape[2]), dtype=np.float64)
+    lse = np.zeros((H, total_q), dtype=np.float64)
+    for s in range(len(cu_seqlens_q) - 1):
+        q0, q1 = int(cu_seqlens_q[s]), int(cu_seqlens_q[s + 1])
+        k0, k1 = int(cu_seqlens_k[s]), int(cu_seqlens_k[s + 1])
+        for h in range(H):
+            o, l = attention_forward(q[q0:q1, h], k[k0:k1, h], v[k0:k1, h], scale, causal)
+            out[q0:q1, h] = o
+            lse[h, q0:q1] = l
+    return out, lse
+
+
+def varlen_attention_backward(q, k, v, do, cu_seqlens_q, cu_seqlens_k, scale, causal):
+    """Packed variable-length backward: (dQ [total_q,H,d], dK [total_k,H,d], dV)."""
+    q = np.asarray(q, dtype=np.float64)
+    dq = np.zeros(q.shape, dtype=np.float64)
+    dk = np.zeros(np.shape(k), dtype=np.float64)
+    dv = np.zeros(np.shape(v), dtype=np.float64)
+    H = q.shape[1]
+    for s in range(len(cu_seqlens_q) - 1):
+        q0, q1 = int(cu_seqlens_q[s]), int(cu_seqlens_q[s + 1])
+        k0, k1 = int(cu_seqlens_k[s]), int(cu_seqlens_k[s + 1])
+        for h in range(H):
+            a, b, c = attention_backward(q[q0:q1, h], k[k0:k1, h], v[k0:k1, h],
+                                         do[q0:q1, h], scale, causal)
+            dq[q0:q1, h], dk[k0:k1, h], dv[k0:k1, h] = a, b, c
+    return dq, dk, dv
