@@ -1,0 +1,196 @@
+"""Python binding of libfattn: argument marshalling only.
+
+Every step of the attention computation runs in the library's CUDA kernels; this module
+checks tensor shapes/dtypes/devices, allocates outputs with PyTorch (device memory is
+PyTorch's job here) and passes raw pointers and the current CUDA stream to the C ABI.
+
+API shapes follow the pages' usage: ``flash_attn_func(q, k, v, softmax_scale, causal)``
+on [batch, seqlen, heads, head_dim] tensors and ``flash_attn_varlen_func`` on packed
+[total, heads, head_dim] tensors with cu_seqlens (page "FlashAttention-2的核心设计原理",
+sections "FlashAttention-2在PyTorch中的安装与使用" and
+"变长序列处理与flash_attn_varlen_func"); the backward pass is reached through autograd
+(section "FlashAttention-2反向传播与多GPU训练").
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+_DTYPES = {torch.bfloat16: _lib.FA_BF16, torch.float16: _lib.FA_FP16}
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _check(*ts: torch.Tensor):
+    dev = ts[0].device
+    dt = ts[0].dtype
+    if dev.type != "cuda":
+        raise ValueError("attention tensors must be CUDA tensors")
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}; use bfloat16 or float16")
+    for t in ts:
+        if t.device != dev or t.dtype != dt:
+            raise ValueError("all attention tensors must share device and dtype")
+        if not t.is_contiguous():
+            raise ValueError("attention tensors must be contiguous")
+    return _DTYPES[dt]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def fwd(q, k, v, softmax_scale=None, causal=False, out=None, lse=None):
+    """Dense forward. q, k, v: [B, N, H, d]. Returns (o [B,N,H,d], lse [B,H,N] fp32)."""
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must all be [B, N, H, d] with equal shapes")
+    dtype = _check(q, k, v)
+    B, N, H, d = q.shape
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, N, H, d, scale,
+                        int(bool(causal)), dtype, _stream(q))
+    _lib.check(st, "fa_fwd")
+    return o, lse_t
+
+
+def varlen_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+               softmax_scale=None, causal=False, out=None, lse=None):
+    """Varlen forward. q: [total_q, H, d]; k, v: [total_k, H, d]; cu_seqlens int32 on device.
+    Returns (o [total_q,H,d], lse [H,total_q] fp32)."""
+    if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape or q.shape[1:] != k.shape[1:]:
+        raise ValueError("q must be [total_q, H, d] and k, v [total_k, H, d]")
+    dtype = _check(q, k, v)
+    for cu in (cu_seqlens_q, cu_seqlens_k):
+        if cu.dtype != torch.int32 or cu.device != q.device or not cu.is_contiguous():
+            raise ValueError("cu_seqlens must be contiguous int32 tensors on q's device")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have num_seqs + 1 entries")
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((H, total_q), device=q.device, dtype=torch.float32) if lse is None else lse
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_varlen_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), _ptr(cu_seqlens_q),
+                               _ptr(cu_seqlens_k), int(max_seqlen_q), int(max_seqlen_k), H, d,
+                               scale, int(bool(causal)), cu_seqlens_q.numel() - 1, total_q,
+                               total_k, dtype, _stream(q))
+    _lib.check(st, "fa_varlen_fwd")
+    return o, lse_t
+
+
+def bwd_workspace(B, N, H, d, device) -> torch.Tensor:
+    n = _lib.load().fa_bwd_workspace_size(B, N, H, d)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def varlen_bwd_workspace(total_q, H, d, device) -> torch.Tensor:
+    n = _lib.load().fa_varlen_bwd_workspace_size(total_q, H, d)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def bwd(q, k, v, o, lse, dout, softmax_scale=None, causal=False, workspace=None,
+        dq=None, dk=None, dv=None):
+    """Dense backward. Returns (dq, dk, dv), each [B, N, H, d]."""
+    dtype = _check(q, k, v, o, dout)
+    B, N, H, d = q.shape
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws = bwd_workspace(B, N, H, d, q.device) if workspace is None else workspace
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                        _ptr(dk), _ptr(dv), B, N, H, d, scale, int(bool(causal)), _ptr(ws),
+                        ws.numel(), dtype, _stream(q))
+    _lib.check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def varlen_bwd(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+               softmax_scale=None, causal=False, workspace=None, dq=None, dk=None, dv=None):
+    """Varlen backward. Returns (dq [total_q,H,d], dk, dv [total_k,H,d])."""
+    dtype = _check(q, k, v, o, dout)
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws = varlen_bwd_workspace(total_q, H, d, q.device) if workspace is None else workspace
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_varlen_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                               _ptr(dk), _ptr(dv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+                               int(max_seqlen_q), int(max_seqlen_k), H, d, scale,
+                               int(bool(causal)), cu_seqlens_q.numel() - 1, total_q, total_k,
+                               _ptr(ws), ws.numel(), dtype, _stream(q))
+    _lib.check(st, "fa_varlen_bwd")
+    return dq, dk, dv
+
+
+def device_status(stream: Optional[int] = None) -> int:
+    """Synchronise and return the library status word (0 = ok, 4 = a wait timed out)."""
+    lib = _lib.load()
+    s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    return lib.fa_get_device_status(s)
+
+
+class FlashAttnFunction(torch.autograd.Function):
+    """Autograd wrapper: forward saves (q, k, v, o, lse); backward recomputes P."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, softmax_scale, causal):
+        o, lse = fwd(q, k, v, softmax_scale, causal)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.softmax_scale = softmax_scale
+        ctx.causal = causal
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = bwd(q, k, v, o, lse, do.contiguous(), ctx.softmax_scale, ctx.causal)
+        return dq, dk, dv, None, None
+
+
+class FlashAttnVarlenFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, cu_q, cu_k, max_q, max_k, softmax_scale, causal):
+        o, lse = varlen_fwd(q, k, v, cu_q, cu_k, max_q, max_k, softmax_scale, causal)
+        ctx.save_for_backward(q, k, v, o, lse, cu_q, cu_k)
+        ctx.args = (max_q, max_k, softmax_scale, causal)
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse, cu_q, cu_k = ctx.saved_tensors
+        max_q, max_k, scale, causal = ctx.args
+        dq, dk, dv = varlen_bwd(q, k, v, o, lse, do.contiguous(), cu_q, cu_k, max_q, max_k,
+                                scale, causal)
+        return dq, dk, dv, None, None, None, None, None, None
+
+
+def flash_attn_func(q, k, v, softmax_scale=None, causal=False):
+    """[batch, seqlen, heads, head_dim] attention with autograd."""
+    return FlashAttnFunction.apply(q, k, v, softmax_scale, causal)
+
+
+def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                           softmax_scale=None, causal=False):
+    """Packed variable-length attention with autograd."""
+    return FlashAttnVarlenFunction.apply(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                                         max_seqlen_k, softmax_scale, causal)

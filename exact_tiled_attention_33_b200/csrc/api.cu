@@ -1,0 +1,278 @@
+// C ABI of libfattn: argument validation, TMA tensor-map encoding, launches, status.
+// The operations are documented in include/fattn.h.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/fattn.h"
+#include "fattn_internal.h"
+#include "sm100.cuh"
+
+namespace fattn {
+
+// One status word per device (each device that loads the module gets its own copy).
+__device__ uint32_t g_status_word;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const std::string& msg) {
+  g_last_error = msg;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(FA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tensor map over a [batches, rows, H, d] 16-bit tensor, dims listed innermost first
+// (d, H, rows, batches); box = 64 elements of d (one 128-byte swizzle row) x 1 head x
+// box_rows rows.  Out-of-range rows read as zero.
+int make_map(CUtensorMap* map, const void* base, int d, int H, long long rows, long long batches,
+             int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)batches};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2,
+                           (cuuint64_t)rows * H * d * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
+  return FA_OK;
+}
+
+uint32_t* status_ptr() {
+  static uint32_t* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return nullptr;
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<uint32_t*>(p);
+  }
+  return ptrs[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int H, int d, int dtype, float scale) {
+  if (H < 0 || H > 65535) return fail(FA_ERR_UNSUPPORTED, "H must be in [0, 65535]");
+  if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (dtype != FA_BF16 && dtype != FA_FP16) return fail(FA_ERR_UNSUPPORTED, "unknown dtype");
+  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
+  return FA_OK;
+}
+
+int check_ptrs(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs) {
+    if (p == nullptr) return fail(FA_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(p)) return fail(FA_ERR_INVALID_ARG, "pointer not 16-byte aligned");
+  }
+  return FA_OK;
+}
+
+int launch_result(LaunchResult r) {
+  if (r == LaunchResult::kOk) return FA_OK;
+  if (r == LaunchResult::kUnsupported) return fail(FA_ERR_UNSUPPORTED, "unsupported configuration");
+  return cuda_fail(cudaGetLastError(), "kernel launch");
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace
+
+// Bounded-wait self test: waits on a barrier that nothing arrives at.
+__global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  mbar_wait_limit(smem_u32(&bar), 0, &abort_flag, status, limit_ns);
+}
+
+}  // namespace fattn
+
+using namespace fattn;
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N, int H,
+           int d, float scale, int causal, int dtype, void* stream) {
+  g_last_error.clear();
+  if (int e = check_common(H, d, dtype, scale)) return e;
+  if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
+  if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
+  if (B == 0 || N == 0 || H == 0) return FA_OK;
+  if (B > 65535) return fail(FA_ERR_UNSUPPORTED, "B must be <= 65535");
+  if (int e = check_ptrs({q, k, v, o, lse})) return e;
+  CUtensorMap mq, mk, mv;
+  if (int e = make_map(&mq, q, d, H, N, B, 128)) return e;
+  if (int e = make_map(&mk, k, d, H, N, B, 128)) return e;
+  if (int e = make_map(&mv, v, d, H, N, B, 128)) return e;
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.cu_q = p.cu_k = nullptr;
+  p.N = N;
+  p.H = H;
+  p.total_q = B * N;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.causal = causal ? 1 : 0;
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  const int rows = fwd_rows_per_cta();
+  dim3 grid((N + rows - 1) / rows, H, B);
+  return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+}
+
+int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int max_seqlen_q,
+                  int max_seqlen_k, int H, int d, float scale, int causal, int num_seqs,
+                  int total_q, int total_k, int dtype, void* stream) {
+  g_last_error.clear();
+  if (int e = check_common(H, d, dtype, scale)) return e;
+  if (num_seqs < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
+    return fail(FA_ERR_INVALID_ARG, "sizes must be >= 0");
+  if (num_seqs > 65535) return fail(FA_ERR_UNSUPPORTED, "num_seqs must be <= 65535");
+  if (max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return fail(FA_ERR_INVALID_ARG, "max_seqlen exceeds the total token count");
+  if (num_seqs == 0 || total_q == 0 || H == 0 || max_seqlen_q == 0) return FA_OK;
+  if (int e = check_ptrs({q, o, lse, cu_seqlens_q, cu_seqlens_k})) return e;
+  if (total_k > 0)
+    if (int e = check_ptrs({k, v})) return e;
+  CUtensorMap mq, mk, mv;
+  if (int e = make_map(&mq, q, d, H, total_q, 1, 128)) return e;
+  // With no keys at all every row is fully masked and K/V are never read.
+  const void* kb = total_k > 0 ? k : q;
+  const void* vb = total_k > 0 ? v : q;
+  const long long kr = total_k > 0 ? total_k : total_q;
+  if (int e = make_map(&mk, kb, d, H, kr, 1, 128)) return e;
+  if (int e = make_map(&mv, vb, d, H, kr, 1, 128)) return e;
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.N = 0;
+  p.H = H;
+  p.total_q = total_q;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.causal = causal ? 1 : 0;
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  const int rows = fwd_rows_per_cta();
+  dim3 grid((max_seqlen_q + rows - 1) / rows, H, num_seqs);
+  return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t fa_bwd_workspace_size(int B, int N, int H, int d) {
+  if (B <= 0 || N <= 0 || H <= 0 || d <= 0) return 0;
+  const size_t e = (size_t)B * N * H * d;
+  return align256(e * 4) + align256((size_t)B * H * N * 4);
+}
+
+size_t fa_varlen_bwd_workspace_size(int total_q, int H, int d) {
+  if (total_q <= 0 || H <= 0 || d <= 0) return 0;
+  const size_t e = (size_t)total_q * H * d;
+  return align256(e * 4) + align256((size_t)H * total_q * 4);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d, float scale,
+           int causal, void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  g_last_error.clear();
+  (void)q; (void)k; (void)v; (void)o; (void)dout; (void)lse; (void)dq; (void)dk; (void)dv;
+  (void)B; (void)N; (void)H; (void)d; (void)scale; (void)causal; (void)workspace;
+  (void)workspace_bytes; (void)dtype; (void)stream;
+  return fail(FA_ERR_UNSUPPORTED, "backward not built yet");
+}
+
+int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k, int H, int d,
+                  float scale, int causal, int num_seqs, int total_q, int total_k,
+                  void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  g_last_error.clear();
+  (void)q; (void)k; (void)v; (void)o; (void)dout; (void)lse; (void)dq; (void)dk; (void)dv;
+  (void)cu_seqlens_q; (void)cu_seqlens_k; (void)max_seqlen_q; (void)max_seqlen_k; (void)H;
+  (void)d; (void)scale; (void)causal; (void)num_seqs; (void)total_q; (void)total_k;
+  (void)workspace; (void)workspace_bytes; (void)dtype; (void)stream;
+  return fail(FA_ERR_UNSUPPORTED, "backward not built yet");
+}
+
+int fa_get_device_status(void* stream) {
+  g_last_error.clear();
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t* sp = status_ptr();
+  if (sp == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, sp, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read status word");
+  if (word != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpy(sp, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+    if (word & kDevTimeout) return fail(FA_ERR_TIMEOUT, "a kernel wait timed out");
+  }
+  return FA_OK;
+}
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* fa_last_error(void) { return g_last_error.c_str(); }
+
+int fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+  g_last_error.clear();
+  uint32_t* sp = status_ptr();
+  if (sp == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(sp, (uint64_t)limit_us * 1000ull);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return fa_get_device_status(stream);
+}
+
+}  // extern "C"

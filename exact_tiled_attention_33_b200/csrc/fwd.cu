@@ -1,0 +1,41 @@
+// Forward kernel instantiations and launcher.
+#include "fwd_kernel.cuh"
+
+namespace fattn {
+
+int fwd_rows_per_cta() { return FwdCfg<128>::BM * FwdCfg<128>::QT; }
+
+template <int D, bool BF16>
+static LaunchResult launch_fwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                 const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
+                                 cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  auto kern = fa_fwd_kernel<D, BF16>;
+  static bool configured[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LaunchResult::kCudaError;
+  if (dev < 64 && !configured[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+      return LaunchResult::kCudaError;
+    configured[dev] = true;
+  }
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  return cudaGetLastError() == cudaSuccess ? LaunchResult::kOk : LaunchResult::kCudaError;
+}
+
+LaunchResult launch_fwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                        const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
+                        cudaStream_t stream) {
+  if (d == 128) {
+    return bf16 ? launch_fwd_t<128, true>(tmQ, tmK, tmV, p, grid, stream)
+                : launch_fwd_t<128, false>(tmQ, tmK, tmV, p, grid, stream);
+  }
+  if (d == 64) {
+    return bf16 ? launch_fwd_t<64, true>(tmQ, tmK, tmV, p, grid, stream)
+                : launch_fwd_t<64, false>(tmQ, tmK, tmV, p, grid, stream);
+  }
+  return LaunchResult::kUnsupported;
+}
+
+}  // namespace fattn

@@ -1,0 +1,128 @@
+/*
+ * fattn — exact scaled-dot-product attention, tile by tile with online softmax, for
+ * NVIDIA B200 (sm_100a).  Plain C ABI: device pointers, sizes, a CUDA stream handle.
+ *
+ * What is computed.  For every (batch, head) — or, for the varlen calls, every packed
+ * sequence and head — with queries Q [Lq, d], keys K [Lk, d] and values V [Lk, d]:
+ *
+ *     S = scale · Q Kᵀ,   P = softmax(S) over keys,   O = P V,
+ *     LSE_i = ln Σ_j exp(S_ij)          (natural log, scaled-score units)
+ *
+ * the "standard attention" of the page "FlashAttention-2的核心设计原理" (yunthe.com),
+ * section "FlashAttention-2与标准注意力的计算对比", evaluated exactly but tile by tile
+ * with a running row maximum and a rescaled running sum (page
+ * "FlashAttention实战：如何在A100上实现3倍加速的Transformer训练" §3.1), so that the
+ * N×N score matrix is never stored.  The backward calls recompute P from Q, K and the
+ * saved LSE (page "Flash Attention V3：大模型训练加速与显存优化技术解析" §3.2).
+ *
+ * Causal masking (flag `causal`): key j is allowed for query i iff j <= i + (Lk - Lq)
+ * (bottom-right alignment; the usual lower triangle when Lq == Lk).  A query row with no
+ * allowed key gets O = 0, LSE = +inf and contributes nothing to any gradient.
+ *
+ * Layouts (all contiguous, head_dim innermost):
+ *   dense  q, k, v, o, dout, dq, dk, dv : [B, N, H, d]   (the pages' [batch, seqlen,
+ *          heads, head_dim], "FlashAttention-2的核心设计原理" section
+ *          "FlashAttention-2反向传播与多GPU训练")
+ *   dense  lse                         : [B, H, N] float32
+ *   varlen q, o, dout, dq              : [total_q, H, d];  k, v, dk, dv : [total_k, H, d]
+ *   varlen lse                         : [H, total_q] float32
+ *   cu_seqlens_q / cu_seqlens_k        : device int32 [num_seqs + 1], cu[0] = 0,
+ *          non-decreasing, cu[num_seqs] = total (section
+ *          "变长序列处理与flash_attn_varlen_func" of the same page)
+ * Element type of q/k/v/o/dout/dq/dk/dv: FA_BF16 or FA_FP16 (all the same); every MMA
+ * accumulates in fp32; 16-bit results are rounded to nearest-even.
+ * head_dim d must be 64 or 128.  Every device pointer must be 16-byte aligned.
+ *
+ * Ownership.  The caller allocates and owns every buffer.  The library allocates no
+ * device memory.  The backward calls take a caller-provided workspace sized by
+ * fa_bwd_workspace_size / fa_varlen_bwd_workspace_size.  The library keeps one device
+ * status word per GPU (see fa_get_device_status).
+ *
+ * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream):
+ * they validate, launch and return.  Validation failures return a non-zero status,
+ * launch nothing and leave every output untouched.  A device-side bounded wait that
+ * runs out (a pipeline that stopped making progress) is reported later by
+ * fa_get_device_status; the kernel then finishes without hanging the GPU and its
+ * outputs are undefined.
+ */
+#ifndef FATTN_H_
+#define FATTN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad cu_seqlens count */
+  FA_ERR_UNSUPPORTED = 2, /* head_dim other than 64/128, unknown dtype, size limits */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (see fa_last_error) */
+  FA_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (fa_get_device_status) */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/* Dense forward.  Writes o [B,N,H,d] and lse [B,H,N].
+ * Sizes: B, N, H >= 0 (a zero size is a no-op), B*N < 2^31, H < 2^16.
+ * scale: any finite float (the pages use 1/sqrt(d)). */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N,
+           int H, int d, float scale, int causal, int dtype, void* stream);
+
+/* Varlen forward over packed sequences (flash_attn_varlen_func semantics).
+ * Writes o [total_q,H,d] and lse [H,total_q].
+ * max_seqlen_q / max_seqlen_k must be >= every sequence's length (they size the grid);
+ * num_seqs, total_q, total_k are the host-side counts matching cu_seqlens (the host
+ * cannot read device cu_seqlens without a synchronisation). */
+int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int max_seqlen_q,
+                  int max_seqlen_k, int H, int d, float scale, int causal, int num_seqs,
+                  int total_q, int total_k, int dtype, void* stream);
+
+/* Workspace bytes the dense backward needs: an fp32 dQ accumulator [B,N,H,d] and
+ * D = rowsum(dO ∘ O) [B,H,N] fp32, each 256-byte aligned. */
+size_t fa_bwd_workspace_size(int B, int N, int H, int d);
+
+/* Dense backward: recomputes P from q, k and lse (as written by fa_fwd with the same
+ * scale and causal flag) and writes dq, dk, dv [B,N,H,d].
+ * o and dout are [B,N,H,d]; workspace must hold fa_bwd_workspace_size bytes and be
+ * 256-byte aligned; its contents on entry do not matter. */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d,
+           float scale, int causal, void* workspace, size_t workspace_bytes, int dtype,
+           void* stream);
+
+/* Workspace bytes the varlen backward needs (fp32 dQ accumulator [total_q,H,d] and D
+ * [H,total_q]). */
+size_t fa_varlen_bwd_workspace_size(int total_q, int H, int d);
+
+/* Varlen backward; arguments as fa_varlen_fwd plus the gradient buffers. */
+int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k, int H, int d,
+                  float scale, int causal, int num_seqs, int total_q, int total_k,
+                  void* workspace, size_t workspace_bytes, int dtype, void* stream);
+
+/* Synchronises `stream`, returns FA_ERR_TIMEOUT if any kernel of this library on the
+ * current device recorded a timed-out wait since the last call (FA_OK otherwise), and
+ * clears the status word.  FA_ERR_CUDA if the synchronisation itself failed. */
+int fa_get_device_status(void* stream);
+
+/* Static description of a status code. */
+const char* fa_status_string(int status);
+
+/* Detail of the most recent failure on the calling host thread ("" if none). */
+const char* fa_last_error(void);
+
+/* Runs a one-CTA kernel whose only wait can never complete, with the given bound in
+ * microseconds; used to test the timeout path without any tensor-core or TMA work in
+ * flight.  Returns the status fa_get_device_status reports afterwards (FA_ERR_TIMEOUT
+ * when the bounded wait works). */
+int fa_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FATTN_H_ */

@@ -1,0 +1,75 @@
+"""Shared helpers for the GPU-vs-oracle parity tests (test code only).
+
+Tolerances are the ones the target fixes for 16-bit inputs with fp32 accumulation:
+  max |O - O_ref| <= 1e-2, max |LSE - LSE_ref| <= 1e-3,
+  max |dX - dX_ref| <= 2e-2 * max |dX_ref| for dX in dQ, dK, dV.
+For O one documented reading applies: the output is stored in 16 bits, and where |O|
+is large (the peaky Q,K x4 workload reaches |O| ~ 5) a correctly rounded 16-bit value
+can sit up to half a 16-bit ulp from the fp64 value, which alone can exceed 1e-2.  The
+check therefore allows 1e-2 plus half an ulp of the output format at O_ref; the literal
+maximum error is reported next to it.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+O_TOL = 1e-2
+LSE_TOL = 1e-3
+GRAD_REL_TOL = 2e-2
+
+
+def half_ulp(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Half the spacing of 16-bit floats at |x| (bf16: 8 significant bits, fp16: 11)."""
+    mant = 8 if dtype == "bf16" else 11
+    ax = np.maximum(np.abs(x), 2.0 ** -14)
+    e = np.floor(np.log2(ax))
+    return 0.5 * 2.0 ** (e - (mant - 1))
+
+
+def check_o(o_gpu: np.ndarray, o_ref: np.ndarray, dtype: str, what: str = "O") -> float:
+    err = np.abs(o_gpu.astype(np.float64) - o_ref)
+    assert np.all(np.isfinite(o_gpu)), f"{what}: non-finite output"
+    allowed = O_TOL + half_ulp(o_ref, dtype)
+    bad = err > allowed
+    assert not bad.any(), (f"{what}: {int(bad.sum())} elements over tolerance; max err "
+                           f"{err.max():.4g}")
+    return float(err.max()) if err.size else 0.0
+
+
+def check_lse(lse_gpu: np.ndarray, lse_ref: np.ndarray, what: str = "LSE") -> float:
+    inf_ref = np.isposinf(lse_ref)
+    assert np.array_equal(np.isposinf(lse_gpu), inf_ref), f"{what}: +inf pattern differs"
+    fin = ~inf_ref
+    if not fin.any():
+        return 0.0
+    err = np.abs(lse_gpu[fin].astype(np.float64) - lse_ref[fin])
+    assert np.all(np.isfinite(lse_gpu[fin])), f"{what}: non-finite values"
+    assert err.max() <= LSE_TOL, f"{what}: max err {err.max():.4g}"
+    return float(err.max())
+
+
+def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, scale_ref=None) -> float:
+    ref_max = np.abs(g_ref).max() if scale_ref is None else scale_ref
+    err = np.abs(g_gpu.astype(np.float64) - g_ref)
+    assert np.all(np.isfinite(g_gpu)), f"{what}: non-finite gradient"
+    tol = GRAD_REL_TOL * max(ref_max, 1e-30)
+    assert err.max() <= tol, f"{what}: max err {err.max():.4g} > {tol:.4g}"
+    return float(err.max() / max(ref_max, 1e-30))
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def guarded_empty(shape, dtype, device, fill=float("nan"), guard=4096):
+    """A tensor view followed by a guard region (filled) to catch out-of-bounds writes."""
+    n = int(np.prod(shape)) if len(shape) else 1
+    buf = torch.full((n + guard,), fill, dtype=dtype, device=device)
+    return buf[:n].view(shape), buf
+
+
+def guard_intact(buf: torch.Tensor, n: int) -> bool:
+    g = buf[n:].float()
+    return bool(torch.isnan(g).all().item())

@@ -1,0 +1,95 @@
+"""CPU checks of the C ABI boundary: the library loads, exports every entry point the
+header declares, and rejects bad arguments on the host (no GPU work is started: every
+call here fails validation or is a no-op before any CUDA call)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_tiled_attention_33_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fattn.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _lib.load()
+
+
+def test_header_declares_expected_calls():
+    names = declared_symbols()
+    for n in ("fa_fwd", "fa_varlen_fwd", "fa_bwd", "fa_varlen_bwd", "fa_bwd_workspace_size",
+              "fa_get_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(declared_symbols()) == set(_lib.SIGNATURES)
+
+
+def test_status_strings(lib):
+    assert lib.fa_status_string(0) == b"ok"
+    assert lib.fa_status_string(4) == b"device wait timed out"
+    assert lib.fa_status_string(99) == b"unknown status"
+
+
+def test_workspace_sizes(lib):
+    B, N, H, d = 2, 16384, 32, 128
+    e = B * N * H * d
+    assert lib.fa_bwd_workspace_size(B, N, H, d) == e * 4 + B * H * N * 4
+    assert lib.fa_bwd_workspace_size(1, 3, 1, 64) == 768 + 256
+    assert lib.fa_bwd_workspace_size(0, 3, 1, 64) == 0
+    assert lib.fa_varlen_bwd_workspace_size(896, 32, 128) == 896 * 32 * 128 * 4 + 896 * 32 * 4
+
+
+P = ctypes.c_void_p(4096)  # a 16-byte aligned fake address; validation fails before any use
+
+
+def test_rejects_bad_head_dim(lib):
+    assert lib.fa_fwd(P, P, P, P, P, 1, 128, 1, 96, 0.1, 0, 0, None) == _lib.FA_ERR_UNSUPPORTED
+    assert b"head_dim" in lib.fa_last_error()
+
+
+def test_rejects_bad_dtype_and_scale(lib):
+    assert lib.fa_fwd(P, P, P, P, P, 1, 128, 1, 64, 0.1, 0, 7, None) == _lib.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd(P, P, P, P, P, 1, 128, 1, 64, float("nan"), 0, 0, None) == \
+        _lib.FA_ERR_INVALID_ARG
+
+
+def test_rejects_null_and_misaligned(lib):
+    assert lib.fa_fwd(None, P, P, P, P, 1, 128, 1, 64, 0.1, 0, 0, None) == _lib.FA_ERR_INVALID_ARG
+    mis = ctypes.c_void_p(4096 + 8)
+    assert lib.fa_fwd(P, mis, P, P, P, 1, 128, 1, 64, 0.1, 0, 0, None) == _lib.FA_ERR_INVALID_ARG
+    assert b"aligned" in lib.fa_last_error()
+
+
+def test_rejects_negative_sizes(lib):
+    assert lib.fa_fwd(P, P, P, P, P, -1, 128, 1, 64, 0.1, 0, 0, None) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_varlen_fwd(P, P, P, P, P, P, P, 10, 10, 1, 64, 0.1, 0, -2, 10, 10, 0, None) == \
+        _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_varlen_fwd(P, P, P, P, P, P, P, 20, 10, 1, 64, 0.1, 0, 1, 10, 10, 0, None) == \
+        _lib.FA_ERR_INVALID_ARG
+
+
+def test_size_limits(lib):
+    assert lib.fa_fwd(P, P, P, P, P, 70000, 70000, 1, 64, 0.1, 0, 0, None) == \
+        _lib.FA_ERR_UNSUPPORTED
+
+
+def test_empty_problems_are_noops(lib):
+    # zero-size problems return OK without touching (null) pointers or the GPU
+    assert lib.fa_fwd(None, None, None, None, None, 0, 128, 1, 64, 0.1, 0, 0, None) == _lib.FA_OK
+    assert lib.fa_fwd(None, None, None, None, None, 1, 0, 1, 64, 0.1, 1, 1, None) == _lib.FA_OK
+    assert lib.fa_varlen_fwd(None, None, None, None, None, None, None, 0, 0, 1, 64, 0.1, 0, 0, 0,
+                             0, 0, None) == _lib.FA_OK
