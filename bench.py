@@ -1,0 +1,389 @@
+"""Benchmark: exact tiled attention forward + backward on one B200 per rank.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fattn|reference]
+                    [--workload long_causal]
+
+One step = the whole hot path once over one batch: fa_fwd (O, LSE) then fa_bwd
+(D preprocess, dK/dV/dQ main kernel, dQ conversion) on the long-context workload
+(B=2, H=32, N=16384, d=128, bf16, causal, seeded N(0,1) inputs).  Throughput is
+attention TFLOPS with 4·B·H·N²·d forward FLOPs (halved when causal) and 2.5x that for
+the backward pass.  Multi-GPU (torchrun) runs one independent problem per rank (heads /
+batches are independent: no collective on the data path, weak scaling); time is the max
+over ranks of CUDA-event time.
+
+--impl reference times the CPU fp64 oracle (the only reference this build has) on a
+bounded sample of the same workload: the last R query rows of one head against all keys,
+which under the bottom-right causal reading is exactly those rows' share of the problem.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOPS (fwd, fwd+bwd) and % of B200 BF16 tensor peak, N=1K–16K"
+UNIT = "TFLOPS"
+FALLBACK_PEAK_TFLOPS = 1590.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
+BWD_SOURCES = ["exact_tiled_attention_33_b200/csrc/bwd_kernel.cuh",
+               "exact_tiled_attention_33_b200/csrc/sm100.cuh"]
+FWD_SOURCES = ["exact_tiled_attention_33_b200/csrc/fwd_kernel.cuh",
+               "exact_tiled_attention_33_b200/csrc/sm100.cuh"]
+
+
+# ------------------------------------------------------------------ helpers (CPU-testable)
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """Max of a per-rank float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput_tflops(flops_per_step_per_rank: float, steps: int, world: int,
+                      max_seconds: float) -> float:
+    """Whole-job throughput: all ranks' work divided by the slowest rank's time."""
+    return flops_per_step_per_rank * steps * world / max_seconds / 1e12
+
+
+def sources_sha(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kernel: str, workload: str, sha: str):
+    """DRAM bytes per launch recorded from an ncu capture, if it matches this source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    for line in open(TRAFFIC_FILE):
+        f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+        if f.get("kernel") == kernel and f.get("workload") == workload and \
+                f.get("source_sha") == sha:
+            return float(f["bytes_per_launch"])
+    return None
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), d.get("hbm_gbs"), "measured"
+    return FALLBACK_PEAK_TFLOPS, 1400.0, 6650.0, "fallback"
+
+
+REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            q = ("index,clocks.sm,clocks.max.sm,power.draw," +
+                 ",".join(f"clocks_event_reasons.{r}" for r in REASONS))
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(gpu_index)], stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 4 + len(REASONS):
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        active = sorted({REASONS[i] for r in rows for i in range(len(REASONS))
+                         if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": active, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ oracle timing
+_HEAD_CACHE = {}
+
+def oracle_sample_seconds(w, rows: int, head=(0, 0)):
+    """Run the fp64 oracle forward + backward for the last `rows` query rows of one head
+    against all keys; return (seconds, metric FLOPs of that share, threads)."""
+    import numpy as np
+    import oracle
+    from exact_tiled_attention_33_b200 import workloads as wl
+    key = (w.name, w.seed, head)
+    if key not in _HEAD_CACHE:
+        t = wl.generate(w)
+        b, h = head
+        _HEAD_CACHE[key] = tuple(wl.to_f64(t[x][b, :, h].clone()) for x in ("q", "k", "v", "do"))
+    q, k, v, do = _HEAD_CACHE[key]
+    N = q.shape[0]
+    r0 = N - rows
+    t0 = time.perf_counter()
+    oracle.attention_forward(q[r0:], k, v, w.softmax_scale, w.causal)
+    oracle.attention_backward(q[r0:], k, v, do[r0:], w.softmax_scale, w.causal)
+    dt = time.perf_counter() - t0
+    keys = np.arange(r0, N) + 1 if w.causal else np.full(rows, N)
+    flops = 3.5 * 4.0 * float(keys.sum()) * w.d
+    threads = os.cpu_count()
+    return dt, flops, threads
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    # size the per-step sample so a step takes about a second on this host
+    rows = 64
+    dt, _, _ = oracle_sample_seconds(w, rows)
+    while dt < 0.5 and rows < w.N:
+        rows = min(w.N, rows * 2)
+        dt, _, _ = oracle_sample_seconds(w, rows)
+    for _ in range(args.warmup):
+        oracle_sample_seconds(w, rows)
+    total_t, total_f = 0.0, 0.0
+    threads = os.cpu_count()
+    for _ in range(args.steps):
+        dt, fl, threads = oracle_sample_seconds(w, rows)
+        total_t += dt
+        total_f += fl
+    value = total_f / total_t / 1e12
+    sample = (f"last {rows} query rows of head (b=0,h=0) of {w.name} against all "
+              f"{w.N} keys, fp64 oracle fwd+bwd, per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(w.describe(), parallelism=f"dp{world}"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_fattn(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from exact_tiled_attention_33_b200 import _lib
+    from exact_tiled_attention_33_b200 import attention as fa
+    from exact_tiled_attention_33_b200 import workloads as wl
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    lib = _lib.load()
+    # each rank owns an independent problem of the same size (its own seed)
+    wr = wl.Workload(**{**w.__dict__, "seed": w.seed + rank})
+    host = wl.generate(wr)
+    B, N, H, d = wr.B, wr.N, wr.H, wr.d
+    scale, causal = wr.softmax_scale, int(wr.causal)
+    dtype = _lib.FA_BF16 if wr.dtype == "bf16" else _lib.FA_FP16
+    q, k, v, do = (host[x].to(dev) for x in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = fa.bwd_workspace(B, N, H, d, dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+
+    def step():
+        _lib.check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), B, N, H, d, scale, causal, dtype, sh), "fa_fwd")
+        _lib.check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                              dv.data_ptr(), B, N, H, d, scale, causal, ws.data_ptr(),
+                              ws.numel(), dtype, sh), "fa_bwd")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert lib.fa_get_device_status(sh) == 0, "device status after warm-up"
+
+    # ---- timed region: inputs (268 MB per tensor) are larger than the 126 MB L2
+    sampler = ClockSampler(local) if rank == 0 else None
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        _lib.check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), B, N, H, d, scale, causal, dtype, sh), "fa_fwd")
+        ev[i][1].record(stream)
+        _lib.check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                              dv.data_ptr(), B, N, H, d, scale, causal, ws.data_ptr(),
+                              ws.numel(), dtype, sh), "fa_bwd")
+        ev[i][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler is not None else None
+    status = lib.fa_get_device_status(sh)
+    assert status == 0, f"device status {status} in timed region"
+    total_ms = t_start.elapsed_time(t_end)
+    fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    bwd_ms = [b.elapsed_time(c) for _, b, c in ev]
+    max_s = max_over_ranks(total_ms / 1e3, world)
+    f_fwd = wr.fwd_flops()
+    f_step = 3.5 * f_fwd
+    value = throughput_tflops(f_step, args.steps, world, max_s)
+    fwd_avg = statistics.mean(fwd_ms)
+    bwd_avg = statistics.mean(bwd_ms)
+
+    # ---- end to end through the C ABI with pinned host buffers (per step: H2D of q, k,
+    # v, dO; fwd; bwd; D2H of O, LSE, dQ, dK, dV)
+    e2e = None
+    if not args.no_e2e:
+        hin = [host[x].pin_memory() for x in ("q", "k", "v", "do")]
+        hout = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (o, lse, dq, dk, dv)]
+        h2d = sum(x.numel() * x.element_size() for x in hin)
+        d2h = sum(x.numel() * x.element_size() for x in hout)
+        e2e_steps = max(2, min(args.steps, 5))
+
+        def e2e_step():
+            for hsrc, ddst in zip(hin, (q, k, v, do)):
+                ddst.copy_(hsrc, non_blocking=True)
+            step()
+            for dsrc, hdst in zip((o, lse, dq, dk, dv), hout):
+                hdst.copy_(dsrc, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_s = max_over_ranks(a.elapsed_time(b) / 1e3, world)
+        e2e = {"value": throughput_tflops(f_step, e2e_steps, world, e2e_s), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    peak_burst, peak_sust, hbm, peak_src = load_peaks()
+    bwd_sha = sources_sha(BWD_SOURCES)
+    fwd_sha = sources_sha(FWD_SOURCES)
+    bwd_ach = 2.5 * f_fwd / (bwd_avg / 1e3) / 1e12
+    fwd_ach = f_fwd / (fwd_avg / 1e3) / 1e12
+    roofline = {
+        "kernel": "fa_bwd_kernel (timed with its D preprocess and dQ conversion launches)",
+        "bound": "tensor", "achieved": bwd_ach, "peak": peak_sust, "unit": "TFLOP/s",
+        "frac": bwd_ach / peak_sust,
+        "peak_source": f"bf16_tflops_sustained ({peak_src})",
+        "traffic": read_traffic("fa_bwd_kernel", wr.name, bwd_sha),
+        "flops_per_launch": 2.5 * f_fwd}
+    fwd_roof = {"kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": fwd_ach,
+                "peak": peak_sust, "unit": "TFLOP/s", "frac": fwd_ach / peak_sust,
+                "frac_of_burst_peak": fwd_ach / peak_burst,
+                "traffic": read_traffic("fa_fwd_kernel", wr.name, fwd_sha),
+                "flops_per_launch": f_fwd}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = 512
+        dt, fl, threads = oracle_sample_seconds(wr, rows)
+        # grow the sample toward ~10 s of CPU work
+        while dt < 5.0 and rows < wr.N:
+            rows = min(wr.N, rows * 2)
+            dt, fl, threads = oracle_sample_seconds(wr, rows)
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"last {rows} query rows of head (b=0,h=0) against all {wr.N} keys, "
+                         f"fp64 oracle fwd+bwd ({dt:.1f} s)"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * max_s / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": wr.dtype, "data": "synthetic",
+                "config": dict(wr.describe(), seed=w.seed, parallelism=f"dp{world}",
+                               l2="inputs larger than L2 (268 MB per tensor), no flush"),
+                "fwd_tflops": f_fwd / (fwd_avg / 1e3) / 1e12,
+                "bwd_tflops": bwd_ach,
+                "pct_of_bf16_peak": {"fwd_bwd": value / world / peak_burst,
+                                     "fwd": fwd_ach / peak_burst,
+                                     "peak_tflops": peak_burst, "peak_source": peak_src},
+                "ms_fwd": fwd_avg, "ms_bwd": bwd_avg,
+                "gpu_launches": 4 * args.steps,
+                "roofline": roofline, "roofline_fwd": fwd_roof,
+                "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="fattn", choices=["fattn", "reference"])
+    ap.add_argument("--workload", default="long_causal")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3) if args.impl == "fattn" else args.warmup
+    from exact_tiled_attention_33_b200 import workloads as wl
+    w = wl.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_fattn(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

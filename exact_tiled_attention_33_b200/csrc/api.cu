@@ -105,6 +105,18 @@ int launch_result(LaunchResult r) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// The forward kernel works with a positive log2-domain factor c: a negative scale is
+// applied by negating Q in the S product, and scale == 0 uses a factor so small that
+// every finite score maps to x = 0 exactly in fp32 (uniform weights) while masked
+// scores (-inf) stay -inf.
+void set_fwd_scale(FwdParams& p, float scale) {
+  p.negate_scores = scale < 0.f ? 1 : 0;
+  const float c = std::fabs(scale) * kLog2e;
+  p.scale_log2 = c > 1e-30f ? c : 1e-30f;
+}
+
 }  // namespace
 
 // Bounded-wait self test: waits on a barrier that nothing arrives at.
@@ -147,7 +159,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.H = H;
   p.total_q = B * N;
   p.scale = scale;
-  p.scale_log2 = scale * kLog2e;
+  set_fwd_scale(p, scale);
   p.causal = causal ? 1 : 0;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
@@ -188,7 +200,7 @@ int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* l
   p.H = H;
   p.total_q = total_q;
   p.scale = scale;
-  p.scale_log2 = scale * kLog2e;
+  set_fwd_scale(p, scale);
   p.causal = causal ? 1 : 0;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
@@ -196,8 +208,6 @@ int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* l
   dim3 grid((max_seqlen_q + rows - 1) / rows, H, num_seqs);
   return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
 }
-
-static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t fa_bwd_workspace_size(int B, int N, int H, int d) {
   if (B <= 0 || N <= 0 || H <= 0 || d <= 0) return 0;
@@ -211,14 +221,59 @@ size_t fa_varlen_bwd_workspace_size(int total_q, int H, int d) {
   return align256(e * 4) + align256((size_t)H * total_q * 4);
 }
 
+namespace {
+
+// Shared validation and launch for both backward entry points.
+int bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dout,
+               const float* lse, void* dq, void* dk, void* dv, const int* cu_q, const int* cu_k,
+               int H, int d, float scale, int causal, long long q_rows, long long k_rows, int N,
+               int batches, int max_seqlen_k, int total_q, int total_k, void* workspace,
+               size_t workspace_bytes, size_t need, int dtype, cudaStream_t stream) {
+  if (int e = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv, workspace})) return e;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (workspace_bytes < need)
+    return fail(FA_ERR_INVALID_ARG, "workspace too small (need " + std::to_string(need) + " bytes)");
+  CUtensorMap mq, mk, mv, mdo;
+  const long long qb = cu_q ? 1 : batches, kb = cu_q ? 1 : batches;
+  const long long qr = cu_q ? q_rows : N, kr = cu_q ? k_rows : N;
+  if (int e = make_map(&mq, q, d, H, qr, qb, 128)) return e;
+  if (int e = make_map(&mdo, dout, d, H, qr, qb, 128)) return e;
+  if (int e = make_map(&mk, k, d, H, kr, kb, 128)) return e;
+  if (int e = make_map(&mv, v, d, H, kr, kb, 128)) return e;
+  BwdParams p{};
+  p.q = q; p.k = k; p.v = v; p.o = o; p.dout = dout; p.lse = lse;
+  p.dq = dq; p.dk = dk; p.dv = dv;
+  const size_t e = (size_t)q_rows * H * d;
+  p.dq_acc = static_cast<float*>(workspace);
+  p.dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(e * 4));
+  p.cu_q = cu_q; p.cu_k = cu_k;
+  p.B = cu_q ? 1 : batches; p.N = N; p.H = H;
+  p.total_q = total_q; p.total_k = total_k;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.causal = causal ? 1 : 0;
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  return launch_result(launch_bwd(d, dtype == FA_BF16, mq, mk, mv, mdo, p, q_rows, max_seqlen_k,
+                                  batches, stream));
+}
+
+}  // namespace
+
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
            const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d, float scale,
            int causal, void* workspace, size_t workspace_bytes, int dtype, void* stream) {
   g_last_error.clear();
-  (void)q; (void)k; (void)v; (void)o; (void)dout; (void)lse; (void)dq; (void)dk; (void)dv;
-  (void)B; (void)N; (void)H; (void)d; (void)scale; (void)causal; (void)workspace;
-  (void)workspace_bytes; (void)dtype; (void)stream;
-  return fail(FA_ERR_UNSUPPORTED, "backward not built yet");
+  if (int e = check_common(H, d, dtype, scale)) return e;
+  if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
+  if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
+  if (B == 0 || N == 0 || H == 0) return FA_OK;
+  if (B > 65535) return fail(FA_ERR_UNSUPPORTED, "B must be <= 65535");
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, nullptr, nullptr, H, d, scale, causal,
+                    (long long)B * N, (long long)B * N, N, B, N, B * N, B * N, workspace,
+                    workspace_bytes, fa_bwd_workspace_size(B, N, H, d), dtype,
+                    (cudaStream_t)stream);
 }
 
 int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -227,11 +282,27 @@ int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, co
                   float scale, int causal, int num_seqs, int total_q, int total_k,
                   void* workspace, size_t workspace_bytes, int dtype, void* stream) {
   g_last_error.clear();
-  (void)q; (void)k; (void)v; (void)o; (void)dout; (void)lse; (void)dq; (void)dk; (void)dv;
-  (void)cu_seqlens_q; (void)cu_seqlens_k; (void)max_seqlen_q; (void)max_seqlen_k; (void)H;
-  (void)d; (void)scale; (void)causal; (void)num_seqs; (void)total_q; (void)total_k;
-  (void)workspace; (void)workspace_bytes; (void)dtype; (void)stream;
-  return fail(FA_ERR_UNSUPPORTED, "backward not built yet");
+  if (int e = check_common(H, d, dtype, scale)) return e;
+  if (num_seqs < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
+    return fail(FA_ERR_INVALID_ARG, "sizes must be >= 0");
+  if (num_seqs > 65535) return fail(FA_ERR_UNSUPPORTED, "num_seqs must be <= 65535");
+  if (max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return fail(FA_ERR_INVALID_ARG, "max_seqlen exceeds the total token count");
+  if (num_seqs == 0 || H == 0 || (total_q == 0 && total_k == 0)) return FA_OK;
+  if (total_q == 0 || total_k == 0) {
+    // One side empty: every gradient that exists is zero.
+    if (int e = check_ptrs({total_q ? dq : dk})) return e;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t err = cudaSuccess;
+    if (total_q) err = cudaMemsetAsync(dq, 0, (size_t)total_q * H * d * 2, st);
+    if (total_k && err == cudaSuccess) err = cudaMemsetAsync(dk, 0, (size_t)total_k * H * d * 2, st);
+    if (total_k && err == cudaSuccess) err = cudaMemsetAsync(dv, 0, (size_t)total_k * H * d * 2, st);
+    return err == cudaSuccess ? FA_OK : cuda_fail(err, "cudaMemsetAsync");
+  }
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, H, d, scale,
+                    causal, total_q, total_k, 0, num_seqs, max_seqlen_k, total_q, total_k,
+                    workspace, workspace_bytes, fa_varlen_bwd_workspace_size(total_q, H, d),
+                    dtype, (cudaStream_t)stream);
 }
 
 int fa_get_device_status(void* stream) {
@@ -248,6 +319,8 @@ int fa_get_device_status(void* stream) {
     e = cudaMemcpy(sp, &zero, sizeof(zero), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(e, "clear status word");
     if (word & kDevTimeout) return fail(FA_ERR_TIMEOUT, "a kernel wait timed out");
+    if (word & kDevSmemAlign)
+      return fail(FA_ERR_UNSUPPORTED, "dynamic shared memory base not 1024-byte alignable");
   }
   return FA_OK;
 }

@@ -20,7 +20,8 @@ struct FwdParams {
   int H;
   int total_q;      // varlen: rows of q/o (row stride of lse)
   float scale;      // softmax scale
-  float scale_log2; // scale * log2(e)
+  float scale_log2; // |scale| * log2(e), > 0 (a tiny positive value when scale == 0)
+  int negate_scores;// 1 when scale < 0: the S product negates Q
   int causal;
   uint32_t* status; // device status word
 };
@@ -58,8 +59,10 @@ LaunchResult launch_fwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensor
 // Forward grid: x = query-tile pairs, y = heads, z = batch (dense) or sequences (varlen).
 int fwd_rows_per_cta();
 
+// Backward launch: preprocess, main kernel, dQ conversion.  q_rows = B*N (dense) or
+// total_q (varlen); grid z = batches (dense B, or varlen num_seqs).
 LaunchResult launch_bwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                         const CUtensorMap& tmV, const CUtensorMap& tmDO, const BwdParams& p,
-                        int max_seqlen_q, int max_seqlen_k, int num_seqs, cudaStream_t stream);
+                        long long q_rows, int max_seqlen_k, int batches, cudaStream_t stream);
 
 }  // namespace fattn

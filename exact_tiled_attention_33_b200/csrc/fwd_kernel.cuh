@@ -166,7 +166,8 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0 && n_kv > 0) {
       // S = Q Kᵀ: A = Q (K-major), B = K (K-major).  O += P V: A = P (tensor memory),
       // B = V stored [key][d], i.e. N-contiguous (MN-major).
-      constexpr uint32_t ID_S = idesc_f16_f32acc(BF16, BM, BN, false, false);
+      const uint32_t ID_S = idesc_f16_f32acc(BF16, BM, BN, false, false) |
+                            (p.negate_scores ? (1u << 13) : 0u);  // bit 13: negate A
       constexpr uint32_t ID_O = idesc_f16_f32acc(BF16, BM, D, false, true);
       auto issue_s = [&](int t, int s) {
         const uint32_t qa = sbase + C::OFF_Q + t * C::Q_TILE;
@@ -232,21 +233,21 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::tm_s(t);
     const uint32_t tO = tmem + lane_off + C::tm_o(t);
-    const float c = p.scale_log2;  // scores are handled as x = s * scale * log2(e)
+    const float c = p.scale_log2;  // > 0: scores are handled as x = s * scale * log2(e)
     float m = -INFINITY;           // reference maximum of x shared by l and O
-    float l = 0.f;
+    float l = 0.f;                 // Σ p (fp32), for the log-sum-exp
+    float l_r = 0.f;               // Σ of the 16-bit P actually multiplied into O
 
     for (int j = 0; j < n_kv; ++j) {
       mbar_wait(BAR(C::B_SFULL + t), (uint32_t)j & 1u, abort_flag, p.status);
       tc_fence_after();
-      // x = s * scale * log2(e), kept in place in the loaded registers.
+      // Raw scores s; the scaled, log2-domain score is x = s * c with c > 0 (a negative
+      // softmax scale is applied by negating Q inside the S product).
       uint32_t sr[128];
 #pragma unroll
       for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[q * 32]));
       tmem_wait_ld();
       reg_fence(sr);
-#pragma unroll
-      for (int e = 0; e < 128; ++e) sr[e] = __float_as_uint(__uint_as_float(sr[e]) * c);
 
       const int k0 = j * BN;
       const bool need_mask = (k0 + BN > Lk) || (p.causal && (k0 + BN - 1 > r0 + diag));
@@ -257,9 +258,16 @@ __global__ void __launch_bounds__(320, 1)
         for (int e = 0; e < 128; ++e)
           if (e >= lim) sr[e] = __float_as_uint(-INFINITY);
       }
-      float mx = __uint_as_float(sr[0]);
+      float mq[4];
 #pragma unroll
-      for (int e = 1; e < 128; ++e) mx = fmaxf(mx, __uint_as_float(sr[e]));
+      for (int q = 0; q < 4; ++q) {
+        float a = __uint_as_float(sr[q * 32]);
+#pragma unroll
+        for (int e = 1; e < 31; e += 2)
+          a = fmax3(a, __uint_as_float(sr[q * 32 + e]), __uint_as_float(sr[q * 32 + e + 1]));
+        mq[q] = fmaxf(a, __uint_as_float(sr[q * 32 + 31]));
+      }
+      const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * c;
 
       // Reference-maximum update.  Keep the stale maximum while the new one exceeds
       // it by at most 8 (a factor 2^8 in P, harmless in fp32 accumulators).
@@ -273,20 +281,34 @@ __global__ void __launch_bounds__(320, 1)
         rescale = true;
       }
       const float m_use = (m == -INFINITY) ? 0.f : m;
-      float rs = 0.f;
+      // p = 2^(s*c - m).  Two sums: l (exact fp32 p) gives the log-sum-exp; lr sums the
+      // 16-bit values the P·V product actually uses and normalises O, so numerator and
+      // denominator share the rounding of P (with the lazy maximum the largest P of a
+      // row is 2^δ, not exactly 1, and its rounding would otherwise bias the output).
+      const uint64_t c2 = f2_pack(c, c);
+      const uint64_t nm2 = f2_pack(-m_use, -m_use);
+      uint64_t ls2 = 0ull, lr2 = 0ull;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2_approx(__uint_as_float(sr[q * 32 + 2 * e]) - m_use);
-          const float p1 = ex2_approx(__uint_as_float(sr[q * 32 + 2 * e + 1]) - m_use);
-          rs += p0 + p1;
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[q * 32 + 2 * e]),
+                                             __uint_as_float(sr[q * 32 + 2 * e + 1])),
+                                     c2, nm2);
+          const float2 xx = f2_unpack(x2);
+          const float p0 = ex2_approx(xx.x);
+          const float p1 = ex2_approx(xx.y);
           pk[e] = pack2<BF16>(p0, p1);
+          const float2 pr = unpack2<BF16>(pk[e]);
+          ls2 = f2_add(ls2, f2_pack(p0, p1));
+          lr2 = f2_add(lr2, f2_pack(pr.x, pr.y));
         }
         tmem_st16(tS + q * 16, pk);
       }
-      l = l * alpha + rs;
+      const float2 ls = f2_unpack(ls2), lr = f2_unpack(lr2);
+      l = l * alpha + (ls.x + ls.y);
+      l_r = l_r * alpha + (lr.x + lr.y);
 
       if (__any_sync(0xffffffffu, rescale)) {
         // O_t was last written by the P·V product of tile j-1, which completed before
@@ -313,7 +335,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
     }
     const bool valid = i < Lq;
-    const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+    const float inv_l = (l_r > 0.f) ? 1.f / l_r : 0.f;
     using elem_t = uint16_t;
     elem_t* orow;
     if (p.cu_q != nullptr)

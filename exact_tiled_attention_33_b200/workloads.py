@@ -128,6 +128,10 @@ def _registry():
                      seed=4))
         add(Workload(f"long_peaky_{c}", B=2, H=32, N=16384, d=128, dtype="bf16",
                      causal=causal, seed=4, qk_mult=4.0))
+    # profiling size of the long-context kernel path: inputs larger than L2 (4 x 67 MB),
+    # about 1 GB on the device in total
+    add(Workload("profile_causal_8k", B=1, H=32, N=8192, d=128, dtype="bf16", causal=True,
+                 seed=4))
     return w
 
 

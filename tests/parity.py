@@ -50,13 +50,34 @@ def check_lse(lse_gpu: np.ndarray, lse_ref: np.ndarray, what: str = "LSE") -> fl
     return float(err.max())
 
 
-def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, scale_ref=None) -> float:
+def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, scale_ref=None,
+               extra=None) -> float:
+    """max |g - g_ref| <= 2e-2 * max|g_ref| (plus an optional per-element `extra`)."""
     ref_max = np.abs(g_ref).max() if scale_ref is None else scale_ref
     err = np.abs(g_gpu.astype(np.float64) - g_ref)
     assert np.all(np.isfinite(g_gpu)), f"{what}: non-finite gradient"
     tol = GRAD_REL_TOL * max(ref_max, 1e-30)
-    assert err.max() <= tol, f"{what}: max err {err.max():.4g} > {tol:.4g}"
+    allowed = tol if extra is None else tol + extra
+    over = err - allowed
+    assert over.max() <= 0, f"{what}: max err {err.max():.4g} > {tol:.4g} (+extra)"
     return float(err.max() / max(ref_max, 1e-30))
+
+
+def o16_term_in_d(q, k, v, do, scale, causal, dtype):
+    """First-order bound on what computing D = rowsum(dO ∘ O) from the 16-bit O (the only
+    O the backward pass receives) changes in dQ and dK, per element.
+
+    |δD_i| <= Σ_c |dO_ic| · ½ulp(O_ic);  δdS_ij = -P_ij δD_i, so
+    |δdQ_ic| <= scale |δD_i| Σ_j P_ij |K_jc|  and  |δdK_jc| <= scale Σ_i P_ij |δD_i| |Q_ic|.
+    Only significant for degenerate sizes (N <= 2) where the exact gradient nearly cancels.
+    """
+    import oracle
+    o, _ = oracle.attention_forward(q, k, v, scale, causal)
+    pm = oracle.softmax_probs(q, k, scale, causal)
+    dd = (np.abs(do) * half_ulp(o, dtype)).sum(axis=1)
+    bq = abs(scale) * dd[:, None] * (pm @ np.abs(k))
+    bk = abs(scale) * (pm * dd[:, None]).T @ np.abs(q)
+    return bq, bk
 
 
 def f64(t: torch.Tensor) -> np.ndarray:
