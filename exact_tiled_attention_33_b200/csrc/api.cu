@@ -1,12 +1,13 @@
 // C ABI of libfattn: argument validation, TMA tensor-map encoding, launches, status.
 // The operations are documented in include/fattn.h.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <string>
 
-#include "../../include/fattn.h"
+#include "fattn.h"
 #include "fattn_internal.h"
 #include "sm100.cuh"
 
@@ -97,6 +98,13 @@ int check_ptrs(std::initializer_list<const void*> ptrs) {
   return FA_OK;
 }
 
+// Grids are x = batches * H, y = 128-row tiles of the sequence.
+int check_grid(long long batches, long long H, long long max_len) {
+  if (batches * H >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "batch*heads must be < 2^31");
+  if (max_len > 65535LL * 128) return fail(FA_ERR_UNSUPPORTED, "sequence length must be <= 8388480");
+  return FA_OK;
+}
+
 int launch_result(LaunchResult r) {
   if (r == LaunchResult::kOk) return FA_OK;
   if (r == LaunchResult::kUnsupported) return fail(FA_ERR_UNSUPPORTED, "unsupported configuration");
@@ -145,7 +153,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
   if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
   if (B == 0 || N == 0 || H == 0) return FA_OK;
-  if (B > 65535) return fail(FA_ERR_UNSUPPORTED, "B must be <= 65535");
+  if (int e = check_grid(B, H, N)) return e;
   if (int e = check_ptrs({q, k, v, o, lse})) return e;
   CUtensorMap mq, mk, mv;
   if (int e = make_map(&mq, q, d, H, N, B, 128)) return e;
@@ -164,7 +172,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   const int rows = fwd_rows_per_cta();
-  dim3 grid((N + rows - 1) / rows, H, B);
+  dim3 grid((unsigned)(B * H), (N + rows - 1) / rows);
   return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
 }
 
@@ -180,6 +188,7 @@ int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* l
   if (max_seqlen_q > total_q || max_seqlen_k > total_k)
     return fail(FA_ERR_INVALID_ARG, "max_seqlen exceeds the total token count");
   if (num_seqs == 0 || total_q == 0 || H == 0 || max_seqlen_q == 0) return FA_OK;
+  if (int e = check_grid(num_seqs, H, std::max(max_seqlen_q, max_seqlen_k))) return e;
   if (int e = check_ptrs({q, o, lse, cu_seqlens_q, cu_seqlens_k})) return e;
   if (total_k > 0)
     if (int e = check_ptrs({k, v})) return e;
@@ -205,20 +214,18 @@ int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* l
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   const int rows = fwd_rows_per_cta();
-  dim3 grid((max_seqlen_q + rows - 1) / rows, H, num_seqs);
+  dim3 grid((unsigned)(num_seqs * H), (max_seqlen_q + rows - 1) / rows);
   return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int N, int H, int d) {
   if (B <= 0 || N <= 0 || H <= 0 || d <= 0) return 0;
-  const size_t e = (size_t)B * N * H * d;
-  return align256(e * 4) + align256((size_t)B * H * N * 4);
+  return align256((size_t)B * H * N * 4);
 }
 
 size_t fa_varlen_bwd_workspace_size(int total_q, int H, int d) {
   if (total_q <= 0 || H <= 0 || d <= 0) return 0;
-  const size_t e = (size_t)total_q * H * d;
-  return align256(e * 4) + align256((size_t)H * total_q * 4);
+  return align256((size_t)H * total_q * 4);
 }
 
 namespace {
@@ -227,7 +234,8 @@ namespace {
 int bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, const int* cu_q, const int* cu_k,
                int H, int d, float scale, int causal, long long q_rows, long long k_rows, int N,
-               int batches, int max_seqlen_k, int total_q, int total_k, void* workspace,
+               int batches, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+               void* workspace,
                size_t workspace_bytes, size_t need, int dtype, cudaStream_t stream) {
   if (int e = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv, workspace})) return e;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -244,9 +252,7 @@ int bwd_common(const void* q, const void* k, const void* v, const void* o, const
   BwdParams p{};
   p.q = q; p.k = k; p.v = v; p.o = o; p.dout = dout; p.lse = lse;
   p.dq = dq; p.dk = dk; p.dv = dv;
-  const size_t e = (size_t)q_rows * H * d;
-  p.dq_acc = static_cast<float*>(workspace);
-  p.dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(e * 4));
+  p.dvec = static_cast<float*>(workspace);
   p.cu_q = cu_q; p.cu_k = cu_k;
   p.B = cu_q ? 1 : batches; p.N = N; p.H = H;
   p.total_q = total_q; p.total_k = total_k;
@@ -255,8 +261,8 @@ int bwd_common(const void* q, const void* k, const void* v, const void* o, const
   p.causal = causal ? 1 : 0;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-  return launch_result(launch_bwd(d, dtype == FA_BF16, mq, mk, mv, mdo, p, q_rows, max_seqlen_k,
-                                  batches, stream));
+  return launch_result(launch_bwd(d, dtype == FA_BF16, mq, mk, mv, mdo, p, q_rows, max_seqlen_q,
+                                  max_seqlen_k, batches, stream));
 }
 
 }  // namespace
@@ -269,9 +275,9 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
   if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
   if (B == 0 || N == 0 || H == 0) return FA_OK;
-  if (B > 65535) return fail(FA_ERR_UNSUPPORTED, "B must be <= 65535");
+  if (int e = check_grid(B, H, N)) return e;
   return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, nullptr, nullptr, H, d, scale, causal,
-                    (long long)B * N, (long long)B * N, N, B, N, B * N, B * N, workspace,
+                    (long long)B * N, (long long)B * N, N, B, N, N, B * N, B * N, workspace,
                     workspace_bytes, fa_bwd_workspace_size(B, N, H, d), dtype,
                     (cudaStream_t)stream);
 }
@@ -299,8 +305,10 @@ int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, co
     if (total_k && err == cudaSuccess) err = cudaMemsetAsync(dv, 0, (size_t)total_k * H * d * 2, st);
     return err == cudaSuccess ? FA_OK : cuda_fail(err, "cudaMemsetAsync");
   }
+  if (int e = check_grid(num_seqs, H, std::max(max_seqlen_q, max_seqlen_k))) return e;
   return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, H, d, scale,
-                    causal, total_q, total_k, 0, num_seqs, max_seqlen_k, total_q, total_k,
+                    causal, total_q, total_k, 0, num_seqs, max_seqlen_q, max_seqlen_k, total_q,
+                    total_k,
                     workspace, workspace_bytes, fa_varlen_bwd_workspace_size(total_q, H, d),
                     dtype, (cudaStream_t)stream);
 }

@@ -1,5 +1,5 @@
-// Backward kernel instantiations and launcher: preprocess, main, dQ conversion, all on
-// the caller's stream.
+// Backward kernel instantiations and launcher: D preprocess, then the dK/dV pass and the
+// dQ pass, all on the caller's stream.
 #include <algorithm>
 
 #include "bwd_kernel.cuh"
@@ -9,8 +9,8 @@ namespace fattn {
 template <int D, bool BF16>
 static LaunchResult launch_bwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                  const CUtensorMap& tmV, const CUtensorMap& tmDO,
-                                 const BwdParams& p, long long q_rows, int max_seqlen_k,
-                                 int batches, cudaStream_t stream) {
+                                 const BwdParams& p, long long q_rows, int max_seqlen_q,
+                                 int max_seqlen_k, int batches, cudaStream_t stream) {
   using C = BwdCfg<D>;
   static bool configured[64] = {};
   int dev = 0;
@@ -18,35 +18,36 @@ static LaunchResult launch_bwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(fa_bwd_kernel<D, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(fa_bwd_dkdv_kernel<D, BF16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_A) != cudaSuccess ||
+        cudaFuncSetAttribute(fa_bwd_dq_kernel<D, BF16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B) != cudaSuccess)
       return LaunchResult::kCudaError;
     configured[dev] = true;
   }
-  // 1) D = rowsum(dO ∘ O), dQ accumulator = 0
+  // 1) D = rowsum(dO ∘ O)
   const long long warps = q_rows * p.H;
   const long long pre_blocks = std::min<long long>((warps + 7) / 8, (long long)sms * 16);
   fa_bwd_pre_kernel<D, BF16><<<(unsigned)pre_blocks, 256, 0, stream>>>(p, q_rows);
-  // 2) dK, dV and the dQ accumulator
-  dim3 grid((max_seqlen_k + C::BN - 1) / C::BN, p.H, batches);
-  fa_bwd_kernel<D, BF16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmDO, p);
-  // 3) dQ = scale · accumulator
-  const long long n8 = q_rows * p.H * D / 8;
-  const long long cv_blocks = std::min<long long>((n8 + 255) / 256, (long long)sms * 16);
-  fa_bwd_dq_kernel<BF16><<<(unsigned)cv_blocks, 256, 0, stream>>>(
-      p.dq_acc, reinterpret_cast<uint16_t*>(p.dq), n8, p.scale);
+  // 2) dK, dV: one CTA per key tile
+  dim3 grid_a((unsigned)(batches * p.H), (max_seqlen_k + C::BN - 1) / C::BN);
+  fa_bwd_dkdv_kernel<D, BF16><<<grid_a, C::THREADS, C::SMEM_A, stream>>>(tmQ, tmK, tmV, tmDO, p);
+  // 3) dQ: one CTA per query tile
+  dim3 grid_b((unsigned)(batches * p.H), (max_seqlen_q + C::BM - 1) / C::BM);
+  fa_bwd_dq_kernel<D, BF16><<<grid_b, C::THREADS, C::SMEM_B, stream>>>(tmQ, tmK, tmV, tmDO, p);
   return cudaGetLastError() == cudaSuccess ? LaunchResult::kOk : LaunchResult::kCudaError;
 }
 
 LaunchResult launch_bwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                         const CUtensorMap& tmV, const CUtensorMap& tmDO, const BwdParams& p,
-                        long long q_rows, int max_seqlen_k, int batches, cudaStream_t stream) {
+                        long long q_rows, int max_seqlen_q, int max_seqlen_k, int batches,
+                        cudaStream_t stream) {
   if (d == 128)
-    return bf16 ? launch_bwd_t<128, true>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream)
-                : launch_bwd_t<128, false>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream);
+    return bf16 ? launch_bwd_t<128, true>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_q, max_seqlen_k, batches, stream)
+                : launch_bwd_t<128, false>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_q, max_seqlen_k, batches, stream);
   if (d == 64)
-    return bf16 ? launch_bwd_t<64, true>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream)
-                : launch_bwd_t<64, false>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream);
+    return bf16 ? launch_bwd_t<64, true>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_q, max_seqlen_k, batches, stream)
+                : launch_bwd_t<64, false>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_q, max_seqlen_k, batches, stream);
   return LaunchResult::kUnsupported;
 }
 

@@ -10,18 +10,17 @@
 // the chain rule applied to the "standard attention" definition of the page
 // "FlashAttention-2的核心设计原理".
 //
-// Kernels:
-//   fa_bwd_pre_kernel   D = rowsum(dO ∘ O) (warp-shuffle reduction), dQ accumulator = 0
-//   fa_bwd_kernel       one CTA per 128-key tile: loops over the 128-row query tiles
-//                       that can see the tile; all five products on tcgen05
-//   fa_bwd_dq_kernel    dQ = scale · accumulator, rounded to 16 bits
-//
-// Main-kernel roles: warp 0 loads (TMA for K, V once and Q_i, dO_i per step; plain
-// loads for LSE_i, D_i), warp 1 issues tcgen05.mma, warps 2..5 ("compute") own one key
-// row each (tensor-memory lane) and form Pᵀ and dSᵀ, warps 6..9 ("dq") drain the dQ
-// tile from tensor memory into the fp32 accumulator with vector atomics.
-// Tensor memory: Sᵀ (Pᵀ aliased as packed 16-bit) | dPᵀ (dQ_i aliased after dSᵀ is
-// formed) | dK | dV.
+// Kernels (the "global gradients split into local updates" of the same page, read as
+// two independent passes so that no gradient is ever accumulated across CTAs):
+//   fa_bwd_pre_kernel   D = rowsum(dO ∘ O), one warp per row, warp-shuffle reduction
+//   fa_bwd_dkdv_kernel  one CTA per 128-key tile, looping over the query tiles that can
+//                       see it: Sᵀ = K Qᵀ, dPᵀ = V dOᵀ, dV += Pᵀ dO, dK += dSᵀ Q
+//   fa_bwd_dq_kernel    one CTA per 128-row query tile, looping over the key tiles it
+//                       can see: S = Q Kᵀ, dP = dO Vᵀ, dQ += dS K
+// P and dS are recomputed in both (7 products instead of 5) in exchange for no fp32
+// atomics at all: every output element is written exactly once, so dQ, dK and dV are
+// bitwise reproducible.  All products run on tcgen05 with fp32 accumulators in tensor
+// memory; P and dS re-enter the tensor core from tensor memory (packed 16-bit).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -64,7 +63,6 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p, long
         acc = fmaf(fa.x, fb.x, acc);
         acc = fmaf(fa.y, fb.y, acc);
       }
-      *reinterpret_cast<float4*>(p.dq_acc + base) = make_float4(0.f, 0.f, 0.f, 0.f);
     } else {
       const uint32_t a = *reinterpret_cast<const uint32_t*>(o);
       const uint32_t b = *reinterpret_cast<const uint32_t*>(g);
@@ -77,7 +75,6 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p, long
         fb = __half22float2(*reinterpret_cast<const __half2*>(&b));
       }
       acc = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, acc));
-      *reinterpret_cast<float2*>(p.dq_acc + base) = make_float2(0.f, 0.f);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -94,101 +91,86 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p, long
   }
 }
 
-// ------------------------------------------------------------------ dQ conversion
-template <bool BF16>
-__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ acc,
-                                                        uint16_t* __restrict__ dq, long long n8,
-                                                        float scale) {
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += stride) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
-    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
-    uint4 r;
-    r.x = pack2<BF16>(a.x * scale, a.y * scale);
-    r.y = pack2<BF16>(a.z * scale, a.w * scale);
-    r.z = pack2<BF16>(b.x * scale, b.y * scale);
-    r.w = pack2<BF16>(b.z * scale, b.w * scale);
-    reinterpret_cast<uint4*>(dq)[i] = r;
-  }
-}
-
-// ------------------------------------------------------------------ main kernel
+// ------------------------------------------------------------------ shared layout
 template <int D>
 struct BwdCfg {
-  static constexpr int BM = 128;  // query rows per step
-  static constexpr int BN = 128;  // keys per CTA = tensor-memory lanes
+  static constexpr int BM = 128;  // query rows per tile
+  static constexpr int BN = 128;  // keys per tile
   static constexpr int STAGES = 2;
   static constexpr int KCH = D / 64;
   static constexpr int CHUNK = 128 * 128;  // one 64-column chunk of a 128-row tile
   static constexpr int TILE = 128 * D * 2;
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + TILE;
-  static constexpr int OFF_Q = OFF_V + TILE;
-  static constexpr int OFF_DO = OFF_Q + STAGES * TILE;
-  static constexpr int OFF_DS = OFF_DO + STAGES * TILE;  // [key 128][query 128] 16-bit
-  static constexpr int OFF_VEC = OFF_DS + 2 * CHUNK;      // per stage: lse2[128], D[128]
-  static constexpr int OFF_BAR = OFF_VEC + STAGES * 2 * BM * 4;
-  static constexpr int B_KV = 0;
-  static constexpr int B_QFULL = 1;
-  static constexpr int B_QEMPTY = B_QFULL + STAGES;
-  static constexpr int B_SFULL = B_QEMPTY + STAGES;
-  static constexpr int B_DPFULL = B_SFULL + 1;
-  static constexpr int B_PFULL = B_DPFULL + 1;
-  static constexpr int B_DSFULL = B_PFULL + 1;
-  static constexpr int B_DSEMPTY = B_DSFULL + 1;
-  static constexpr int B_DQFULL = B_DSEMPTY + 1;
-  static constexpr int B_DQEMPTY = B_DQFULL + 1;
-  static constexpr int B_DONE = B_DQEMPTY + 1;
-  static constexpr int NBAR = B_DONE + 1;
-  static constexpr int USED = OFF_BAR + 8 * NBAR + 16;
-  static constexpr int SMEM_MAX = 232448;  // opt-in limit per CTA on sm_100
-  static constexpr int SLACK = (USED + 1024 <= SMEM_MAX) ? 1024 : (SMEM_MAX - USED) & ~15;
-  static constexpr int SMEM_BYTES = USED + SLACK;
-  static constexpr int THREADS = 320;
+  // dK/dV kernel: K, V resident; Q and dO streamed with per-tile vectors
+  static constexpr int A_OFF_K = 0;
+  static constexpr int A_OFF_V = A_OFF_K + TILE;
+  static constexpr int A_OFF_Q = A_OFF_V + TILE;
+  static constexpr int A_OFF_DO = A_OFF_Q + STAGES * TILE;
+  static constexpr int A_OFF_VEC = A_OFF_DO + STAGES * TILE;  // per stage: -lse*log2e, D
+  static constexpr int A_OFF_BAR = A_OFF_VEC + STAGES * 2 * BM * 4;
+  // dQ kernel: Q, dO resident; K and V streamed
+  static constexpr int B_OFF_Q = 0;
+  static constexpr int B_OFF_DO = B_OFF_Q + TILE;
+  static constexpr int B_OFF_K = B_OFF_DO + TILE;
+  static constexpr int B_OFF_V = B_OFF_K + STAGES * TILE;
+  static constexpr int B_OFF_BAR = B_OFF_V + STAGES * TILE;
+  static constexpr int NBAR = 16;
+  static constexpr int SMEM_A = A_OFF_BAR + 8 * NBAR + 16 + 1024;
+  static constexpr int SMEM_B = B_OFF_BAR + 8 * NBAR + 16 + 1024;
+  static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DK = 256, TM_DV = 256 + D;
+  // packed 16-bit operand column for K-elements 16*kk .. 16*kk+15 of a 128-wide row:
+  // half 0 (elements 0..63) packs into columns 0..31, half 1 into 64..95 of its region
+  __device__ static constexpr uint32_t packed_col(int kk) {
+    return (uint32_t)(kk * 8 + (kk >= 4 ? 32 : 0));
+  }
 };
 
+// Roles (12 warps): 0 loads, 1 issues MMAs, 2-3 idle, 4-7 and 8-11 are two compute
+// warpgroups, each owning half of the 128 columns of every score tile (one tensor-memory
+// lane = one row per thread).
+
+// ------------------------------------------------------------------ dK, dV
+// Tensor memory: Sᵀ [0,128) (Pᵀ packed into it) | dPᵀ [128,256) (dSᵀ packed into it) |
+// dK [256, 256+D) | dV [256+D, 256+2D).
+// Grid: x = (batch or sequence) * H + head, y = key tile (tile 0, which has the most
+// query tiles when causal, first for every head).
 template <int D, bool BF16>
-__global__ void __launch_bounds__(320, 1)
-    fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                  const BwdParams p) {
+__global__ void __launch_bounds__(384, 1)
+    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                       const BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int BM = C::BM, BN = C::BN, ST = C::STAGES;
+  constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DK = 256, TM_DV = 256 + D;
+  enum { B_KV = 0, B_QFULL = 1, B_QEMPTY = B_QFULL + ST, B_SFULL = B_QEMPTY + ST, B_DPFULL,
+         B_PFULL, B_DSFULL, B_DONE };
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
-  if (pad > (uint32_t)C::SLACK) {  // cannot place 1024-byte aligned tiles: report, do nothing
-    if (threadIdx.x == 0) atomicOr(p.status, kDevSmemAlign);
-    return;
-  }
-  const uint32_t sbase = raw + pad;
-  uint8_t* sgen = smem_raw + pad;
-  auto BAR = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * (uint32_t)i; };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + C::OFF_BAR + 8 * C::NBAR);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::A_OFF_BAR + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + C::A_OFF_BAR + 8 * C::NBAR);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---------------------------------------------------------------- work item
-  const int h = blockIdx.y;
+  const int h = blockIdx.x % p.H;
+  const int bz = blockIdx.x / p.H;
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
-    const int s = blockIdx.z;
-    q_row0 = p.cu_q[s];
-    Lq = p.cu_q[s + 1] - q_row0;
-    k_row0 = p.cu_k[s];
-    Lk = p.cu_k[s + 1] - k_row0;
+    q_row0 = p.cu_q[bz];
+    Lq = p.cu_q[bz + 1] - q_row0;
+    k_row0 = p.cu_k[bz];
+    Lk = p.cu_k[bz + 1] - k_row0;
     bcoord = 0;
   } else {
     q_row0 = k_row0 = 0;
     Lq = Lk = p.N;
-    bcoord = blockIdx.z;
+    bcoord = bz;
   }
-  const int k0 = blockIdx.x * BN;
+  const int k0 = blockIdx.y * BN;
   if (k0 >= Lk) return;
-  const int diag = Lk - Lq;
+  const int diag = Lk - Lq;  // key j is allowed for query i iff j <= i + diag (causal)
   const int q_tiles = (Lq + BM - 1) / BM;
   int i_begin = 0;
   if (p.causal) {
@@ -197,21 +179,17 @@ __global__ void __launch_bounds__(320, 1)
   }
   const int n_q = q_tiles > i_begin ? q_tiles - i_begin : 0;
 
-  // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
-    mbar_init(BAR(C::B_KV), 1);
+    mbar_init(BAR(B_KV), 1);
     for (int s = 0; s < ST; ++s) {
-      mbar_init(BAR(C::B_QFULL + s), 32);
-      mbar_init(BAR(C::B_QEMPTY + s), 1);
+      mbar_init(BAR(B_QFULL + s), 32);
+      mbar_init(BAR(B_QEMPTY + s), 1);
     }
-    mbar_init(BAR(C::B_SFULL), 1);
-    mbar_init(BAR(C::B_DPFULL), 1);
-    mbar_init(BAR(C::B_PFULL), 128);
-    mbar_init(BAR(C::B_DSFULL), 128);
-    mbar_init(BAR(C::B_DSEMPTY), 1);
-    mbar_init(BAR(C::B_DQFULL), 1);
-    mbar_init(BAR(C::B_DQEMPTY), 128);
-    mbar_init(BAR(C::B_DONE), 1);
+    mbar_init(BAR(B_SFULL), 1);
+    mbar_init(BAR(B_DPFULL), 1);
+    mbar_init(BAR(B_PFULL), 256);
+    mbar_init(BAR(B_DSFULL), 256);
+    mbar_init(BAR(B_DONE), 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
@@ -233,45 +211,44 @@ __global__ void __launch_bounds__(320, 1)
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmDO);
-        mbar_arrive_expect_tx(BAR(C::B_KV), 2 * C::TILE);
+        mbar_arrive_expect_tx(BAR(B_KV), 2 * C::TILE);
         for (int c = 0; c < C::KCH; ++c) {
-          tma_load_4d(&tmK, BAR(C::B_KV), sbase + C::OFF_K + c * C::CHUNK, c * 64, h, k_row0 + k0,
+          tma_load_4d(&tmK, BAR(B_KV), sbase + C::A_OFF_K + c * C::CHUNK, c * 64, h, k_row0 + k0,
                       bcoord);
-          tma_load_4d(&tmV, BAR(C::B_KV), sbase + C::OFF_V + c * C::CHUNK, c * 64, h, k_row0 + k0,
+          tma_load_4d(&tmV, BAR(B_KV), sbase + C::A_OFF_V + c * C::CHUNK, c * 64, h, k_row0 + k0,
                       bcoord);
         }
       }
       for (int it = 0; it < n_q; ++it) {
         const int s = it % ST;
         const int q0 = (i_begin + it) * BM;
-        mbar_wait(BAR(C::B_QEMPTY + s), ((uint32_t)(it / ST) & 1u) ^ 1u, abort_flag, p.status);
-        // LSE (as log2 units) and D for the 128 query rows of this step; rows past the
-        // sequence get LSE = +inf (P = 0) and D = 0.
-        float* vec = reinterpret_cast<float*>(sgen + C::OFF_VEC + s * 2 * BM * 4);
+        mbar_wait(BAR(B_QEMPTY + s), ((uint32_t)(it / ST) & 1u) ^ 1u, abort_flag, p.status);
+        // -LSE·log2(e) and D of the 128 query rows; rows past the sequence: -inf, 0.
+        float* vec = reinterpret_cast<float*>(sgen + C::A_OFF_VEC + s * 2 * BM * 4);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int qc = lane * 4 + e;
           const int qg = q0 + qc;
-          float l2 = INFINITY, dd = 0.f;
+          float nl2 = -INFINITY, dd = 0.f;
           if (qg < Lq) {
-            size_t vi = (p.cu_q != nullptr) ? (size_t)h * p.total_q + q_row0 + qg
-                                            : ((size_t)bcoord * p.H + h) * p.N + qg;
-            l2 = p.lse[vi] * kLog2e;
+            const size_t vi = (p.cu_q != nullptr) ? (size_t)h * p.total_q + q_row0 + qg
+                                                  : ((size_t)bcoord * p.H + h) * p.N + qg;
+            nl2 = -p.lse[vi] * kLog2e;
             dd = p.dvec[vi];
           }
-          vec[qc] = l2;
+          vec[qc] = nl2;
           vec[BM + qc] = dd;
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(BAR(C::B_QFULL + s), 2 * C::TILE);
+          mbar_arrive_expect_tx(BAR(B_QFULL + s), 2 * C::TILE);
           for (int c = 0; c < C::KCH; ++c) {
-            tma_load_4d(&tmQ, BAR(C::B_QFULL + s), sbase + C::OFF_Q + s * C::TILE + c * C::CHUNK,
+            tma_load_4d(&tmQ, BAR(B_QFULL + s), sbase + C::A_OFF_Q + s * C::TILE + c * C::CHUNK,
                         c * 64, h, q_row0 + q0, bcoord);
-            tma_load_4d(&tmDO, BAR(C::B_QFULL + s), sbase + C::OFF_DO + s * C::TILE + c * C::CHUNK,
+            tma_load_4d(&tmDO, BAR(B_QFULL + s), sbase + C::A_OFF_DO + s * C::TILE + c * C::CHUNK,
                         c * 64, h, q_row0 + q0, bcoord);
           }
         } else {
-          mbar_arrive(BAR(C::B_QFULL + s));
+          mbar_arrive(BAR(B_QFULL + s));
         }
       }
     }
@@ -279,230 +256,156 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == 1) {
     // ============================================================ MMA issuer
     if (lane == 0 && n_q > 0) {
-      constexpr uint32_t ID_SS_KK = idesc_f16_f32acc(BF16, 128, 128, false, false);  // Sᵀ, dPᵀ
-      constexpr uint32_t ID_KMN = idesc_f16_f32acc(BF16, 128, D, false, true);       // dV, dK
-      constexpr uint32_t ID_MNMN = idesc_f16_f32acc(BF16, 128, D, true, true);       // dQ
-      const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V, sDS = sbase + C::OFF_DS;
-      mbar_wait(BAR(C::B_KV), 0, abort_flag, p.status);
+      constexpr uint32_t ID_ST = idesc_f16_f32acc(BF16, 128, 128, false, false);  // Sᵀ, dPᵀ
+      constexpr uint32_t ID_ACC = idesc_f16_f32acc(BF16, 128, D, false, true);    // dV, dK
+      const uint32_t sK = sbase + C::A_OFF_K, sV = sbase + C::A_OFF_V;
+      // X = A Bᵀ with A = [keys][d] (K-major) and B = [queries][d] (K-major)
+      auto issue_kt = [&](uint32_t dst, uint32_t sa, uint32_t sb) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          mma_ss(tmem + dst, sdesc_sw128(sa + off, 16, 1024), sdesc_sw128(sb + off, 16, 1024),
+                 ID_ST, kk > 0 ? 1u : 0u);
+        }
+      };
+      // Acc += Xᵀ-packed (tensor memory, keys x queries) · B with B = [queries][d]
+      auto issue_acc = [&](uint32_t acc, uint32_t src, uint32_t sb, bool accumulate) {
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ts(tmem + acc, tmem + src + C::packed_col(kk), sdesc_sw128(sb + kk * 2048, C::CHUNK, 1024),
+                 ID_ACC, (accumulate || kk > 0) ? 1u : 0u);
+      };
+      auto wait_q = [&](int it) {
+        mbar_wait(BAR(B_QFULL + it % ST), (uint32_t)(it / ST) & 1u, abort_flag, p.status);
+        tc_fence_after();
+      };
+      mbar_wait(BAR(B_KV), 0, abort_flag, p.status);
+      wait_q(0);
+      issue_kt(TM_S, sK, sbase + C::A_OFF_Q);
+      mma_commit(BAR(B_SFULL));
+      issue_kt(TM_DP, sV, sbase + C::A_OFF_DO);
+      mma_commit(BAR(B_DPFULL));
       for (int it = 0; it < n_q; ++it) {
         const int s = it % ST;
         const uint32_t ph = (uint32_t)it & 1u;
-        const uint32_t sQ = sbase + C::OFF_Q + s * C::TILE;
-        const uint32_t sDO = sbase + C::OFF_DO + s * C::TILE;
-        mbar_wait(BAR(C::B_QFULL + s), (uint32_t)(it / ST) & 1u, abort_flag, p.status);
+        const uint32_t sQ = sbase + C::A_OFF_Q + s * C::TILE;
+        const uint32_t sDO = sbase + C::A_OFF_DO + s * C::TILE;
+        mbar_wait(BAR(B_PFULL), ph, abort_flag, p.status);
         tc_fence_after();
-        // Sᵀ = K Qᵀ   (M = keys, N = queries, K = d; both operands K-major)
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + C::TM_S, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024),
-                 ID_SS_KK, kk > 0 ? 1u : 0u);
+        issue_acc(TM_DV, TM_S, sDO, it > 0);          // dV += Pᵀ dO
+        if (it + 1 < n_q) {                          // Sᵀ of the next step over Pᵀ
+          wait_q(it + 1);
+          issue_kt(TM_S, sK, sbase + C::A_OFF_Q + ((it + 1) % ST) * C::TILE);
+          mma_commit(BAR(B_SFULL));
         }
-        mma_commit(BAR(C::B_SFULL));
-        // dPᵀ = V dOᵀ, written where dQ of the previous step lived: wait until drained.
-        if (it > 0) mbar_wait(BAR(C::B_DQEMPTY), ph ^ 1u, abort_flag, p.status);
+        mbar_wait(BAR(B_DSFULL), ph, abort_flag, p.status);
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + C::TM_DP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024),
-                 ID_SS_KK, kk > 0 ? 1u : 0u);
+        issue_acc(TM_DK, TM_DP, sQ, it > 0);         // dK += dSᵀ Q
+        mma_commit(BAR(B_QEMPTY + s));
+        if (it + 1 < n_q) {                          // dPᵀ of the next step over dSᵀ
+          issue_kt(TM_DP, sV, sbase + C::A_OFF_DO + ((it + 1) % ST) * C::TILE);
+          mma_commit(BAR(B_DPFULL));
         }
-        mma_commit(BAR(C::B_DPFULL));
-        // dV += Pᵀ dO   (A = Pᵀ in tensor memory; B = dO as [d x queries], d-contiguous)
-        mbar_wait(BAR(C::B_PFULL), ph, abort_flag, p.status);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8,
-                 sdesc_sw128(sDO + kk * 2048, C::CHUNK, 1024), ID_KMN, (it > 0 || kk > 0) ? 1u : 0u);
-        // dK += dSᵀ Q   (A = dSᵀ [keys x queries] K-major; B = Q as [d x queries])
-        mbar_wait(BAR(C::B_DSFULL), ph, abort_flag, p.status);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint32_t offa = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + C::TM_DK, sdesc_sw128(sDS + offa, 16, 1024),
-                 sdesc_sw128(sQ + kk * 2048, C::CHUNK, 1024), ID_KMN, (it > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(BAR(C::B_QEMPTY + s));
-        // dQ_i = dS K   (M = queries: A = dS read from the [key][query] buffer, query-
-        // contiguous = MN-major; B = K as [d x keys], d-contiguous), into dPᵀ's columns.
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ss(tmem + C::TM_DP, sdesc_sw128(sDS + kk * 2048, C::CHUNK, 1024),
-                 sdesc_sw128(sK + kk * 2048, C::CHUNK, 1024), ID_MNMN, kk > 0 ? 1u : 0u);
-        mma_commit(BAR(C::B_DSEMPTY));
-        mma_commit(BAR(C::B_DQFULL));
       }
-      mma_commit(BAR(C::B_DONE));
+      mma_commit(BAR(B_DONE));
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (warp >= 4) {
     // ============================================================ compute: Pᵀ, dSᵀ
+    const int half = (warp - 4) >> 2;   // query columns 64*half .. 64*half+63
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row within the tile
     const int kg = k0 + r;              // key index within the sequence
+    const bool key_ok = kg < Lk;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::TM_S;
-    const uint32_t tDP = tmem + lane_off + C::TM_DP;
-    const float c = p.scale_log2;
-    uint8_t* ds_row = sgen + C::OFF_DS + r * 128;
+    const uint32_t tS = tmem + lane_off + TM_S + 64 * half;
+    const uint32_t tDP = tmem + lane_off + TM_DP + 64 * half;
+    const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+    const int cbase = 64 * half;
     for (int it = 0; it < n_q; ++it) {
       const int s = it % ST;
       const uint32_t ph = (uint32_t)it & 1u;
       const int q0 = (i_begin + it) * BM;
-      const float* vec = reinterpret_cast<const float*>(sgen + C::OFF_VEC + s * 2 * BM * 4);
+      const float* vec = reinterpret_cast<const float*>(sgen + C::A_OFF_VEC + s * 2 * BM * 4);
       const bool need_mask =
           (k0 + BN > Lk) || (q0 + BM > Lq) || (p.causal && (k0 + BN - 1 > q0 + diag));
-      // Allowed queries for this key: q >= kg - diag (causal) and q < Lq.
-      const int qmin = p.causal ? kg - diag - q0 : -1;  // column index bound
-      const bool key_ok = kg < Lk;
-      mbar_wait(BAR(C::B_QFULL + s), (uint32_t)(it / ST) & 1u, abort_flag, p.status);
-      mbar_wait(BAR(C::B_SFULL), ph, abort_flag, p.status);
+      const int qmin = p.causal ? kg - diag - q0 : -1;  // allowed columns: c >= qmin
+      mbar_wait(BAR(B_QFULL + s), (uint32_t)(it / ST) & 1u, abort_flag, p.status);
+      mbar_wait(BAR(B_SFULL), ph, abort_flag, p.status);
       tc_fence_after();
-      uint32_t pk[64];  // Pᵀ row as packed 16-bit pairs
+      uint32_t sv[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_wait_ld();
+      reg_fence(sv);
+      uint32_t pk[32];  // Pᵀ row segment, packed 16-bit pairs
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t sv[32];
-        tmem_ld32(tS + q * 32, sv);
-        tmem_wait_ld();
-        reg_fence(sv);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = q * 32 + 2 * e;
-          float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * e]), c, -vec[c0]));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), c, -vec[c0 + 1]));
-          if (need_mask) {
-            if (!key_ok || c0 < qmin || q0 + c0 >= Lq) p0 = 0.f;
-            if (!key_ok || c0 + 1 < qmin || q0 + c0 + 1 >= Lq) p1 = 0.f;
-          }
-          pk[q * 16 + e] = pack2<BF16>(p0, p1);
+      for (int e = 0; e < 32; ++e) {
+        const int c0 = cbase + 2 * e;
+        const float2 nl = *reinterpret_cast<const float2*>(&vec[c0]);
+        const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
+                                          c2, f2_pack(nl.x, nl.y)));
+        float p0 = ex2_approx(x.x);
+        float p1 = ex2_approx(x.y);
+        if (need_mask) {
+          if (!key_ok || c0 < qmin || q0 + c0 >= Lq) p0 = 0.f;
+          if (!key_ok || c0 + 1 < qmin || q0 + c0 + 1 >= Lq) p1 = 0.f;
         }
-        tmem_st16(tS + q * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[q * 16]));
+        pk[e] = pack2<BF16>(p0, p1);
       }
+      tmem_st32(tS, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(BAR(C::B_PFULL));
+      mbar_arrive(BAR(B_PFULL));
 
-      // dSᵀ = Pᵀ ∘ (dPᵀ − D) into shared memory, 128-byte swizzled [key][query].
-      mbar_wait(BAR(C::B_DPFULL), ph, abort_flag, p.status);
-      if (it > 0) mbar_wait(BAR(C::B_DSEMPTY), ph ^ 1u, abort_flag, p.status);
+      // dSᵀ = Pᵀ ∘ (dPᵀ − D), packed over this thread's own dPᵀ columns.
+      mbar_wait(BAR(B_DPFULL), ph, abort_flag, p.status);
       tc_fence_after();
+      uint32_t dv[64];
+      tmem_ld32(tDP, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
+      tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
+      tmem_wait_ld();
+      reg_fence(dv);
+      uint32_t ds[32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t dv[32];
-        tmem_ld32(tDP + q * 32, dv);
-        tmem_wait_ld();
-        reg_fence(dv);
-        uint32_t o[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = q * 32 + 2 * e;
-          float2 pf;
-          if constexpr (BF16)
-            pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[q * 16 + e]));
-          else
-            pf = __half22float2(*reinterpret_cast<const __half2*>(&pk[q * 16 + e]));
-          const float d0 = pf.x * (__uint_as_float(dv[2 * e]) - vec[BM + c0]);
-          const float d1 = pf.y * (__uint_as_float(dv[2 * e + 1]) - vec[BM + c0 + 1]);
-          o[e] = pack2<BF16>(d0, d1);
-        }
-        // columns q*32 .. q*32+31 = chunk (q/2), 16-byte units (q%2)*4 .. +3
-        const int chunk = q >> 1;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = (q & 1) * 4 + u;
-          uint4* dst = reinterpret_cast<uint4*>(ds_row + chunk * C::CHUNK + ((unit ^ (r & 7)) << 4));
-          *dst = make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
-        }
+      for (int e = 0; e < 32; ++e) {
+        const int c0 = cbase + 2 * e;
+        const float2 dd = *reinterpret_cast<const float2*>(&vec[BM + c0]);
+        const float2 pf = unpack2<BF16>(pk[e]);
+        const uint64_t t = f2_add(f2_pack(__uint_as_float(dv[2 * e]), __uint_as_float(dv[2 * e + 1])),
+                                  f2_pack(-dd.x, -dd.y));
+        const float2 d2 = f2_unpack(f2_mul(t, f2_pack(pf.x, pf.y)));
+        ds[e] = pack2<BF16>(d2.x, d2.y);
       }
-      fence_proxy_async_smem();
+      tmem_st32(tDP, ds);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(BAR(C::B_DSFULL));
+      mbar_arrive(BAR(B_DSFULL));
     }
-    // ---------------------------------------------------------------- dV epilogue
+    // ---------------------------------------------------------------- epilogue
+    // half 0 stores dV, half 1 stores dK = scale · Σ dSᵀ Q
     if (n_q > 0) {
-      mbar_wait(BAR(C::B_DONE), 0, abort_flag, p.status);
+      mbar_wait(BAR(B_DONE), 0, abort_flag, p.status);
       tc_fence_after();
     }
-    uint16_t* dvrow = reinterpret_cast<uint16_t*>(p.dv) +
-                      (p.cu_q != nullptr ? ((size_t)(k_row0 + kg) * p.H + h) * D
-                                         : (((size_t)bcoord * p.N + kg) * p.H + h) * D);
+    uint16_t* orow = reinterpret_cast<uint16_t*>(half == 0 ? p.dv : p.dk) +
+                     (p.cu_q != nullptr ? ((size_t)(k_row0 + kg) * p.H + h) * D
+                                        : (((size_t)bcoord * p.N + kg) * p.H + h) * D);
+    const float sc = half == 0 ? 1.f : p.scale;
+    const uint32_t tsrc = tmem + lane_off + (half == 0 ? TM_DV : TM_DK);
 #pragma unroll 1
     for (int q = 0; q < D / 32; ++q) {
       uint32_t v[32];
       if (n_q > 0) {
-        tmem_ld32(tmem + lane_off + C::TM_DV + q * 32, v);
+        tmem_ld32(tsrc + q * 32, v);
         tmem_wait_ld();
         reg_fence(v);
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0u;
       }
-      if (kg < Lk) {
-        uint4* dst = reinterpret_cast<uint4*>(dvrow + q * 32);
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          dst[u] = make_uint4(pack2<BF16>(__uint_as_float(v[8 * u]), __uint_as_float(v[8 * u + 1])),
-                              pack2<BF16>(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3])),
-                              pack2<BF16>(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5])),
-                              pack2<BF16>(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7])));
-      }
-    }
-  } else {
-    // ============================================================ dq: drain dQ_i, dK epilogue
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // query row within the step (dQ) / key row (dK)
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tDQ = tmem + lane_off + C::TM_DP;
-    for (int it = 0; it < n_q; ++it) {
-      const uint32_t ph = (uint32_t)it & 1u;
-      const int qg = (i_begin + it) * BM + r;
-      mbar_wait(BAR(C::B_DQFULL), ph, abort_flag, p.status);
-      tc_fence_after();
-      float* dst = p.dq_acc + (p.cu_q != nullptr ? ((size_t)(q_row0 + qg) * p.H + h) * D
-                                                 : (((size_t)bcoord * p.N + qg) * p.H + h) * D);
-#pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t v[32];
-        tmem_ld32(tDQ + q * 32, v);
-        tmem_wait_ld();
-        reg_fence(v);
-        if (qg < Lq) {
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            atomicAdd(reinterpret_cast<float4*>(dst + q * 32) + u,
-                      make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
-                                  __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3])));
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(BAR(C::B_DQEMPTY));
-    }
-    // dK = scale · (Σ dSᵀ Q)
-    if (n_q > 0) {
-      mbar_wait(BAR(C::B_DONE), 0, abort_flag, p.status);
-      tc_fence_after();
-    }
-    const int kg = k0 + r;
-    uint16_t* dkrow = reinterpret_cast<uint16_t*>(p.dk) +
-                      (p.cu_q != nullptr ? ((size_t)(k_row0 + kg) * p.H + h) * D
-                                         : (((size_t)bcoord * p.N + kg) * p.H + h) * D);
-    const float sc = p.scale;
-#pragma unroll 1
-    for (int q = 0; q < D / 32; ++q) {
-      uint32_t v[32];
-      if (n_q > 0) {
-        tmem_ld32(tmem + lane_off + C::TM_DK + q * 32, v);
-        tmem_wait_ld();
-        reg_fence(v);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0u;
-      }
-      if (kg < Lk) {
-        uint4* dst = reinterpret_cast<uint4*>(dkrow + q * 32);
+      if (key_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
           dst[u] = make_uint4(
@@ -514,7 +417,271 @@ __global__ void __launch_bounds__(320, 1)
     }
   }
 
-  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ dQ
+// Tensor memory: S two buffers [0,128), [128,256) | dP [256,384) (dS packed into it) |
+// dQ [384, 384+D).
+// Grid: x = (batch or sequence) * H + head, y = query tile (when causal, the tile that
+// sees the most key tiles first for every head).
+template <int D, bool BF16>
+__global__ void __launch_bounds__(384, 1)
+    fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                     const BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int BM = C::BM, BN = C::BN, ST = C::STAGES;
+  constexpr uint32_t TM_DP = 256, TM_DQ = 384;
+  enum { B_QFULL = 0, B_KFULL = 1, B_VFULL = B_KFULL + ST, B_KVEMPTY = B_VFULL + ST,
+         B_SFULL = B_KVEMPTY + ST, B_SEMPTY = B_SFULL + 2, B_DPFULL = B_SEMPTY + 2, B_DSFULL,
+         B_DONE };
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::B_OFF_BAR + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + C::B_OFF_BAR + 8 * C::NBAR);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int h = blockIdx.x % p.H;
+  const int bz = blockIdx.x / p.H;
+  int Lq, Lk, q_row0, k_row0, bcoord;
+  if (p.cu_q != nullptr) {
+    q_row0 = p.cu_q[bz];
+    Lq = p.cu_q[bz + 1] - q_row0;
+    k_row0 = p.cu_k[bz];
+    Lk = p.cu_k[bz + 1] - k_row0;
+    bcoord = 0;
+  } else {
+    q_row0 = k_row0 = 0;
+    Lq = Lk = p.N;
+    bcoord = bz;
+  }
+  const int tile = p.causal ? (int)(gridDim.y - 1 - blockIdx.y) : (int)blockIdx.y;
+  const int q0 = tile * BM;
+  if (q0 >= Lq) return;
+  const int diag = Lk - Lq;
+  const int kv_tiles_all = (Lk + BN - 1) / BN;
+  int n_kv = kv_tiles_all;
+  if (p.causal) {
+    const int j_last = min(q0 + BM - 1, Lq - 1) + diag;
+    n_kv = (j_last < 0) ? 0 : min(kv_tiles_all, j_last / BN + 1);
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(B_QFULL), 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(BAR(B_KFULL + s), 1);
+      mbar_init(BAR(B_VFULL + s), 1);
+      mbar_init(BAR(B_KVEMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(BAR(B_SFULL + b), 1);
+      mbar_init(BAR(B_SEMPTY + b), 256);
+    }
+    mbar_init(BAR(B_DPFULL), 1);
+    mbar_init(BAR(B_DSFULL), 256);
+    mbar_init(BAR(B_DONE), 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ============================================================ loads
+    if (lane == 0 && n_kv > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(BAR(B_QFULL), 2 * C::TILE);
+      for (int c = 0; c < C::KCH; ++c) {
+        tma_load_4d(&tmQ, BAR(B_QFULL), sbase + C::B_OFF_Q + c * C::CHUNK, c * 64, h, q_row0 + q0,
+                    bcoord);
+        tma_load_4d(&tmDO, BAR(B_QFULL), sbase + C::B_OFF_DO + c * C::CHUNK, c * 64, h, q_row0 + q0,
+                    bcoord);
+      }
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % ST;
+        mbar_wait(BAR(B_KVEMPTY + s), ((uint32_t)(j / ST) & 1u) ^ 1u, abort_flag, p.status);
+        mbar_arrive_expect_tx(BAR(B_KFULL + s), C::TILE);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_4d(&tmK, BAR(B_KFULL + s), sbase + C::B_OFF_K + s * C::TILE + c * C::CHUNK,
+                      c * 64, h, k_row0 + j * BN, bcoord);
+        mbar_arrive_expect_tx(BAR(B_VFULL + s), C::TILE);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_4d(&tmV, BAR(B_VFULL + s), sbase + C::B_OFF_V + s * C::TILE + c * C::CHUNK,
+                      c * 64, h, k_row0 + j * BN, bcoord);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0 && n_kv > 0) {
+      constexpr uint32_t ID_S = idesc_f16_f32acc(BF16, 128, 128, false, false);   // S, dP
+      constexpr uint32_t ID_DQ = idesc_f16_f32acc(BF16, 128, D, false, true);     // dQ
+      const uint32_t sQ = sbase + C::B_OFF_Q, sDO = sbase + C::B_OFF_DO;
+      auto issue_qt = [&](uint32_t dst, uint32_t sa, uint32_t sb) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          mma_ss(tmem + dst, sdesc_sw128(sa + off, 16, 1024), sdesc_sw128(sb + off, 16, 1024),
+                 ID_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_s = [&](int j) {  // S_j = Q K_jᵀ into buffer j % 2
+        const int s = j % ST, b = j & 1;
+        if (j >= 2) mbar_wait(BAR(B_SEMPTY + b), ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, p.status);
+        mbar_wait(BAR(B_KFULL + s), (uint32_t)(j / ST) & 1u, abort_flag, p.status);
+        tc_fence_after();
+        issue_qt(128u * b, sQ, sbase + C::B_OFF_K + s * C::TILE);
+        mma_commit(BAR(B_SFULL + b));
+      };
+      auto issue_dp = [&](int j) {  // dP_j = dO V_jᵀ
+        const int s = j % ST;
+        mbar_wait(BAR(B_VFULL + s), (uint32_t)(j / ST) & 1u, abort_flag, p.status);
+        tc_fence_after();
+        issue_qt(TM_DP, sDO, sbase + C::B_OFF_V + s * C::TILE);
+        mma_commit(BAR(B_DPFULL));
+      };
+      mbar_wait(BAR(B_QFULL), 0, abort_flag, p.status);
+      issue_s(0);
+      if (n_kv > 1) issue_s(1);
+      issue_dp(0);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % ST;
+        // dQ += dS K_j  (A = dS in tensor memory; B = K_j as [d x keys], d-contiguous)
+        mbar_wait(BAR(B_DSFULL), (uint32_t)j & 1u, abort_flag, p.status);
+        tc_fence_after();
+        const uint32_t kb = sbase + C::B_OFF_K + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(tmem + TM_DQ, tmem + TM_DP + C::packed_col(kk),
+                 sdesc_sw128(kb + kk * 2048, C::CHUNK, 1024), ID_DQ, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(BAR(B_KVEMPTY + s));
+        if (j + 2 < n_kv) issue_s(j + 2);
+        if (j + 1 < n_kv) issue_dp(j + 1);  // over dS_j, after the product that reads it
+      }
+      mma_commit(BAR(B_DONE));
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ============================================================ compute: dS
+    const int half = (warp - 4) >> 2;   // key columns 64*half .. 64*half+63
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // query row within the tile
+    const int i = q0 + r;               // query index within the sequence
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tDP = tmem + lane_off + TM_DP + 64 * half;
+    const float kLog2e = 1.4426950408889634f;
+    float nl2 = -INFINITY, dd = 0.f;  // this row's -LSE·log2(e) and D
+    if (i < Lq) {
+      const size_t vi = (p.cu_q != nullptr) ? (size_t)h * p.total_q + q_row0 + i
+                                            : ((size_t)bcoord * p.H + h) * p.N + i;
+      nl2 = -p.lse[vi] * kLog2e;
+      dd = p.dvec[vi];
+    }
+    const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+    const uint64_t nl22 = f2_pack(nl2, nl2);
+    const uint64_t nd2 = f2_pack(-dd, -dd);
+    for (int j = 0; j < n_kv; ++j) {
+      const int b = j & 1;
+      const int k0 = j * BN + 64 * half;  // first key of this thread's columns
+      const bool need_mask = (j * BN + BN > Lk) || (p.causal && (j * BN + BN - 1 > q0 + diag));
+      const int lim = min(Lk - k0, p.causal ? i + diag - k0 + 1 : 64);  // columns c < lim allowed
+      mbar_wait(BAR(B_SFULL + b), (uint32_t)(j >> 1) & 1u, abort_flag, p.status);
+      tc_fence_after();
+      uint32_t sv[64];
+      const uint32_t tS = tmem + lane_off + 128u * b + 64 * half;
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_wait_ld();
+      reg_fence(sv);
+      tc_fence_before();
+      mbar_arrive(BAR(B_SEMPTY + b));  // the S buffer may be overwritten now
+      float pv[64];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
+                                          c2, nl22));
+        pv[2 * e] = ex2_approx(x.x);
+        pv[2 * e + 1] = ex2_approx(x.y);
+      }
+      if (need_mask) {
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+          if (e >= lim) pv[e] = 0.f;
+      }
+      mbar_wait(BAR(B_DPFULL), (uint32_t)j & 1u, abort_flag, p.status);
+      tc_fence_after();
+      uint32_t dv[64];
+      tmem_ld32(tDP, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
+      tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
+      tmem_wait_ld();
+      reg_fence(dv);
+      uint32_t ds[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        // P is rounded to 16 bits first, as in the dK/dV pass and the forward P·V product
+        const float2 pr = unpack2<BF16>(pack2<BF16>(pv[2 * e], pv[2 * e + 1]));
+        const uint64_t t = f2_add(f2_pack(__uint_as_float(dv[2 * e]), __uint_as_float(dv[2 * e + 1])), nd2);
+        const float2 d2 = f2_unpack(f2_mul(t, f2_pack(pr.x, pr.y)));
+        ds[e] = pack2<BF16>(d2.x, d2.y);
+      }
+      tmem_st32(tDP, ds);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR(B_DSFULL));
+    }
+    // ---------------------------------------------------------------- epilogue
+    // dQ = scale · Σ dS K; half h stores columns [D/2 * h, D/2 * (h+1))
+    if (n_kv > 0) {
+      mbar_wait(BAR(B_DONE), 0, abort_flag, p.status);
+      tc_fence_after();
+    }
+    uint16_t* orow = reinterpret_cast<uint16_t*>(p.dq) +
+                     (p.cu_q != nullptr ? ((size_t)(q_row0 + i) * p.H + h) * D
+                                        : (((size_t)bcoord * p.N + i) * p.H + h) * D);
+    const float sc = p.scale;
+#pragma unroll 1
+    for (int q = half * (D / 64); q < (half + 1) * (D / 64); ++q) {
+      uint32_t v[32];
+      if (n_kv > 0) {
+        tmem_ld32(tmem + lane_off + TM_DQ + q * 32, v);
+        tmem_wait_ld();
+        reg_fence(v);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
+      }
+      if (i < Lq) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          dst[u] = make_uint4(
+              pack2<BF16>(__uint_as_float(v[8 * u]) * sc, __uint_as_float(v[8 * u + 1]) * sc),
+              pack2<BF16>(__uint_as_float(v[8 * u + 2]) * sc, __uint_as_float(v[8 * u + 3]) * sc),
+              pack2<BF16>(__uint_as_float(v[8 * u + 4]) * sc, __uint_as_float(v[8 * u + 5]) * sc),
+              pack2<BF16>(__uint_as_float(v[8 * u + 6]) * sc, __uint_as_float(v[8 * u + 7]) * sc));
+      }
+    }
+  }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -37,8 +37,7 @@ struct BwdParams {
   void* dq;
   void* dk;
   void* dv;
-  float* dq_acc;      // fp32 accumulator, same element layout as q
-  float* dvec;        // D = rowsum(dO ∘ O), same layout as lse
+  float* dvec;        // D = rowsum(dO ∘ O), same layout as lse (caller's workspace)
   const int* cu_q;
   const int* cu_k;
   int B, N, H;
@@ -59,10 +58,11 @@ LaunchResult launch_fwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensor
 // Forward grid: x = query-tile pairs, y = heads, z = batch (dense) or sequences (varlen).
 int fwd_rows_per_cta();
 
-// Backward launch: preprocess, main kernel, dQ conversion.  q_rows = B*N (dense) or
-// total_q (varlen); grid z = batches (dense B, or varlen num_seqs).
+// Backward launch: D preprocess, dK/dV pass, dQ pass.  q_rows = B*N (dense) or total_q
+// (varlen); batches = B (dense) or num_seqs (varlen).
 LaunchResult launch_bwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                         const CUtensorMap& tmV, const CUtensorMap& tmDO, const BwdParams& p,
-                        long long q_rows, int max_seqlen_k, int batches, cudaStream_t stream);
+                        long long q_rows, int max_seqlen_q, int max_seqlen_k, int batches,
+                        cudaStream_t stream);
 
 }  // namespace fattn

@@ -80,11 +80,14 @@ __global__ void __launch_bounds__(320, 1)
   const int lane = threadIdx.x & 31;
 
   // ---------------------------------------------------------------- work item
-  const int h = blockIdx.y;
-  const int pair = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  // grid: x = (batch or sequence) * H + head, y = query-tile pair; when causal the pair
+  // with the most key tiles is launched first for every head.
+  const int h = blockIdx.x % p.H;
+  const int bz = blockIdx.x / p.H;
+  const int pair = p.causal ? (int)(gridDim.y - 1 - blockIdx.y) : (int)blockIdx.y;
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
-    const int s = blockIdx.z;
+    const int s = bz;
     q_row0 = p.cu_q[s];
     Lq = p.cu_q[s + 1] - q_row0;
     k_row0 = p.cu_k[s];
@@ -94,7 +97,7 @@ __global__ void __launch_bounds__(320, 1)
     q_row0 = 0;
     k_row0 = 0;
     Lq = Lk = p.N;
-    bcoord = blockIdx.z;
+    bcoord = bz;
   }
   const int q0 = pair * (BM * QT);
   if (q0 >= Lq) return;  // uniform for the whole CTA

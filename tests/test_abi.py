@@ -45,12 +45,12 @@ def test_status_strings(lib):
 
 
 def test_workspace_sizes(lib):
+    # the backward workspace holds D = rowsum(dO ∘ O): fp32 [B, H, N], 256-byte rounded
     B, N, H, d = 2, 16384, 32, 128
-    e = B * N * H * d
-    assert lib.fa_bwd_workspace_size(B, N, H, d) == e * 4 + B * H * N * 4
-    assert lib.fa_bwd_workspace_size(1, 3, 1, 64) == 768 + 256
+    assert lib.fa_bwd_workspace_size(B, N, H, d) == B * H * N * 4
+    assert lib.fa_bwd_workspace_size(1, 3, 1, 64) == 256
     assert lib.fa_bwd_workspace_size(0, 3, 1, 64) == 0
-    assert lib.fa_varlen_bwd_workspace_size(896, 32, 128) == 896 * 32 * 128 * 4 + 896 * 32 * 4
+    assert lib.fa_varlen_bwd_workspace_size(896, 32, 128) == 896 * 32 * 4
 
 
 P = ctypes.c_void_p(4096)  # a 16-byte aligned fake address; validation fails before any use
@@ -84,7 +84,11 @@ def test_rejects_negative_sizes(lib):
 
 def test_size_limits(lib):
     assert lib.fa_fwd(P, P, P, P, P, 70000, 70000, 1, 64, 0.1, 0, 0, None) == \
-        _lib.FA_ERR_UNSUPPORTED
+        _lib.FA_ERR_UNSUPPORTED          # B*N >= 2^31
+    assert lib.fa_fwd(P, P, P, P, P, 1, 9000000, 1, 64, 0.1, 0, 0, None) == \
+        _lib.FA_ERR_UNSUPPORTED          # more 128-row tiles than a grid dimension holds
+    assert lib.fa_bwd(P, P, P, P, P, P, P, P, P, 1, 9000000, 1, 64, 0.1, 0, P, 1 << 40, 0,
+                      None) == _lib.FA_ERR_UNSUPPORTED
 
 
 def test_empty_problems_are_noops(lib):
