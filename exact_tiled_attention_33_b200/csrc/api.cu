@@ -98,10 +98,11 @@ int check_ptrs(std::initializer_list<const void*> ptrs) {
   return FA_OK;
 }
 
-// Grids are x = batches * H, y = 128-row tiles of the sequence.
+// Grids are x = 128-row tiles of the sequence, y = heads, z = batches or sequences.
 int check_grid(long long batches, long long H, long long max_len) {
-  if (batches * H >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "batch*heads must be < 2^31");
-  if (max_len > 65535LL * 128) return fail(FA_ERR_UNSUPPORTED, "sequence length must be <= 8388480");
+  if (batches > 65535) return fail(FA_ERR_UNSUPPORTED, "batch / number of sequences must be <= 65535");
+  if (H > 65535) return fail(FA_ERR_UNSUPPORTED, "H must be <= 65535");
+  (void)max_len;  // B*N < 2^31 bounds the tile count far below the x-dimension limit
   return FA_OK;
 }
 
@@ -172,7 +173,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   const int rows = fwd_rows_per_cta();
-  dim3 grid((unsigned)(B * H), (N + rows - 1) / rows);
+  dim3 grid((N + rows - 1) / rows, H, B);
   return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
 }
 
@@ -214,7 +215,7 @@ int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* l
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   const int rows = fwd_rows_per_cta();
-  dim3 grid((unsigned)(num_seqs * H), (max_seqlen_q + rows - 1) / rows);
+  dim3 grid((max_seqlen_q + rows - 1) / rows, H, num_seqs);
   return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
 }
 

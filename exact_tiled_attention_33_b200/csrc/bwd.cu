@@ -30,10 +30,10 @@ static LaunchResult launch_bwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
   const long long pre_blocks = std::min<long long>((warps + 7) / 8, (long long)sms * 16);
   fa_bwd_pre_kernel<D, BF16><<<(unsigned)pre_blocks, 256, 0, stream>>>(p, q_rows);
   // 2) dK, dV: one CTA per key tile
-  dim3 grid_a((unsigned)(batches * p.H), (max_seqlen_k + C::BN - 1) / C::BN);
+  dim3 grid_a((max_seqlen_k + C::BN - 1) / C::BN, p.H, batches);
   fa_bwd_dkdv_kernel<D, BF16><<<grid_a, C::THREADS, C::SMEM_A, stream>>>(tmQ, tmK, tmV, tmDO, p);
   // 3) dQ: one CTA per query tile
-  dim3 grid_b((unsigned)(batches * p.H), (max_seqlen_q + C::BM - 1) / C::BM);
+  dim3 grid_b((max_seqlen_q + C::BM - 1) / C::BM, p.H, batches);
   fa_bwd_dq_kernel<D, BF16><<<grid_b, C::THREADS, C::SMEM_B, stream>>>(tmQ, tmK, tmV, tmDO, p);
   return cudaGetLastError() == cudaSuccess ? LaunchResult::kOk : LaunchResult::kCudaError;
 }

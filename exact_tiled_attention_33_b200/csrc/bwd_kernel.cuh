@@ -107,15 +107,18 @@ struct BwdCfg {
   static constexpr int A_OFF_DO = A_OFF_Q + STAGES * TILE;
   static constexpr int A_OFF_VEC = A_OFF_DO + STAGES * TILE;  // per stage: -lse*log2e, D
   static constexpr int A_OFF_BAR = A_OFF_VEC + STAGES * 2 * BM * 4;
-  // dQ kernel: Q, dO resident; K and V streamed
+  // dQ kernel: Q, dO resident; K streamed through 3 stages (it is needed from the S
+  // product two steps ahead until the dQ product), V through 2
+  static constexpr int K_STAGES = 3;
   static constexpr int B_OFF_Q = 0;
   static constexpr int B_OFF_DO = B_OFF_Q + TILE;
   static constexpr int B_OFF_K = B_OFF_DO + TILE;
-  static constexpr int B_OFF_V = B_OFF_K + STAGES * TILE;
+  static constexpr int B_OFF_V = B_OFF_K + K_STAGES * TILE;
   static constexpr int B_OFF_BAR = B_OFF_V + STAGES * TILE;
-  static constexpr int NBAR = 16;
+  static constexpr int NBAR = 24;  // mbarrier slots reserved in either kernel
   static constexpr int SMEM_A = A_OFF_BAR + 8 * NBAR + 16 + 1024;
   static constexpr int SMEM_B = B_OFF_BAR + 8 * NBAR + 16 + 1024;
+  static_assert(SMEM_A <= 232448 && SMEM_B <= 232448, "shared memory per CTA");
   static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
   // packed 16-bit operand column for K-elements 16*kk .. 16*kk+15 of a 128-wide row:
@@ -132,8 +135,9 @@ struct BwdCfg {
 // ------------------------------------------------------------------ dK, dV
 // Tensor memory: Sᵀ [0,128) (Pᵀ packed into it) | dPᵀ [128,256) (dSᵀ packed into it) |
 // dK [256, 256+D) | dV [256+D, 256+2D).
-// Grid: x = (batch or sequence) * H + head, y = key tile (tile 0, which has the most
-// query tiles when causal, first for every head).
+// Grid: x = key tile (fastest, so the CTAs running together share one head's Q/dO in
+// L2; tile 0, which has the most query tiles when causal, first), y = head, z = batch or
+// sequence.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(384, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -144,6 +148,7 @@ __global__ void __launch_bounds__(384, 1)
   constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DK = 256, TM_DV = 256 + D;
   enum { B_KV = 0, B_QFULL = 1, B_QEMPTY = B_QFULL + ST, B_SFULL = B_QEMPTY + ST, B_DPFULL,
          B_PFULL, B_DSFULL, B_DONE };
+  static_assert(B_DONE < C::NBAR, "mbarrier slots");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -154,8 +159,8 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int h = blockIdx.x % p.H;
-  const int bz = blockIdx.x / p.H;
+  const int h = blockIdx.y;
+  const int bz = blockIdx.z;
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
     q_row0 = p.cu_q[bz];
@@ -168,7 +173,7 @@ __global__ void __launch_bounds__(384, 1)
     Lq = Lk = p.N;
     bcoord = bz;
   }
-  const int k0 = blockIdx.y * BN;
+  const int k0 = blockIdx.x * BN;
   if (k0 >= Lk) return;
   const int diag = Lk - Lq;  // key j is allowed for query i iff j <= i + diag (causal)
   const int q_tiles = (Lq + BM - 1) / BM;
@@ -258,22 +263,27 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0 && n_q > 0) {
       constexpr uint32_t ID_ST = idesc_f16_f32acc(BF16, 128, 128, false, false);  // Sᵀ, dPᵀ
       constexpr uint32_t ID_ACC = idesc_f16_f32acc(BF16, 128, D, false, true);    // dV, dK
-      const uint32_t sK = sbase + C::A_OFF_K, sV = sbase + C::A_OFF_V;
+      // Descriptors built once; each MMA only adds a compile-time offset.
+      const uint64_t dK = sdesc_sw128(sbase + C::A_OFF_K, 16, 1024);
+      const uint64_t dV = sdesc_sw128(sbase + C::A_OFF_V, 16, 1024);
+      const uint64_t dQk = sdesc_sw128(sbase + C::A_OFF_Q, 16, 1024);          // K-major
+      const uint64_t dDOk = sdesc_sw128(sbase + C::A_OFF_DO, 16, 1024);        // K-major
+      const uint64_t dQm = sdesc_sw128(sbase + C::A_OFF_Q, C::CHUNK, 1024);    // MN-major
+      const uint64_t dDOm = sdesc_sw128(sbase + C::A_OFF_DO, C::CHUNK, 1024);  // MN-major
       // X = A Bᵀ with A = [keys][d] (K-major) and B = [queries][d] (K-major)
-      auto issue_kt = [&](uint32_t dst, uint32_t sa, uint32_t sb) {
+      auto issue_kt = [&](uint32_t dst, uint64_t da, uint64_t db) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + dst, sdesc_sw128(sa + off, 16, 1024), sdesc_sw128(sb + off, 16, 1024),
-                 ID_ST, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + dst, sdesc_adv(da, off), sdesc_adv(db, off), ID_ST, kk > 0 ? 1u : 0u);
         }
       };
       // Acc += Xᵀ-packed (tensor memory, keys x queries) · B with B = [queries][d]
-      auto issue_acc = [&](uint32_t acc, uint32_t src, uint32_t sb, bool accumulate) {
+      auto issue_acc = [&](uint32_t acc, uint32_t src, uint64_t db, bool accumulate) {
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + acc, tmem + src + C::packed_col(kk), sdesc_sw128(sb + kk * 2048, C::CHUNK, 1024),
-                 ID_ACC, (accumulate || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + acc, tmem + src + C::packed_col(kk), sdesc_adv(db, kk * 2048), ID_ACC,
+                 (accumulate || kk > 0) ? 1u : 0u);
       };
       auto wait_q = [&](int it) {
         mbar_wait(BAR(B_QFULL + it % ST), (uint32_t)(it / ST) & 1u, abort_flag, p.status);
@@ -281,29 +291,28 @@ __global__ void __launch_bounds__(384, 1)
       };
       mbar_wait(BAR(B_KV), 0, abort_flag, p.status);
       wait_q(0);
-      issue_kt(TM_S, sK, sbase + C::A_OFF_Q);
+      issue_kt(TM_S, dK, dQk);
       mma_commit(BAR(B_SFULL));
-      issue_kt(TM_DP, sV, sbase + C::A_OFF_DO);
+      issue_kt(TM_DP, dV, dDOk);
       mma_commit(BAR(B_DPFULL));
       for (int it = 0; it < n_q; ++it) {
         const int s = it % ST;
+        const int s1 = (it + 1) % ST;
         const uint32_t ph = (uint32_t)it & 1u;
-        const uint32_t sQ = sbase + C::A_OFF_Q + s * C::TILE;
-        const uint32_t sDO = sbase + C::A_OFF_DO + s * C::TILE;
         mbar_wait(BAR(B_PFULL), ph, abort_flag, p.status);
         tc_fence_after();
-        issue_acc(TM_DV, TM_S, sDO, it > 0);          // dV += Pᵀ dO
+        issue_acc(TM_DV, TM_S, sdesc_adv(dDOm, s * C::TILE), it > 0);   // dV += Pᵀ dO
         if (it + 1 < n_q) {                          // Sᵀ of the next step over Pᵀ
           wait_q(it + 1);
-          issue_kt(TM_S, sK, sbase + C::A_OFF_Q + ((it + 1) % ST) * C::TILE);
+          issue_kt(TM_S, dK, sdesc_adv(dQk, s1 * C::TILE));
           mma_commit(BAR(B_SFULL));
         }
         mbar_wait(BAR(B_DSFULL), ph, abort_flag, p.status);
         tc_fence_after();
-        issue_acc(TM_DK, TM_DP, sQ, it > 0);         // dK += dSᵀ Q
+        issue_acc(TM_DK, TM_DP, sdesc_adv(dQm, s * C::TILE), it > 0);   // dK += dSᵀ Q
         mma_commit(BAR(B_QEMPTY + s));
         if (it + 1 < n_q) {                          // dPᵀ of the next step over dSᵀ
-          issue_kt(TM_DP, sV, sbase + C::A_OFF_DO + ((it + 1) % ST) * C::TILE);
+          issue_kt(TM_DP, dV, sdesc_adv(dDOk, s1 * C::TILE));
           mma_commit(BAR(B_DPFULL));
         }
       }
@@ -428,8 +437,8 @@ __global__ void __launch_bounds__(384, 1)
 // ------------------------------------------------------------------ dQ
 // Tensor memory: S two buffers [0,128), [128,256) | dP [256,384) (dS packed into it) |
 // dQ [384, 384+D).
-// Grid: x = (batch or sequence) * H + head, y = query tile (when causal, the tile that
-// sees the most key tiles first for every head).
+// Grid: x = query tile (fastest, sharing one head's K/V in L2; when causal the tile
+// that sees the most key tiles first), y = head, z = batch or sequence.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(384, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -438,9 +447,11 @@ __global__ void __launch_bounds__(384, 1)
   using C = BwdCfg<D>;
   constexpr int BM = C::BM, BN = C::BN, ST = C::STAGES;
   constexpr uint32_t TM_DP = 256, TM_DQ = 384;
-  enum { B_QFULL = 0, B_KFULL = 1, B_VFULL = B_KFULL + ST, B_KVEMPTY = B_VFULL + ST,
-         B_SFULL = B_KVEMPTY + ST, B_SEMPTY = B_SFULL + 2, B_DPFULL = B_SEMPTY + 2, B_DSFULL,
-         B_DONE };
+  constexpr int KST = C::K_STAGES;
+  enum { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KST, B_VFULL = B_KEMPTY + KST,
+         B_VEMPTY = B_VFULL + ST, B_SFULL = B_VEMPTY + ST, B_SEMPTY = B_SFULL + 2,
+         B_DPFULL = B_SEMPTY + 2, B_DSFULL, B_DONE };
+  static_assert(B_DONE < C::NBAR, "mbarrier slots");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -451,8 +462,8 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int h = blockIdx.x % p.H;
-  const int bz = blockIdx.x / p.H;
+  const int h = blockIdx.y;
+  const int bz = blockIdx.z;
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
     q_row0 = p.cu_q[bz];
@@ -465,7 +476,7 @@ __global__ void __launch_bounds__(384, 1)
     Lq = Lk = p.N;
     bcoord = bz;
   }
-  const int tile = p.causal ? (int)(gridDim.y - 1 - blockIdx.y) : (int)blockIdx.y;
+  const int tile = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
   const int q0 = tile * BM;
   if (q0 >= Lq) return;
   const int diag = Lk - Lq;
@@ -478,10 +489,13 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(B_QFULL), 1);
-    for (int s = 0; s < ST; ++s) {
+    for (int s = 0; s < KST; ++s) {
       mbar_init(BAR(B_KFULL + s), 1);
+      mbar_init(BAR(B_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < ST; ++s) {
       mbar_init(BAR(B_VFULL + s), 1);
-      mbar_init(BAR(B_KVEMPTY + s), 1);
+      mbar_init(BAR(B_VEMPTY + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(BAR(B_SFULL + b), 1);
@@ -517,12 +531,13 @@ __global__ void __launch_bounds__(384, 1)
                     bcoord);
       }
       for (int j = 0; j < n_kv; ++j) {
-        const int s = j % ST;
-        mbar_wait(BAR(B_KVEMPTY + s), ((uint32_t)(j / ST) & 1u) ^ 1u, abort_flag, p.status);
-        mbar_arrive_expect_tx(BAR(B_KFULL + s), C::TILE);
+        const int ks = j % KST, s = j % ST;
+        mbar_wait(BAR(B_KEMPTY + ks), ((uint32_t)(j / KST) & 1u) ^ 1u, abort_flag, p.status);
+        mbar_arrive_expect_tx(BAR(B_KFULL + ks), C::TILE);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_4d(&tmK, BAR(B_KFULL + s), sbase + C::B_OFF_K + s * C::TILE + c * C::CHUNK,
+          tma_load_4d(&tmK, BAR(B_KFULL + ks), sbase + C::B_OFF_K + ks * C::TILE + c * C::CHUNK,
                       c * 64, h, k_row0 + j * BN, bcoord);
+        mbar_wait(BAR(B_VEMPTY + s), ((uint32_t)(j / ST) & 1u) ^ 1u, abort_flag, p.status);
         mbar_arrive_expect_tx(BAR(B_VFULL + s), C::TILE);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(&tmV, BAR(B_VFULL + s), sbase + C::B_OFF_V + s * C::TILE + c * C::CHUNK,
@@ -535,47 +550,54 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0 && n_kv > 0) {
       constexpr uint32_t ID_S = idesc_f16_f32acc(BF16, 128, 128, false, false);   // S, dP
       constexpr uint32_t ID_DQ = idesc_f16_f32acc(BF16, 128, D, false, true);     // dQ
-      const uint32_t sQ = sbase + C::B_OFF_Q, sDO = sbase + C::B_OFF_DO;
-      auto issue_qt = [&](uint32_t dst, uint32_t sa, uint32_t sb) {
+      // Descriptors built once; each MMA only adds a compile-time offset.
+      const uint64_t dQ = sdesc_sw128(sbase + C::B_OFF_Q, 16, 1024);
+      const uint64_t dDO = sdesc_sw128(sbase + C::B_OFF_DO, 16, 1024);
+      const uint64_t dKk = sdesc_sw128(sbase + C::B_OFF_K, 16, 1024);         // K-major
+      const uint64_t dKm = sdesc_sw128(sbase + C::B_OFF_K, C::CHUNK, 1024);   // MN-major
+      const uint64_t dVk = sdesc_sw128(sbase + C::B_OFF_V, 16, 1024);
+      auto issue_qt = [&](uint32_t dst, uint64_t da, uint64_t db) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + dst, sdesc_sw128(sa + off, 16, 1024), sdesc_sw128(sb + off, 16, 1024),
-                 ID_S, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + dst, sdesc_adv(da, off), sdesc_adv(db, off), ID_S, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_s = [&](int j) {  // S_j = Q K_jᵀ into buffer j % 2
-        const int s = j % ST, b = j & 1;
+        const int ks = j % KST, b = j & 1;
         if (j >= 2) mbar_wait(BAR(B_SEMPTY + b), ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, p.status);
-        mbar_wait(BAR(B_KFULL + s), (uint32_t)(j / ST) & 1u, abort_flag, p.status);
+        mbar_wait(BAR(B_KFULL + ks), (uint32_t)(j / KST) & 1u, abort_flag, p.status);
         tc_fence_after();
-        issue_qt(128u * b, sQ, sbase + C::B_OFF_K + s * C::TILE);
+        issue_qt(128u * b, dQ, sdesc_adv(dKk, ks * C::TILE));
         mma_commit(BAR(B_SFULL + b));
       };
-      auto issue_dp = [&](int j) {  // dP_j = dO V_jᵀ
+      auto issue_dp = [&](int j) {  // dP_j = dO V_jᵀ; V_j is free once it completes
         const int s = j % ST;
         mbar_wait(BAR(B_VFULL + s), (uint32_t)(j / ST) & 1u, abort_flag, p.status);
         tc_fence_after();
-        issue_qt(TM_DP, sDO, sbase + C::B_OFF_V + s * C::TILE);
+        issue_qt(TM_DP, dDO, sdesc_adv(dVk, s * C::TILE));
         mma_commit(BAR(B_DPFULL));
+        mma_commit(BAR(B_VEMPTY + s));
       };
       mbar_wait(BAR(B_QFULL), 0, abort_flag, p.status);
       issue_s(0);
       if (n_kv > 1) issue_s(1);
       issue_dp(0);
       for (int j = 0; j < n_kv; ++j) {
-        const int s = j % ST;
+        const int ks = j % KST;
         // dQ += dS K_j  (A = dS in tensor memory; B = K_j as [d x keys], d-contiguous)
         mbar_wait(BAR(B_DSFULL), (uint32_t)j & 1u, abort_flag, p.status);
         tc_fence_after();
-        const uint32_t kb = sbase + C::B_OFF_K + s * C::TILE;
+        const uint64_t kb = sdesc_adv(dKm, ks * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + TM_DQ, tmem + TM_DP + C::packed_col(kk),
-                 sdesc_sw128(kb + kk * 2048, C::CHUNK, 1024), ID_DQ, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(BAR(B_KVEMPTY + s));
+          mma_ts(tmem + TM_DQ, tmem + TM_DP + C::packed_col(kk), sdesc_adv(kb, kk * 2048), ID_DQ,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(BAR(B_KEMPTY + ks));
+        // dP of the next step goes first (the compute warps wait for it); it overwrites
+        // dS_j only after the product above that reads it (in-order pipe).
+        if (j + 1 < n_kv) issue_dp(j + 1);
         if (j + 2 < n_kv) issue_s(j + 2);
-        if (j + 1 < n_kv) issue_dp(j + 1);  // over dS_j, after the product that reads it
       }
       mma_commit(BAR(B_DONE));
     }

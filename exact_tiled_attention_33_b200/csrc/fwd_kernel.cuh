@@ -54,6 +54,7 @@ struct FwdCfg {
   static constexpr int B_OFULL = B_PFULL + QT;
   static constexpr int NBAR = B_OFULL + QT;
   static constexpr int SMEM_BYTES = OFF_BAR + 8 * NBAR + 16 + 1024;  // + alignment slack
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static constexpr int THREADS = 320;
   static constexpr uint32_t TMEM_COLS = 512;
   // tensor-memory column of S_t (P_t aliases its first BN/2 columns) and of O_t
@@ -80,11 +81,12 @@ __global__ void __launch_bounds__(320, 1)
   const int lane = threadIdx.x & 31;
 
   // ---------------------------------------------------------------- work item
-  // grid: x = (batch or sequence) * H + head, y = query-tile pair; when causal the pair
-  // with the most key tiles is launched first for every head.
-  const int h = blockIdx.x % p.H;
-  const int bz = blockIdx.x / p.H;
-  const int pair = p.causal ? (int)(gridDim.y - 1 - blockIdx.y) : (int)blockIdx.y;
+  // grid: x = query-tile pair (fastest, so the CTAs running together share one head's
+  // K/V in L2), y = head, z = batch or sequence; when causal the pair with the most key
+  // tiles of each head is launched first.
+  const int h = blockIdx.y;
+  const int bz = blockIdx.z;
+  const int pair = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
     const int s = bz;
@@ -172,25 +174,26 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t ID_S = idesc_f16_f32acc(BF16, BM, BN, false, false) |
                             (p.negate_scores ? (1u << 13) : 0u);  // bit 13: negate A
       constexpr uint32_t ID_O = idesc_f16_f32acc(BF16, BM, D, false, true);
+      // Descriptors built once; each MMA only adds a compile-time offset.
+      const uint64_t dQ0 = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(sbase + C::OFF_V, C::KV_CHUNK, 1024);
       auto issue_s = [&](int t, int s) {
-        const uint32_t qa = sbase + C::OFF_Q + t * C::Q_TILE;
-        const uint32_t ka = sbase + C::OFF_K + s * C::KV_TILE;
+        const uint64_t da = sdesc_adv(dQ0, (uint32_t)(t * C::Q_TILE));
+        const uint64_t db = sdesc_adv(dK0, (uint32_t)(s * C::KV_TILE));
+        const uint32_t dst = tmem + C::tm_s(t);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
-          const uint32_t ok = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + C::tm_s(t), sdesc_sw128(qa + oq, 16, 1024), sdesc_sw128(ka + ok, 16, 1024),
-                 ID_S, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(dst, sdesc_adv(da, (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32),
+                 sdesc_adv(db, (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32), ID_S, kk > 0 ? 1u : 0u);
       };
       auto issue_pv = [&](int t, int s, bool accumulate) {
-        const uint32_t va = sbase + C::OFF_V + s * C::KV_TILE;
+        const uint64_t db = sdesc_adv(dV0, (uint32_t)(s * C::KV_TILE));
+        const uint32_t dst = tmem + C::tm_o(t), src = tmem + C::tm_s(t);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          mma_ts(tmem + C::tm_o(t), tmem + C::tm_s(t) + kk * 8,
-                 sdesc_sw128(va + kk * 16 * 128, C::KV_CHUNK, 1024), ID_O,
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(dst, src + kk * 8, sdesc_adv(db, kk * 16 * 128), ID_O,
                  (accumulate || kk > 0) ? 1u : 0u);
-        }
       };
       mbar_wait(BAR(C::B_QFULL), 0, abort_flag, p.status);
       tc_fence_after();

@@ -181,6 +181,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// Descriptor with its start address advanced by `bytes` (a multiple of 16).  Shared
+// addresses stay below 256 KB, so the 14-bit start-address field never carries: building
+// a descriptor once and adding compile-time offsets keeps the single MMA-issuing thread
+// at one instruction pair per MMA (rebuilding descriptors per MMA made issue, not the
+// tensor core, the bottleneck).
+__device__ __forceinline__ uint64_t sdesc_adv(uint64_t d, uint32_t bytes) {
+  return d + (uint64_t)(bytes >> 4);
+}
+
 // ------------------------------------------------------------------ tcgen05.mma
 // D[tmem] (+)= A[smem] * B[smem]
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,

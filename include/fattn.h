@@ -65,8 +65,8 @@ typedef enum {
 typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
 
 /* Dense forward.  Writes o [B,N,H,d] and lse [B,H,N].
- * Sizes: B, N, H >= 0 (a zero size is a no-op), B*N < 2^31, B*H < 2^31, H < 2^16,
- * N <= 8388480 (= 65535 * 128).
+ * Sizes: B, N, H >= 0 (a zero size is a no-op), B*N < 2^31, H < 2^16,
+ * B <= 65535.
  * scale: any finite float (the pages use 1/sqrt(d)). */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N,
            int H, int d, float scale, int causal, int dtype, void* stream);
@@ -75,8 +75,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
  * Writes o [total_q,H,d] and lse [H,total_q].
  * max_seqlen_q / max_seqlen_k must be >= every sequence's length (they size the grid);
  * num_seqs, total_q, total_k are the host-side counts matching cu_seqlens (the host
- * cannot read device cu_seqlens without a synchronisation).  num_seqs * H < 2^31 and
- * max_seqlen_q, max_seqlen_k <= 8388480. */
+ * cannot read device cu_seqlens without a synchronisation).  num_seqs <= 65535. */
 int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                   const int* cu_seqlens_q, const int* cu_seqlens_k, int max_seqlen_q,
                   int max_seqlen_k, int H, int d, float scale, int causal, int num_seqs,

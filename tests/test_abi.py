@@ -85,9 +85,9 @@ def test_rejects_negative_sizes(lib):
 def test_size_limits(lib):
     assert lib.fa_fwd(P, P, P, P, P, 70000, 70000, 1, 64, 0.1, 0, 0, None) == \
         _lib.FA_ERR_UNSUPPORTED          # B*N >= 2^31
-    assert lib.fa_fwd(P, P, P, P, P, 1, 9000000, 1, 64, 0.1, 0, 0, None) == \
-        _lib.FA_ERR_UNSUPPORTED          # more 128-row tiles than a grid dimension holds
-    assert lib.fa_bwd(P, P, P, P, P, P, P, P, P, 1, 9000000, 1, 64, 0.1, 0, P, 1 << 40, 0,
+    assert lib.fa_fwd(P, P, P, P, P, 70000, 16, 1, 64, 0.1, 0, 0, None) == \
+        _lib.FA_ERR_UNSUPPORTED          # more batches than a grid dimension holds
+    assert lib.fa_bwd(P, P, P, P, P, P, P, P, P, 70000, 16, 1, 64, 0.1, 0, P, 1 << 40, 0,
                       None) == _lib.FA_ERR_UNSUPPORTED
 
 
