@@ -8,6 +8,7 @@ from .attention import (  # noqa: F401
     FlashAttnFunction,
     FlashAttnVarlenFunction,
     bwd,
+    bwd_noalloc,
     bwd_workspace,
     device_status,
     flash_attn_func,

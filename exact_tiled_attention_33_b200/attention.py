@@ -120,6 +120,26 @@ def bwd(q, k, v, o, lse, dout, softmax_scale=None, causal=False, workspace=None,
     return dq, dk, dv
 
 
+def bwd_noalloc(q, k, v, o, lse, dout, softmax_scale=None, causal=False, dq=None, dk=None,
+                dv=None):
+    """Dense backward without a workspace (fa_bwd_noalloc): D lives in the library's fixed
+    device array, so B*H*N must not exceed its capacity.  Calls on one device must not
+    overlap on the GPU."""
+    dtype = _check(q, k, v, o, dout)
+    B, N, H, d = q.shape
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, d, scale, int(bool(causal)),
+                                dtype, _stream(q))
+    _lib.check(st, "fa_bwd_noalloc")
+    return dq, dk, dv
+
+
 def varlen_bwd(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
                softmax_scale=None, causal=False, workspace=None, dq=None, dk=None, dv=None):
     """Varlen backward. Returns (dq [total_q,H,d], dk, dv [total_k,H,d])."""

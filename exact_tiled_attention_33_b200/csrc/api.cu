@@ -314,6 +314,52 @@ int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, co
                     dtype, (cudaStream_t)stream);
 }
 
+// ------------------------------------------------------------------ allocation-free backward
+// Scratch for D = rowsum(dO ∘ O) when the caller cannot provide a workspace: a fixed array
+// in this module's device memory (every GPU that loads the library holds it until exit).
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 22;  // 16 MiB: B*H*N <= 4194304
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+// Device address of the scratch array on the current device, looked up once per device
+// (the host-side symbol is only a stand-in and must never be handed to a kernel).
+static int noalloc_scratch(float** out) {
+  static float* ptrs[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev >= 64) return fail(FA_ERR_UNSUPPORTED, "device index >= 64");
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    ptrs[dev] = static_cast<float*>(p);
+  }
+  *out = ptrs[dev];
+  return FA_OK;
+}
+
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d,
+                   float scale, int causal, int dtype, void* stream) {
+  g_last_error.clear();
+  if (int e = check_common(H, d, dtype, scale)) return e;
+  if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
+  if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
+  if (B == 0 || N == 0 || H == 0) return FA_OK;
+  if ((unsigned long long)B * H * N > kNoAllocScratchFloats)
+    return fail(FA_ERR_UNSUPPORTED,
+                "B*H*N = " + std::to_string((unsigned long long)B * H * N) +
+                    " exceeds the allocation-free scratch capacity of " +
+                    std::to_string(kNoAllocScratchFloats) + " (use fa_bwd with a workspace)");
+  if (int e = check_grid(B, H, N)) return e;
+  float* scratch = nullptr;
+  if (int e = noalloc_scratch(&scratch)) return e;
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, nullptr, nullptr, H, d, scale, causal,
+                    (long long)B * N, (long long)B * N, N, B, N, N, B * N, B * N, scratch,
+                    sizeof(float) * kNoAllocScratchFloats, fa_bwd_workspace_size(B, N, H, d), dtype,
+                    (cudaStream_t)stream);
+}
+
 int fa_get_device_status(void* stream) {
   g_last_error.clear();
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

@@ -105,6 +105,25 @@ int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, co
                   float scale, int causal, int num_seqs, int total_q, int total_k,
                   void* workspace, size_t workspace_bytes, int dtype, void* stream);
 
+/* Allocation-free dense backward (no counterpart on the source pages: an interface
+ * addition).  Same arguments and results as fa_bwd, without the workspace: the D vector
+ * lives in a fixed array inside the library's device memory (16 MiB, held by every GPU
+ * that loads the library until the process exits).  For callers that cannot obtain
+ * device memory at call time: hosts whose device memory belongs entirely to another
+ * allocator, or latency-critical loops that cannot afford cudaMalloc's implicit
+ * synchronisation.  Nothing is allocated: no cudaMalloc, cudaFree or allocating library
+ * routine is called.
+ *   Limit: B*H*N <= 4194304, else FA_ERR_UNSUPPORTED with a message naming the limit.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *   with that device current; make that first call before any stream capture.
+ *   All calls on a device share the one array, which keeps the last call's contents
+ *   (nothing in it needs to start at zero: every value read is written earlier in the
+ *   same call).  Calls that overlap on the GPU (different streams, or host threads
+ *   without ordering) race on it: order them on one stream or with events. */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d,
+                   float scale, int causal, int dtype, void* stream);
+
 /* Synchronises `stream`, returns FA_ERR_TIMEOUT if any kernel of this library on the
  * current device recorded a timed-out wait since the last call (FA_OK otherwise), and
  * clears the status word.  FA_ERR_CUDA if the synchronisation itself failed. */

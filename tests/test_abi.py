@@ -91,6 +91,13 @@ def test_size_limits(lib):
                       None) == _lib.FA_ERR_UNSUPPORTED
 
 
+def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
+    # B*H*N above the fixed scratch capacity is refused on the host with a clear message
+    st = lib.fa_bwd_noalloc(P, P, P, P, P, P, P, P, P, 8, 16384, 64, 128, 0.1, 1, 0, None)
+    assert st == _lib.FA_ERR_UNSUPPORTED
+    assert b"scratch capacity" in lib.fa_last_error()
+
+
 def test_empty_problems_are_noops(lib):
     # zero-size problems return OK without touching (null) pointers or the GPU
     assert lib.fa_fwd(None, None, None, None, None, 0, 128, 1, 64, 0.1, 0, 0, None) == _lib.FA_OK
