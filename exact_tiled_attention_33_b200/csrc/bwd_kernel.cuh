@@ -347,21 +347,33 @@ __global__ void __launch_bounds__(384, 1)
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
       reg_fence(sv);
+      // p = 2^(s*c - LSE*log2e): one branch-free pass (so the exp latency of different
+      // columns overlaps), masks applied afterwards only on boundary tiles.
+      const float4* nl4 = reinterpret_cast<const float4*>(&vec[cbase]);
+      float pv[64];
+#pragma unroll
+      for (int e4 = 0; e4 < 16; ++e4) {
+        const float4 nl = nl4[e4];
+        const float2 x0 = f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[4 * e4]), __uint_as_float(sv[4 * e4 + 1])),
+                                           c2, f2_pack(nl.x, nl.y)));
+        const float2 x1 = f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[4 * e4 + 2]), __uint_as_float(sv[4 * e4 + 3])),
+                                           c2, f2_pack(nl.z, nl.w)));
+        pv[4 * e4] = ex2_approx(x0.x);
+        pv[4 * e4 + 1] = ex2_approx(x0.y);
+        pv[4 * e4 + 2] = ex2_approx(x1.x);
+        pv[4 * e4 + 3] = ex2_approx(x1.y);
+      }
+      if (need_mask) {
+        // allowed columns c: key in range, c >= qmin (causal), query row q0 + c < Lq
+        const int lo = key_ok ? max(qmin, 0) - cbase : 64;
+        const int hi = min(Lq - q0, 128) - cbase;
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+          if (e < lo || e >= hi) pv[e] = 0.f;
+      }
       uint32_t pk[32];  // Pᵀ row segment, packed 16-bit pairs
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int c0 = cbase + 2 * e;
-        const float2 nl = *reinterpret_cast<const float2*>(&vec[c0]);
-        const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
-                                          c2, f2_pack(nl.x, nl.y)));
-        float p0 = ex2_approx(x.x);
-        float p1 = ex2_approx(x.y);
-        if (need_mask) {
-          if (!key_ok || c0 < qmin || q0 + c0 >= Lq) p0 = 0.f;
-          if (!key_ok || c0 + 1 < qmin || q0 + c0 + 1 >= Lq) p1 = 0.f;
-        }
-        pk[e] = pack2<BF16>(p0, p1);
-      }
+      for (int e = 0; e < 32; ++e) pk[e] = pack2<BF16>(pv[2 * e], pv[2 * e + 1]);
       tmem_st32(tS, pk);
       tmem_wait_st();
       tc_fence_before();
@@ -375,16 +387,21 @@ __global__ void __launch_bounds__(384, 1)
       tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
       tmem_wait_ld();
       reg_fence(dv);
+      const float4* d4 = reinterpret_cast<const float4*>(&vec[BM + cbase]);
       uint32_t ds[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int c0 = cbase + 2 * e;
-        const float2 dd = *reinterpret_cast<const float2*>(&vec[BM + c0]);
-        const float2 pf = unpack2<BF16>(pk[e]);
-        const uint64_t t = f2_add(f2_pack(__uint_as_float(dv[2 * e]), __uint_as_float(dv[2 * e + 1])),
-                                  f2_pack(-dd.x, -dd.y));
-        const float2 d2 = f2_unpack(f2_mul(t, f2_pack(pf.x, pf.y)));
-        ds[e] = pack2<BF16>(d2.x, d2.y);
+      for (int e4 = 0; e4 < 16; ++e4) {
+        const float4 dd = d4[e4];
+        const float2 pa = unpack2<BF16>(pk[2 * e4]);
+        const float2 pb = unpack2<BF16>(pk[2 * e4 + 1]);
+        const float2 da = f2_unpack(f2_mul(f2_add(f2_pack(__uint_as_float(dv[4 * e4]), __uint_as_float(dv[4 * e4 + 1])),
+                                                  f2_pack(-dd.x, -dd.y)),
+                                           f2_pack(pa.x, pa.y)));
+        const float2 db = f2_unpack(f2_mul(f2_add(f2_pack(__uint_as_float(dv[4 * e4 + 2]), __uint_as_float(dv[4 * e4 + 3])),
+                                                  f2_pack(-dd.z, -dd.w)),
+                                           f2_pack(pb.x, pb.y)));
+        ds[2 * e4] = pack2<BF16>(da.x, da.y);
+        ds[2 * e4 + 1] = pack2<BF16>(db.x, db.y);
       }
       tmem_st32(tDP, ds);
       tmem_wait_st();
