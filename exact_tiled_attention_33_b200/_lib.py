@@ -37,6 +37,7 @@ SIGNATURES = {
     "fa_status_string": (ctypes.c_char_p, [_i]),
     "fa_last_error": (ctypes.c_char_p, []),
     "fa_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
+    "fa_selftest_exp2": (_i, [_vp, _vp, _i, _vp]),
 }
 
 _LIB = None

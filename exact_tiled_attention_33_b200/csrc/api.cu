@@ -141,6 +141,19 @@ __global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns) {
   mbar_wait_limit(smem_u32(&bar), 0, &abort_flag, status, limit_ns);
 }
 
+// Evaluates the FMA-pipe exponential used by the forward softmax, for testing it against
+// the hardware ex2 and against exact values.
+__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(x[i], x[i + 1]);
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_poly2(x[i], 0.f).x;
+  }
+}
+
 }  // namespace fattn
 
 using namespace fattn;
@@ -392,6 +405,17 @@ const char* fa_status_string(int status) {
 }
 
 const char* fa_last_error(void) { return g_last_error.c_str(); }
+
+int fa_selftest_exp2(const float* x, float* y, int n, void* stream) {
+  g_last_error.clear();
+  if (n < 0) return fail(FA_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return FA_OK;
+  if (x == nullptr || y == nullptr) return fail(FA_ERR_INVALID_ARG, "null pointer argument");
+  const int pairs = (n + 1) / 2;
+  selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y, n);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e, "selftest_exp2 launch");
+}
 
 int fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {
   g_last_error.clear();

@@ -15,13 +15,15 @@
 //   * warp 0 issues TMA loads (Q once; K and V through a STAGES-deep ring);
 //   * warp 1, one thread, issues tcgen05.mma: S_t = Q_t K_jᵀ into tensor memory
 //     (shared x shared), and O_t += P_t V_j with P_t read from tensor memory;
-//   * warps 2..9 form two softmax warpgroups, one per query tile; thread r of a group
+//   * warps 4..11 form two softmax warpgroups, one per query tile; thread r of a group
 //     owns row r (= tensor-memory lane r): it reads its row of S with tcgen05.ld, masks,
 //     updates m and l in the exp2 domain, writes P back over S as packed 16-bit values,
 //     and rescales its row of O only when the row maximum grew by more than 2^8
 //     (exact: O and l always share the same reference maximum);
 //   * tensor memory: S0 | S1 | O0 | O1 (128 + 128 + D + D columns of 32 bits).
 #pragma once
+
+#include <type_traits>
 
 #include "fattn_internal.h"
 #include "sm100.cuh"
@@ -55,15 +57,22 @@ struct FwdCfg {
   static constexpr int NBAR = B_OFULL + QT;
   static constexpr int SMEM_BYTES = OFF_BAR + 8 * NBAR + 16 + 1024;  // + alignment slack
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-  static constexpr int THREADS = 320;
+  // 12 warps: warpgroup 0 = {loads, MMA, 2 idle}, warpgroups 1 and 2 = softmax for query
+  // tiles 0 and 1.  Registers move from warpgroup 0 to the softmax warpgroups:
+  // 128 x 112 + 256 x 192 = 63488 <= 384 x 168 (the launch allocation); with these
+  // neither the MMA issuer nor the softmax (128 scores per thread) spills.
+  static constexpr int THREADS = 384;
+  static constexpr uint32_t REGS_LOAD = 112, REGS_SOFTMAX = 192;
   static constexpr uint32_t TMEM_COLS = 512;
+  // pairs of every 16 (per 32-column chunk) whose exponentials use exp2_poly2
+  static constexpr int kPolyPairs = 4;
   // tensor-memory column of S_t (P_t aliases its first BN/2 columns) and of O_t
   __device__ static constexpr uint32_t tm_s(int t) { return (uint32_t)t * 128u; }
   __device__ static constexpr uint32_t tm_o(int t) { return 256u + (uint32_t)t * D; }
 };
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D>;
@@ -138,7 +147,9 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp < 4) {
+   regs_dealloc<C::REGS_LOAD>();
+   if (warp == 0) {
     // ============================================================ TMA producer
     if (lane == 0 && n_kv > 0) {
       tma_prefetch_desc(&tmQ);
@@ -229,9 +240,11 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
+   }
   } else {
+    regs_alloc<C::REGS_SOFTMAX>();
     // ============================================================ softmax warpgroups
-    const int t = (warp - 2) >> 2;
+    const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;  // tensor-memory lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const int r0 = q0 + t * BM;  // first query row of this tile (within the sequence)
@@ -264,16 +277,21 @@ __global__ void __launch_bounds__(320, 1)
         for (int e = 0; e < 128; ++e)
           if (e >= lim) sr[e] = __float_as_uint(-INFINITY);
       }
-      float mq[4];
+      // Row maximum as a tree of 3-input maxima (depth 5 instead of a 64-long chain).
+      float t1[43];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float a = __uint_as_float(sr[q * 32]);
+      for (int e = 0; e < 42; ++e)
+        t1[e] = fmax3(__uint_as_float(sr[3 * e]), __uint_as_float(sr[3 * e + 1]),
+                      __uint_as_float(sr[3 * e + 2]));
+      t1[42] = fmaxf(__uint_as_float(sr[126]), __uint_as_float(sr[127]));
+      float t2[15];
 #pragma unroll
-        for (int e = 1; e < 31; e += 2)
-          a = fmax3(a, __uint_as_float(sr[q * 32 + e]), __uint_as_float(sr[q * 32 + e + 1]));
-        mq[q] = fmaxf(a, __uint_as_float(sr[q * 32 + 31]));
-      }
-      const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * c;
+      for (int e = 0; e < 14; ++e) t2[e] = fmax3(t1[3 * e], t1[3 * e + 1], t1[3 * e + 2]);
+      t2[14] = t1[42];
+      const float t3a = fmax3(t2[0], t2[1], t2[2]), t3b = fmax3(t2[3], t2[4], t2[5]);
+      const float t3c = fmax3(t2[6], t2[7], t2[8]), t3d = fmax3(t2[9], t2[10], t2[11]);
+      const float t3e = fmax3(t2[12], t2[13], t2[14]);
+      const float mx = fmax3(fmax3(t3a, t3b, t3c), t3d, t3e) * c;
 
       // Reference-maximum update.  Keep the stale maximum while the new one exceeds
       // it by at most 8 (a factor 2^8 in P, harmless in fp32 accumulators).
@@ -294,24 +312,41 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t c2 = f2_pack(c, c);
       const uint64_t nm2 = f2_pack(-m_use, -m_use);
       uint64_t ls2 = 0ull, lr2 = 0ull;
+      // A quarter of the exponentials run on the FMA pipe (tiles without masked keys), the
+      // rest on the special-function unit, so that both units finish within the time of
+      // the tile's two matrix products.  The choice is made once per tile: the loop
+      // bodies stay branch-free.
+      auto exp_pass = [&](auto use_poly) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t pk[16];
+        for (int q = 0; q < 4; ++q) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[q * 32 + 2 * e]),
-                                             __uint_as_float(sr[q * 32 + 2 * e + 1])),
-                                     c2, nm2);
-          const float2 xx = f2_unpack(x2);
-          const float p0 = ex2_approx(xx.x);
-          const float p1 = ex2_approx(xx.y);
-          pk[e] = pack2<BF16>(p0, p1);
-          const float2 pr = unpack2<BF16>(pk[e]);
-          ls2 = f2_add(ls2, f2_pack(p0, p1));
-          lr2 = f2_add(lr2, f2_pack(pr.x, pr.y));
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[q * 32 + 2 * e]),
+                                               __uint_as_float(sr[q * 32 + 2 * e + 1])),
+                                       c2, nm2);
+            const float2 xx = f2_unpack(x2);
+            float p0, p1;
+            if (decltype(use_poly)::value && e < C::kPolyPairs) {
+              const float2 pp = exp2_poly2(xx.x, xx.y);
+              p0 = pp.x;
+              p1 = pp.y;
+            } else {
+              p0 = ex2_approx(xx.x);
+              p1 = ex2_approx(xx.y);
+            }
+            pk[e] = pack2<BF16>(p0, p1);
+            const float2 pr = unpack2<BF16>(pk[e]);
+            ls2 = f2_add(ls2, f2_pack(p0, p1));
+            lr2 = f2_add(lr2, f2_pack(pr.x, pr.y));
+          }
+          tmem_st16(tS + q * 16, pk);
         }
-        tmem_st16(tS + q * 16, pk);
-      }
+      };
+      if (need_mask)
+        exp_pass(std::false_type{});
+      else
+        exp_pass(std::true_type{});
       const float2 ls = f2_unpack(ls2), lr = f2_unpack(lr2);
       l = l * alpha + (ls.x + ls.y);
       l_r = l_r * alpha + (lr.x + lr.y);

@@ -92,6 +92,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   return mbar_wait_limit(bar, parity, abort_flag, status, FATTN_WAIT_LIMIT_NS);
 }
 
+// ------------------------------------------------------------------ register reallocation
+// Executed by every warp of a warpgroup.  The sum over warpgroups must stay within the
+// registers the CTA was launched with (threads x registers per thread at launch).
+template <uint32_t N>
+__device__ __forceinline__ void regs_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------ proxies and fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -339,6 +351,34 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// 2^x for two values at once on the FMA pipe (paired fp32), so that part of the softmax
+// exponentials bypass the special-function unit.  Method: Cody–Waite range reduction,
+// x = j + f with j = rint(x) obtained by the 1.5·2^23 shift (round to nearest) and
+// f in [-0.5, 0.5]; 2^f by a degree-3 polynomial whose coefficients were fitted for this
+// library (minimax relative error on [-0.5, 0.5] by Lawson-weighted least squares; max
+// relative error 7.5e-5); 2^j by adding j to the exponent field.  Inputs below -126 are
+// clamped to -126; below about -125 results approach the denormal range (~1e-38) and lose
+// relative accuracy, and they are never exactly 0: do not use it where an exact 0 is
+// required (masked keys).
+__device__ __forceinline__ float2 exp2_poly2(float a, float b) {
+  a = fmaxf(a, -126.f);
+  b = fmaxf(b, -126.f);
+  const uint64_t x = f2_pack(a, b);
+  const uint64_t t = f2_add(x, f2_pack(12582912.f, 12582912.f));   // 1.5·2^23 + j
+  const uint64_t j = f2_add(t, f2_pack(-12582912.f, -12582912.f));  // j (exact)
+  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x);             // f = x - j
+  uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
+                      f2_pack(0.2426111400127411f, 0.2426111400127411f));
+  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  const float2 pf = f2_unpack(p), tf = f2_unpack(t);
+  // bits(2^f) + (j << 23): j sits in the low mantissa bits of t (t = 0x4B400000 + j)
+  const uint32_t ea = (__float_as_uint(tf.x) - 0x4B400000u) << 23;
+  const uint32_t eb = (__float_as_uint(tf.y) - 0x4B400000u) << 23;
+  return make_float2(__uint_as_float(__float_as_uint(pf.x) + ea),
+                     __uint_as_float(__float_as_uint(pf.y) + eb));
 }
 
 // Unpack two 16-bit floats (lo = first) to fp32.

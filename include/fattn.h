@@ -141,6 +141,13 @@ const char* fa_last_error(void);
  * when the bounded wait works). */
 int fa_selftest_wait_timeout(unsigned int limit_us, void* stream);
 
+/* Evaluates, on the GPU, the FMA-pipe 2^x the forward softmax uses for part of its
+ * exponentials (Cody–Waite range reduction plus a fitted degree-3 polynomial; inputs below
+ * -126 clamp to -126; relative error <= 1e-4 for x >= -125, results of order 1e-38 below):
+ * y[i] = 2^x[i] for i < n, device pointers, asynchronous on `stream`.
+ * A self-test hook with no counterpart on the pages. */
+int fa_selftest_exp2(const float* x, float* y, int n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

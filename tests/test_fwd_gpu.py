@@ -199,3 +199,24 @@ def test_timeout_selftest():
     assert fa.device_status() == 0  # cleared
     x = torch.ones(4, device=DEV)
     assert float((x * 2).sum()) == 8.0
+
+
+def test_fma_pipe_exp2_accuracy():
+    # The forward computes a quarter of its exponentials with its own FMA-pipe 2^x
+    # (fa_selftest_exp2 evaluates it).  Check against exact 2^x (bound 1e-4 relative, the
+    # fitted polynomial's 7.5e-5 plus fp32 evaluation) and against CUDA's exp2 on the GPU.
+    from exact_tiled_attention_33_b200 import _lib
+    lib = _lib.load()
+    x = torch.linspace(-126.0, 8.0, 2_000_001, dtype=torch.float32, device=DEV)
+    x = torch.cat([x, torch.tensor([-1000.0, -200.0, -126.5, 0.0, -0.5, 0.5, 7.999],
+                                   device=DEV)])
+    y = torch.empty_like(x)
+    assert lib.fa_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(),
+                                torch.cuda.current_stream().cuda_stream) == 0
+    xs, ys = x.double().cpu().numpy(), y.double().cpu().numpy()
+    ok = xs >= -125.0                              # results in the normal fp32 range
+    rel = np.abs(ys[ok] / np.exp2(xs[ok]) - 1.0)
+    assert rel.max() <= 1e-4, rel.max()
+    assert np.all(np.abs(ys[~ok]) <= 2.0 ** -124)  # clamped / denormal boundary: ~1e-38
+    cuda = torch.exp2(x).double().cpu().numpy()
+    assert np.abs(ys[ok] / cuda[ok] - 1.0).max() <= 1.2e-4
