@@ -3,7 +3,7 @@
 
 namespace fattn {
 
-int fwd_rows_per_cta() { return FwdCfg<128>::BM * FwdCfg<128>::QT; }
+int fwd_rows_per_cta() { return FwdCfg<128>::BM; }
 
 template <int D, bool BF16>
 static LaunchResult launch_fwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
