@@ -43,16 +43,29 @@ import numpy as np
 ROW_BLOCK = 1024
 
 
-def allowed_mask(rows: np.ndarray, Lq: int, Lk: int, causal: bool) -> np.ndarray:
+def allowed_mask(rows: np.ndarray, Lq: int, Lk: int, causal: bool, window=None) -> np.ndarray:
     """Boolean [len(rows), Lk]: which keys each listed query row may attend to.
 
     Causal reading (bottom-right): key j is allowed for query i iff j <= i + (Lk - Lq).
+    Sliding window (w_left, w_right), the local attention the pages list without
+    parameters (page "FlashAttention技术深度解析" (pwwt.cn/news/595117), CUDA backend feature
+    table and "局部注意力机制"), read around the same bottom-right diagonal:
+    key j is allowed iff i + diag - w_left <= j <= i + diag + w_right, diag = Lk - Lq, a
+    negative bound meaning no bound on that side.  A window, when given, replaces
+    `causal`; causal is the window (-1, 0).
     """
     rows = np.asarray(rows, dtype=np.int64)
     keys = np.arange(Lk, dtype=np.int64)
-    if not causal:
-        return np.ones((rows.shape[0], Lk), dtype=bool)
-    return keys[None, :] <= (rows[:, None] + (Lk - Lq))
+    if window is None:
+        window = (-1, 0) if causal else (-1, -1)
+    w_left, w_right = window
+    center = rows[:, None] + (Lk - Lq)
+    ok = np.ones((rows.shape[0], Lk), dtype=bool)
+    if w_right >= 0:
+        ok &= keys[None, :] <= center + w_right
+    if w_left >= 0:
+        ok &= keys[None, :] >= center - w_left
+    return ok
 
 
 def _scores(q_rows: np.ndarray, k: np.ndarray, scale: float, mask: np.ndarray) -> np.ndarray:
@@ -76,7 +89,7 @@ def _row_softmax_stats(s: np.ndarray):
     return m_safe, l, lse, e, dead
 
 
-def softmax_probs(q, k, scale, causal, rows=None):
+def softmax_probs(q, k, scale, causal, rows=None, window=None):
     """P = softmax(scale Q Kᵀ) for the listed query rows: [len(rows), Lk] float64.
 
     Fully masked rows are all zero.
@@ -85,16 +98,17 @@ def softmax_probs(q, k, scale, causal, rows=None):
     k = np.asarray(k, dtype=np.float64)
     Lq, Lk = q.shape[0], k.shape[0]
     rows = np.arange(Lq) if rows is None else np.asarray(rows, dtype=np.int64)
-    s = _scores(q[rows], k, scale, allowed_mask(rows, Lq, Lk, causal))
+    s = _scores(q[rows], k, scale, allowed_mask(rows, Lq, Lk, causal, window))
     _, l, _, e, dead = _row_softmax_stats(s)
     return e / np.where(dead, 1.0, l)[:, None]
 
 
-def attention_forward(q, k, v, scale, causal, rows=None):
+def attention_forward(q, k, v, scale, causal, rows=None, window=None):
     """O and LSE of one (batch, head) or one packed segment.
 
     q: [Lq, d], k: [Lk, d], v: [Lk, dv] (any float dtype; upcast to float64).
     rows: optional sorted query-row indices; only those rows are evaluated.
+    window: optional (w_left, w_right) sliding window (see allowed_mask).
     Returns (O [n_rows, dv], LSE [n_rows]) in float64.
     """
     q = np.asarray(q, dtype=np.float64)
@@ -106,7 +120,7 @@ def attention_forward(q, k, v, scale, causal, rows=None):
     lse = np.zeros(rows.shape[0], dtype=np.float64)
     for b0 in range(0, rows.shape[0], ROW_BLOCK):
         r = rows[b0:b0 + ROW_BLOCK]
-        s = _scores(q[r], k, scale, allowed_mask(r, Lq, Lk, causal))
+        s = _scores(q[r], k, scale, allowed_mask(r, Lq, Lk, causal, window))
         _, l, blk_lse, e, dead = _row_softmax_stats(s)
         p = e / np.where(dead, 1.0, l)[:, None]
         out[b0:b0 + r.shape[0]] = p @ v
@@ -114,7 +128,7 @@ def attention_forward(q, k, v, scale, causal, rows=None):
     return out, lse
 
 
-def attention_backward(q, k, v, do, scale, causal, dq_rows=None, dkv_rows=None):
+def attention_backward(q, k, v, do, scale, causal, dq_rows=None, dkv_rows=None, window=None):
     """Analytic gradients of O = softmax(scale Q Kᵀ) V for one (batch, head) / segment.
 
     With P the softmax weights and D_i = sum_c dO_ic O_ic (O from this oracle, float64):
@@ -140,7 +154,7 @@ def attention_backward(q, k, v, do, scale, causal, dq_rows=None, dkv_rows=None):
     dq = np.zeros((dq_rows.shape[0], q.shape[1]), dtype=np.float64)
     for b0 in range(0, dq_rows.shape[0], ROW_BLOCK):
         r = dq_rows[b0:b0 + ROW_BLOCK]
-        p = softmax_probs(q, k, scale, causal, rows=r)
+        p = softmax_probs(q, k, scale, causal, rows=r, window=window)
         o = p @ v
         d_row = (do[r] * o).sum(axis=1)
         dp = do[r] @ v.T
@@ -153,7 +167,7 @@ def attention_backward(q, k, v, do, scale, causal, dq_rows=None, dkv_rows=None):
     if dkv_rows.shape[0] > 0 and Lq > 0:
         for b0 in range(0, Lq, ROW_BLOCK):
             r = np.arange(b0, min(Lq, b0 + ROW_BLOCK))
-            mask = allowed_mask(r, Lq, Lk, causal)
+            mask = allowed_mask(r, Lq, Lk, causal, window)
             s_full = _scores(q[r], k, scale, mask)
             _, l, lse, e, dead = _row_softmax_stats(s_full)
             p_full = e / np.where(dead, 1.0, l)[:, None]
@@ -167,7 +181,7 @@ def attention_backward(q, k, v, do, scale, causal, dq_rows=None, dkv_rows=None):
     return dq, dk, dv
 
 
-def attention_forward_bhsd(q, k, v, scale, causal):
+def attention_forward_bhsd(q, k, v, scale, causal, window=None):
     """Dense batched forward over the pages' [batch, seqlen, heads, head_dim] layout.
 
     Returns O [B, N, H, d] and LSE [B, H, N] (float64).
@@ -180,13 +194,14 @@ def attention_forward_bhsd(q, k, v, scale, causal):
     lse = np.zeros((B, H, N), dtype=np.float64)
     for b in range(B):
         for h in range(H):
-            o, l = attention_forward(q[b, :, h], k[b, :, h], v[b, :, h], scale, causal)
+            o, l = attention_forward(q[b, :, h], k[b, :, h], v[b, :, h], scale, causal,
+                                     window=window)
             out[b, :, h] = o
             lse[b, h] = l
     return out, lse
 
 
-def attention_backward_bhsd(q, k, v, do, scale, causal):
+def attention_backward_bhsd(q, k, v, do, scale, causal, window=None):
     """Dense batched backward over [batch, seqlen, heads, head_dim]: (dQ, dK, dV)."""
     q = np.asarray(q, dtype=np.float64)
     B, _, H, _ = q.shape
@@ -196,12 +211,12 @@ def attention_backward_bhsd(q, k, v, do, scale, causal):
     for b in range(B):
         for h in range(H):
             a, bb, c = attention_backward(q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h],
-                                          scale, causal)
+                                          scale, causal, window=window)
             dq[b, :, h], dk[b, :, h], dv[b, :, h] = a, bb, c
     return dq, dk, dv
 
 
-def varlen_attention_forward(q, k, v, cu_seqlens_q, cu_seqlens_k, scale, causal):
+def varlen_attention_forward(q, k, v, cu_seqlens_q, cu_seqlens_k, scale, causal, window=None):
     """Packed variable-length forward: [total, H, d] tensors, one segment per sequence.
 
     Segment s holds query rows cu_seqlens_q[s]:cu_seqlens_q[s+1] and key/value rows
@@ -219,13 +234,15 @@ def varlen_attention_forward(q, k, v, cu_seqlens_q, cu_seqlens_k, scale, causal)
         q0, q1 = int(cu_seqlens_q[s]), int(cu_seqlens_q[s + 1])
         k0, k1 = int(cu_seqlens_k[s]), int(cu_seqlens_k[s + 1])
         for h in range(H):
-            o, l = attention_forward(q[q0:q1, h], k[k0:k1, h], v[k0:k1, h], scale, causal)
+            o, l = attention_forward(q[q0:q1, h], k[k0:k1, h], v[k0:k1, h], scale, causal,
+                                     window=window)
             out[q0:q1, h] = o
             lse[h, q0:q1] = l
     return out, lse
 
 
-def varlen_attention_backward(q, k, v, do, cu_seqlens_q, cu_seqlens_k, scale, causal):
+def varlen_attention_backward(q, k, v, do, cu_seqlens_q, cu_seqlens_k, scale, causal,
+                              window=None):
     """Packed variable-length backward: (dQ [total_q,H,d], dK [total_k,H,d], dV)."""
     q = np.asarray(q, dtype=np.float64)
     dq = np.zeros(q.shape, dtype=np.float64)
@@ -237,6 +254,6 @@ def varlen_attention_backward(q, k, v, do, cu_seqlens_q, cu_seqlens_k, scale, ca
         k0, k1 = int(cu_seqlens_k[s]), int(cu_seqlens_k[s + 1])
         for h in range(H):
             a, b, c = attention_backward(q[q0:q1, h], k[k0:k1, h], v[k0:k1, h],
-                                         do[q0:q1, h], scale, causal)
+                                         do[q0:q1, h], scale, causal, window=window)
             dq[q0:q1, h], dk[k0:k1, h], dv[k0:k1, h] = a, b, c
     return dq, dk, dv
