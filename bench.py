@@ -4,10 +4,11 @@
                     [--workload long_causal]
 
 One step = the whole hot path once over one batch: fa_fwd (O, LSE) then fa_bwd
-(D preprocess, dK/dV/dQ main kernel, dQ conversion) on the long-context workload
-(B=2, H=32, N=16384, d=128, bf16, causal, seeded N(0,1) inputs).  Throughput is
-attention TFLOPS with 4·B·H·N²·d forward FLOPs (halved when causal) and 2.5x that for
-the backward pass.  Multi-GPU (torchrun) runs one independent problem per rank (heads /
+(D preprocess, dK/dV kernel, dQ kernel) on the long-context workload (B=2, H=32,
+N=16384, d=128, bf16, causal, seeded N(0,1) inputs).  Throughput is attention TFLOPS
+with 4·B·H·N²·d forward FLOPs (halved when causal) and 2.5x that for the backward pass.
+Sliding-window workloads (--workload long_local_w4096) call fa_fwd_local / fa_bwd_local
+and count 4·d FLOPs per allowed (query, key) pair.  Multi-GPU (torchrun) runs one independent problem per rank (heads /
 batches are independent: no collective on the data path, weak scaling); time is the max
 over ranks of CUDA-event time.
 
@@ -159,11 +160,19 @@ def oracle_sample_seconds(w, rows: int, head=(0, 0)):
     N = q.shape[0]
     r0 = N - rows
     t0 = time.perf_counter()
-    oracle.attention_forward(q[r0:], k, v, w.softmax_scale, w.causal)
-    oracle.attention_backward(q[r0:], k, v, do[r0:], w.softmax_scale, w.causal)
+    if w.window is None:
+        oracle.attention_forward(q[r0:], k, v, w.softmax_scale, w.causal)
+        oracle.attention_backward(q[r0:], k, v, do[r0:], w.softmax_scale, w.causal)
+    else:
+        # the sampled rows keep their positions: the window is taken against all N keys
+        # by running the last rows as a shorter query block (bottom-right alignment)
+        oracle.attention_forward(q[r0:], k, v, w.softmax_scale, False, window=w.window)
+        oracle.attention_backward(q[r0:], k, v, do[r0:], w.softmax_scale, False,
+                                  window=w.window)
     dt = time.perf_counter() - t0
-    keys = np.arange(r0, N) + 1 if w.causal else np.full(rows, N)
-    flops = 3.5 * 4.0 * float(keys.sum()) * w.d
+    win = w.window if w.window is not None else ((-1, 0) if w.causal else (-1, -1))
+    keys = wl.window_pairs(rows, N, win)
+    flops = 3.5 * 4.0 * float(keys) * w.d
     threads = os.cpu_count()
     return dt, flops, threads
 
@@ -233,13 +242,31 @@ def run_fattn(args, w):
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
 
+    def launch_fwd():
+        if wr.window is None:
+            _lib.check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  lse.data_ptr(), B, N, H, d, scale, causal, dtype, sh), "fa_fwd")
+        else:
+            _lib.check(lib.fa_fwd_local(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                        lse.data_ptr(), B, N, H, d, scale, wr.window[0],
+                                        wr.window[1], dtype, sh), "fa_fwd_local")
+
+    def launch_bwd():
+        if wr.window is None:
+            _lib.check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                  dv.data_ptr(), B, N, H, d, scale, causal, ws.data_ptr(),
+                                  ws.numel(), dtype, sh), "fa_bwd")
+        else:
+            _lib.check(lib.fa_bwd_local(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                        do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+                                        dk.data_ptr(), dv.data_ptr(), B, N, H, d, scale,
+                                        wr.window[0], wr.window[1], ws.data_ptr(), ws.numel(),
+                                        dtype, sh), "fa_bwd_local")
+
     def step():
-        _lib.check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                              lse.data_ptr(), B, N, H, d, scale, causal, dtype, sh), "fa_fwd")
-        _lib.check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                              do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                              dv.data_ptr(), B, N, H, d, scale, causal, ws.data_ptr(),
-                              ws.numel(), dtype, sh), "fa_bwd")
+        launch_fwd()
+        launch_bwd()
 
     for _ in range(args.warmup):
         step()
@@ -258,13 +285,9 @@ def run_fattn(args, w):
     t_start.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
-        _lib.check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                              lse.data_ptr(), B, N, H, d, scale, causal, dtype, sh), "fa_fwd")
+        launch_fwd()
         ev[i][1].record(stream)
-        _lib.check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                              do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                              dv.data_ptr(), B, N, H, d, scale, causal, ws.data_ptr(),
-                              ws.numel(), dtype, sh), "fa_bwd")
+        launch_bwd()
         ev[i][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
@@ -320,7 +343,7 @@ def run_fattn(args, w):
     bwd_ach = 2.5 * f_fwd / (bwd_avg / 1e3) / 1e12
     fwd_ach = f_fwd / (fwd_avg / 1e3) / 1e12
     roofline = {
-        "kernel": "fa_bwd_kernel (timed with its D preprocess and dQ conversion launches)",
+        "kernel": "fa_bwd (D preprocess + dK/dV kernel + dQ kernel, timed as one call)",
         "bound": "tensor", "achieved": bwd_ach, "peak": peak_sust, "unit": "TFLOP/s",
         "frac": bwd_ach / peak_sust,
         "peak_source": f"bf16_tflops_sustained ({peak_src})",
@@ -341,8 +364,9 @@ def run_fattn(args, w):
             rows = min(wr.N, rows * 2)
             dt, fl, threads = oracle_sample_seconds(wr, rows)
         cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"last {rows} query rows of head (b=0,h=0) against all {wr.N} keys, "
-                         f"fp64 oracle fwd+bwd ({dt:.1f} s)"}
+               "sample": f"last {rows} query rows of head (b=0,h=0) against all {wr.N} keys"
+                         f"{'' if wr.window is None else ' (window ' + str(list(wr.window)) + ')'}"
+                         f", fp64 oracle fwd+bwd ({dt:.1f} s)"}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,

@@ -33,6 +33,13 @@ SIGNATURES = {
                            _f, _i, _i, _i, _i, _vp, _sz, _i, _vp]),
     "fa_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                             _i, _vp]),
+    "fa_fwd_local": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _i, _vp]),
+    "fa_varlen_fwd_local": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i,
+                                 _i, _i, _i, _i, _vp]),
+    "fa_bwd_local": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
+                          _i, _vp, _sz, _i, _vp]),
+    "fa_varlen_bwd_local": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
+                                 _i, _i, _f, _i, _i, _i, _i, _i, _vp, _sz, _i, _vp]),
     "fa_get_device_status": (_i, [_vp]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
     "fa_last_error": (ctypes.c_char_p, []),

@@ -162,6 +162,107 @@ def varlen_bwd(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, 
     return dq, dk, dv
 
 
+# ------------------------------------------------------------------ local attention
+# Sliding-window attention (page "FlashAttention技术深度解析" (pwwt.cn/news/595117): CUDA
+# backend feature table and the section on local attention).  window = (left, right):
+# key j is allowed for query i iff i + (Lk - Lq) - left <= j <= i + (Lk - Lq) + right,
+# a negative bound meaning no bound; (-1, 0) is causal, (-1, -1) full attention.
+
+def _window(window):
+    left, right = (int(x) for x in window)
+    return left, right
+
+
+def fwd_local(q, k, v, window, softmax_scale=None, out=None, lse=None):
+    """Dense sliding-window forward (fa_fwd_local). Returns (o, lse) as fwd."""
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must all be [B, N, H, d] with equal shapes")
+    dtype = _check(q, k, v)
+    B, N, H, d = q.shape
+    wl, wr = _window(window)
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_fwd_local(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, N, H, d, scale,
+                              wl, wr, dtype, _stream(q))
+    _lib.check(st, "fa_fwd_local")
+    return o, lse_t
+
+
+def varlen_fwd_local(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, window,
+                     softmax_scale=None, out=None, lse=None):
+    """Packed sliding-window forward (fa_varlen_fwd_local). Returns (o, lse) as varlen_fwd."""
+    if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape or q.shape[1:] != k.shape[1:]:
+        raise ValueError("q must be [total_q, H, d] and k, v [total_k, H, d]")
+    dtype = _check(q, k, v)
+    for cu in (cu_seqlens_q, cu_seqlens_k):
+        if cu.dtype != torch.int32 or cu.device != q.device or not cu.is_contiguous():
+            raise ValueError("cu_seqlens must be contiguous int32 tensors on q's device")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have num_seqs + 1 entries")
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    wl, wr = _window(window)
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((H, total_q), device=q.device, dtype=torch.float32) if lse is None else lse
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_varlen_fwd_local(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t),
+                                     _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q),
+                                     int(max_seqlen_k), H, d, scale, wl, wr,
+                                     cu_seqlens_q.numel() - 1, total_q, total_k, dtype,
+                                     _stream(q))
+    _lib.check(st, "fa_varlen_fwd_local")
+    return o, lse_t
+
+
+def bwd_local(q, k, v, o, lse, dout, window, softmax_scale=None, workspace=None, dq=None,
+              dk=None, dv=None):
+    """Dense sliding-window backward (fa_bwd_local). Returns (dq, dk, dv)."""
+    dtype = _check(q, k, v, o, dout)
+    B, N, H, d = q.shape
+    wl, wr = _window(window)
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws = bwd_workspace(B, N, H, d, q.device) if workspace is None else workspace
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_bwd_local(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                              _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, d, scale, wl, wr, _ptr(ws),
+                              ws.numel(), dtype, _stream(q))
+    _lib.check(st, "fa_bwd_local")
+    return dq, dk, dv
+
+
+def varlen_bwd_local(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                     max_seqlen_k, window, softmax_scale=None, workspace=None, dq=None, dk=None,
+                     dv=None):
+    """Packed sliding-window backward (fa_varlen_bwd_local). Returns (dq, dk, dv)."""
+    dtype = _check(q, k, v, o, dout)
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    wl, wr = _window(window)
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws = varlen_bwd_workspace(total_q, H, d, q.device) if workspace is None else workspace
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_varlen_bwd_local(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                     _ptr(dq), _ptr(dk), _ptr(dv), _ptr(cu_seqlens_q),
+                                     _ptr(cu_seqlens_k), int(max_seqlen_q), int(max_seqlen_k), H,
+                                     d, scale, wl, wr, cu_seqlens_q.numel() - 1, total_q, total_k,
+                                     _ptr(ws), ws.numel(), dtype, _stream(q))
+    _lib.check(st, "fa_varlen_bwd_local")
+    return dq, dk, dv
+
+
 def device_status(stream: Optional[int] = None) -> int:
     """Synchronise and return the library status word (0 = ok, 4 = a wait timed out)."""
     lib = _lib.load()
@@ -170,47 +271,64 @@ def device_status(stream: Optional[int] = None) -> int:
 
 
 class FlashAttnFunction(torch.autograd.Function):
-    """Autograd wrapper: forward saves (q, k, v, o, lse); backward recomputes P."""
+    """Autograd wrapper: forward saves (q, k, v, o, lse); backward recomputes P.
+    window None: the causal flag decides; else the sliding-window calls."""
 
     @staticmethod
-    def forward(ctx, q, k, v, softmax_scale, causal):
-        o, lse = fwd(q, k, v, softmax_scale, causal)
+    def forward(ctx, q, k, v, softmax_scale, causal, window):
+        if window is None:
+            o, lse = fwd(q, k, v, softmax_scale, causal)
+        else:
+            o, lse = fwd_local(q, k, v, window, softmax_scale)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.softmax_scale = softmax_scale
-        ctx.causal = causal
+        ctx.args = (softmax_scale, causal, window)
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse = ctx.saved_tensors
-        dq, dk, dv = bwd(q, k, v, o, lse, do.contiguous(), ctx.softmax_scale, ctx.causal)
-        return dq, dk, dv, None, None
+        scale, causal, window = ctx.args
+        if window is None:
+            dq, dk, dv = bwd(q, k, v, o, lse, do.contiguous(), scale, causal)
+        else:
+            dq, dk, dv = bwd_local(q, k, v, o, lse, do.contiguous(), window, scale)
+        return dq, dk, dv, None, None, None
 
 
 class FlashAttnVarlenFunction(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, cu_q, cu_k, max_q, max_k, softmax_scale, causal):
-        o, lse = varlen_fwd(q, k, v, cu_q, cu_k, max_q, max_k, softmax_scale, causal)
+    def forward(ctx, q, k, v, cu_q, cu_k, max_q, max_k, softmax_scale, causal, window):
+        if window is None:
+            o, lse = varlen_fwd(q, k, v, cu_q, cu_k, max_q, max_k, softmax_scale, causal)
+        else:
+            o, lse = varlen_fwd_local(q, k, v, cu_q, cu_k, max_q, max_k, window, softmax_scale)
         ctx.save_for_backward(q, k, v, o, lse, cu_q, cu_k)
-        ctx.args = (max_q, max_k, softmax_scale, causal)
+        ctx.args = (max_q, max_k, softmax_scale, causal, window)
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse, cu_q, cu_k = ctx.saved_tensors
-        max_q, max_k, scale, causal = ctx.args
-        dq, dk, dv = varlen_bwd(q, k, v, o, lse, do.contiguous(), cu_q, cu_k, max_q, max_k,
-                                scale, causal)
-        return dq, dk, dv, None, None, None, None, None, None
+        max_q, max_k, scale, causal, window = ctx.args
+        if window is None:
+            dq, dk, dv = varlen_bwd(q, k, v, o, lse, do.contiguous(), cu_q, cu_k, max_q, max_k,
+                                    scale, causal)
+        else:
+            dq, dk, dv = varlen_bwd_local(q, k, v, o, lse, do.contiguous(), cu_q, cu_k, max_q,
+                                          max_k, window, scale)
+        return dq, dk, dv, None, None, None, None, None, None, None
 
 
-def flash_attn_func(q, k, v, softmax_scale=None, causal=False):
-    """[batch, seqlen, heads, head_dim] attention with autograd."""
-    return FlashAttnFunction.apply(q, k, v, softmax_scale, causal)
+def flash_attn_func(q, k, v, softmax_scale=None, causal=False, window=None):
+    """[batch, seqlen, heads, head_dim] attention with autograd.  window=(left, right)
+    selects sliding-window attention (and overrides causal)."""
+    return FlashAttnFunction.apply(q, k, v, softmax_scale, causal,
+                                   None if window is None else _window(window))
 
 
 def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                           softmax_scale=None, causal=False):
-    """Packed variable-length attention with autograd."""
+                           softmax_scale=None, causal=False, window=None):
+    """Packed variable-length attention with autograd (window as in flash_attn_func)."""
     return FlashAttnVarlenFunction.apply(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
-                                         max_seqlen_k, softmax_scale, causal)
+                                         max_seqlen_k, softmax_scale, causal,
+                                         None if window is None else _window(window))

@@ -48,6 +48,28 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Tensor-map encoding is a driver call and needs a current context on the calling
+// thread.  A host thread that has made no CUDA runtime call yet (an autograd worker
+// thread, for instance) has none; make the runtime's primary context current then.
+int ensure_context() {
+  using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+  static CtxGetCurrentFn get_current = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (get_current != nullptr && get_current(&ctx) == CUDA_SUCCESS && ctx != nullptr) return FA_OK;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaSetDevice(dev);  // initialises and binds the primary context
+  return e == cudaSuccess ? FA_OK : cuda_fail(e, "making the device context current");
+}
+
 // Tensor map over a [batches, rows, H, d] 16-bit tensor, dims listed innermost first
 // (d, H, rows, batches); box = 64 elements of d (one 128-byte swizzle row) x 1 head x
 // box_rows rows.  Out-of-range rows read as zero.
@@ -55,6 +77,7 @@ int make_map(CUtensorMap* map, const void* base, int d, int H, long long rows, l
              int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  if (int e = ensure_context()) return e;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)batches};
   cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2,
                            (cuuint64_t)rows * H * d * 2};
@@ -126,6 +149,100 @@ void set_fwd_scale(FwdParams& p, float scale) {
   p.scale_log2 = c > 1e-30f ? c : 1e-30f;
 }
 
+// Attention window arguments: any negative bound means "no bound" (-1); a bound that
+// already admits every key of every sequence (right >= max_seqlen_q - 1, left >=
+// max_seqlen_k - 1) becomes -1 too, so the kernels only see bounds below the sequence
+// lengths.  Index sums stay in int32 when max_seqlen_q + max_seqlen_k < 2^31.
+int normalize_window(int* wl, int* wr, long long max_q, long long max_k) {
+  if (*wl < 0) *wl = -1;
+  if (*wr < 0) *wr = -1;
+  if (*wr >= 0 && (long long)*wr >= max_q - 1) *wr = -1;
+  if (*wl >= 0 && (long long)*wl >= max_k - 1) *wl = -1;
+  if ((*wl >= 0 || *wr > 0) && max_q + max_k >= (1LL << 31))
+    return fail(FA_ERR_UNSUPPORTED, "windowed attention needs max_seqlen_q + max_seqlen_k < 2^31");
+  return FA_OK;
+}
+
+// Causal-style windows (no left bound) give the last query tiles the most key tiles;
+// those are launched first.
+int reverse_tiles(int wl, int wr) { return (wl < 0 && wr >= 0) ? 1 : 0; }
+
+int fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N,
+              int H, int d, float scale, int wl, int wr, int dtype, void* stream) {
+  if (int e = check_common(H, d, dtype, scale)) return e;
+  if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
+  if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
+  if (B == 0 || N == 0 || H == 0) return FA_OK;
+  if (int e = check_grid(B, H, N)) return e;
+  if (int e = normalize_window(&wl, &wr, N, N)) return e;
+  if (int e = check_ptrs({q, k, v, o, lse})) return e;
+  CUtensorMap mq, mk, mv;
+  if (int e = make_map(&mq, q, d, H, N, B, 128)) return e;
+  if (int e = make_map(&mk, k, d, H, N, B, 128)) return e;
+  if (int e = make_map(&mv, v, d, H, N, B, 128)) return e;
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.cu_q = p.cu_k = nullptr;
+  p.N = N;
+  p.H = H;
+  p.total_q = B * N;
+  p.scale = scale;
+  set_fwd_scale(p, scale);
+  p.win_left = wl;
+  p.win_right = wr;
+  p.reverse_tiles = reverse_tiles(wl, wr);
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  const int rows = fwd_rows_per_cta();
+  dim3 grid((N + rows - 1) / rows, H, B);
+  return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+}
+
+int fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+               const int* cu_seqlens_q, const int* cu_seqlens_k, int max_seqlen_q,
+               int max_seqlen_k, int H, int d, float scale, int wl, int wr, int num_seqs,
+               int total_q, int total_k, int dtype, void* stream) {
+  if (int e = check_common(H, d, dtype, scale)) return e;
+  if (num_seqs < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
+    return fail(FA_ERR_INVALID_ARG, "sizes must be >= 0");
+  if (num_seqs > 65535) return fail(FA_ERR_UNSUPPORTED, "num_seqs must be <= 65535");
+  if (max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return fail(FA_ERR_INVALID_ARG, "max_seqlen exceeds the total token count");
+  if (num_seqs == 0 || total_q == 0 || H == 0 || max_seqlen_q == 0) return FA_OK;
+  if (int e = check_grid(num_seqs, H, std::max(max_seqlen_q, max_seqlen_k))) return e;
+  if (int e = normalize_window(&wl, &wr, max_seqlen_q, max_seqlen_k)) return e;
+  if (int e = check_ptrs({q, o, lse, cu_seqlens_q, cu_seqlens_k})) return e;
+  if (total_k > 0)
+    if (int e = check_ptrs({k, v})) return e;
+  CUtensorMap mq, mk, mv;
+  if (int e = make_map(&mq, q, d, H, total_q, 1, 128)) return e;
+  // With no keys at all every row is fully masked and K/V are never read.
+  const void* kb = total_k > 0 ? k : q;
+  const void* vb = total_k > 0 ? v : q;
+  const long long kr = total_k > 0 ? total_k : total_q;
+  if (int e = make_map(&mk, kb, d, H, kr, 1, 128)) return e;
+  if (int e = make_map(&mv, vb, d, H, kr, 1, 128)) return e;
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.N = 0;
+  p.H = H;
+  p.total_q = total_q;
+  p.scale = scale;
+  set_fwd_scale(p, scale);
+  p.win_left = wl;
+  p.win_right = wr;
+  p.reverse_tiles = reverse_tiles(wl, wr);
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  const int rows = fwd_rows_per_cta();
+  dim3 grid((max_seqlen_q + rows - 1) / rows, H, num_seqs);
+  return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+}
+
 }  // namespace
 
 // Bounded-wait self test: waits on a barrier that nothing arrives at.
@@ -163,31 +280,14 @@ extern "C" {
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N, int H,
            int d, float scale, int causal, int dtype, void* stream) {
   g_last_error.clear();
-  if (int e = check_common(H, d, dtype, scale)) return e;
-  if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
-  if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
-  if (B == 0 || N == 0 || H == 0) return FA_OK;
-  if (int e = check_grid(B, H, N)) return e;
-  if (int e = check_ptrs({q, k, v, o, lse})) return e;
-  CUtensorMap mq, mk, mv;
-  if (int e = make_map(&mq, q, d, H, N, B, 128)) return e;
-  if (int e = make_map(&mk, k, d, H, N, B, 128)) return e;
-  if (int e = make_map(&mv, v, d, H, N, B, 128)) return e;
-  FwdParams p{};
-  p.o = o;
-  p.lse = lse;
-  p.cu_q = p.cu_k = nullptr;
-  p.N = N;
-  p.H = H;
-  p.total_q = B * N;
-  p.scale = scale;
-  set_fwd_scale(p, scale);
-  p.causal = causal ? 1 : 0;
-  p.status = status_ptr();
-  if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-  const int rows = fwd_rows_per_cta();
-  dim3 grid((N + rows - 1) / rows, H, B);
-  return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+  return fwd_dense(q, k, v, o, lse, B, N, H, d, scale, -1, causal ? 0 : -1, dtype, stream);
+}
+
+int fa_fwd_local(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N,
+                 int H, int d, float scale, int window_left, int window_right, int dtype,
+                 void* stream) {
+  g_last_error.clear();
+  return fwd_dense(q, k, v, o, lse, B, N, H, d, scale, window_left, window_right, dtype, stream);
 }
 
 int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -195,41 +295,19 @@ int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* l
                   int max_seqlen_k, int H, int d, float scale, int causal, int num_seqs,
                   int total_q, int total_k, int dtype, void* stream) {
   g_last_error.clear();
-  if (int e = check_common(H, d, dtype, scale)) return e;
-  if (num_seqs < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
-    return fail(FA_ERR_INVALID_ARG, "sizes must be >= 0");
-  if (num_seqs > 65535) return fail(FA_ERR_UNSUPPORTED, "num_seqs must be <= 65535");
-  if (max_seqlen_q > total_q || max_seqlen_k > total_k)
-    return fail(FA_ERR_INVALID_ARG, "max_seqlen exceeds the total token count");
-  if (num_seqs == 0 || total_q == 0 || H == 0 || max_seqlen_q == 0) return FA_OK;
-  if (int e = check_grid(num_seqs, H, std::max(max_seqlen_q, max_seqlen_k))) return e;
-  if (int e = check_ptrs({q, o, lse, cu_seqlens_q, cu_seqlens_k})) return e;
-  if (total_k > 0)
-    if (int e = check_ptrs({k, v})) return e;
-  CUtensorMap mq, mk, mv;
-  if (int e = make_map(&mq, q, d, H, total_q, 1, 128)) return e;
-  // With no keys at all every row is fully masked and K/V are never read.
-  const void* kb = total_k > 0 ? k : q;
-  const void* vb = total_k > 0 ? v : q;
-  const long long kr = total_k > 0 ? total_k : total_q;
-  if (int e = make_map(&mk, kb, d, H, kr, 1, 128)) return e;
-  if (int e = make_map(&mv, vb, d, H, kr, 1, 128)) return e;
-  FwdParams p{};
-  p.o = o;
-  p.lse = lse;
-  p.cu_q = cu_seqlens_q;
-  p.cu_k = cu_seqlens_k;
-  p.N = 0;
-  p.H = H;
-  p.total_q = total_q;
-  p.scale = scale;
-  set_fwd_scale(p, scale);
-  p.causal = causal ? 1 : 0;
-  p.status = status_ptr();
-  if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-  const int rows = fwd_rows_per_cta();
-  dim3 grid((max_seqlen_q + rows - 1) / rows, H, num_seqs);
-  return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+  return fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, H,
+                    d, scale, -1, causal ? 0 : -1, num_seqs, total_q, total_k, dtype, stream);
+}
+
+int fa_varlen_fwd_local(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int max_seqlen_q,
+                        int max_seqlen_k, int H, int d, float scale, int window_left,
+                        int window_right, int num_seqs, int total_q, int total_k, int dtype,
+                        void* stream) {
+  g_last_error.clear();
+  return fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, H,
+                    d, scale, window_left, window_right, num_seqs, total_q, total_k, dtype,
+                    stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int N, int H, int d) {
@@ -247,10 +325,11 @@ namespace {
 // Shared validation and launch for both backward entry points.
 int bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, const int* cu_q, const int* cu_k,
-               int H, int d, float scale, int causal, long long q_rows, long long k_rows, int N,
-               int batches, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+               int H, int d, float scale, int wl, int wr, long long q_rows, long long k_rows,
+               int N, int batches, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
                void* workspace,
                size_t workspace_bytes, size_t need, int dtype, cudaStream_t stream) {
+  if (int e = normalize_window(&wl, &wr, max_seqlen_q, max_seqlen_k)) return e;
   if (int e = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv, workspace})) return e;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(FA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
@@ -272,7 +351,9 @@ int bwd_common(const void* q, const void* k, const void* v, const void* o, const
   p.total_q = total_q; p.total_k = total_k;
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
-  p.causal = causal ? 1 : 0;
+  p.win_left = wl;
+  p.win_right = wr;
+  p.reverse_tiles = reverse_tiles(wl, wr);
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   return launch_result(launch_bwd(d, dtype == FA_BF16, mq, mk, mv, mdo, p, q_rows, max_seqlen_q,
@@ -281,27 +362,28 @@ int bwd_common(const void* q, const void* k, const void* v, const void* o, const
 
 }  // namespace
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-           const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d, float scale,
-           int causal, void* workspace, size_t workspace_bytes, int dtype, void* stream) {
-  g_last_error.clear();
+namespace {
+
+int bwd_dense(const void* q, const void* k, const void* v, const void* o, const void* dout,
+              const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d,
+              float scale, int wl, int wr, void* workspace, size_t workspace_bytes, int dtype,
+              void* stream) {
   if (int e = check_common(H, d, dtype, scale)) return e;
   if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
   if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
   if (B == 0 || N == 0 || H == 0) return FA_OK;
   if (int e = check_grid(B, H, N)) return e;
-  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, nullptr, nullptr, H, d, scale, causal,
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, nullptr, nullptr, H, d, scale, wl, wr,
                     (long long)B * N, (long long)B * N, N, B, N, N, B * N, B * N, workspace,
                     workspace_bytes, fa_bwd_workspace_size(B, N, H, d), dtype,
                     (cudaStream_t)stream);
 }
 
-int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                  const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
-                  const int* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k, int H, int d,
-                  float scale, int causal, int num_seqs, int total_q, int total_k,
-                  void* workspace, size_t workspace_bytes, int dtype, void* stream) {
-  g_last_error.clear();
+int bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
+               const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+               const int* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k, int H, int d,
+               float scale, int wl, int wr, int num_seqs, int total_q, int total_k,
+               void* workspace, size_t workspace_bytes, int dtype, void* stream) {
   if (int e = check_common(H, d, dtype, scale)) return e;
   if (num_seqs < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
     return fail(FA_ERR_INVALID_ARG, "sizes must be >= 0");
@@ -321,10 +403,51 @@ int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, co
   }
   if (int e = check_grid(num_seqs, H, std::max(max_seqlen_q, max_seqlen_k))) return e;
   return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, H, d, scale,
-                    causal, total_q, total_k, 0, num_seqs, max_seqlen_q, max_seqlen_k, total_q,
-                    total_k,
-                    workspace, workspace_bytes, fa_varlen_bwd_workspace_size(total_q, H, d),
-                    dtype, (cudaStream_t)stream);
+                    wl, wr, total_q, total_k, 0, num_seqs, max_seqlen_q, max_seqlen_k, total_q,
+                    total_k, workspace, workspace_bytes,
+                    fa_varlen_bwd_workspace_size(total_q, H, d), dtype, (cudaStream_t)stream);
+}
+
+}  // namespace
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d, float scale,
+           int causal, void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  g_last_error.clear();
+  return bwd_dense(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, d, scale, -1, causal ? 0 : -1,
+                   workspace, workspace_bytes, dtype, stream);
+}
+
+int fa_bwd_local(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d,
+                 float scale, int window_left, int window_right, void* workspace,
+                 size_t workspace_bytes, int dtype, void* stream) {
+  g_last_error.clear();
+  return bwd_dense(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, d, scale, window_left,
+                   window_right, workspace, workspace_bytes, dtype, stream);
+}
+
+int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k, int H, int d,
+                  float scale, int causal, int num_seqs, int total_q, int total_k,
+                  void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  g_last_error.clear();
+  return bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                    max_seqlen_k, H, d, scale, -1, causal ? 0 : -1, num_seqs, total_q, total_k,
+                    workspace, workspace_bytes, dtype, stream);
+}
+
+int fa_varlen_bwd_local(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int max_seqlen_q,
+                        int max_seqlen_k, int H, int d, float scale, int window_left,
+                        int window_right, int num_seqs, int total_q, int total_k,
+                        void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  g_last_error.clear();
+  return bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                    max_seqlen_k, H, d, scale, window_left, window_right, num_seqs, total_q,
+                    total_k, workspace, workspace_bytes, dtype, stream);
 }
 
 // ------------------------------------------------------------------ allocation-free backward
@@ -367,8 +490,9 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   if (int e = check_grid(B, H, N)) return e;
   float* scratch = nullptr;
   if (int e = noalloc_scratch(&scratch)) return e;
-  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, nullptr, nullptr, H, d, scale, causal,
-                    (long long)B * N, (long long)B * N, N, B, N, N, B * N, B * N, scratch,
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, nullptr, nullptr, H, d, scale, -1,
+                    causal ? 0 : -1, (long long)B * N, (long long)B * N, N, B, N, N, B * N, B * N,
+                    scratch,
                     sizeof(float) * kNoAllocScratchFloats, fa_bwd_workspace_size(B, N, H, d), dtype,
                     (cudaStream_t)stream);
 }

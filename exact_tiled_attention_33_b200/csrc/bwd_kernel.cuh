@@ -175,14 +175,10 @@ __global__ void __launch_bounds__(384, 1)
   }
   const int k0 = blockIdx.x * BN;
   if (k0 >= Lk) return;
-  const int diag = Lk - Lq;  // key j is allowed for query i iff j <= i + diag (causal)
-  const int q_tiles = (Lq + BM - 1) / BM;
-  int i_begin = 0;
-  if (p.causal) {
-    const int first_q = k0 - diag;  // first query row that may see key k0
-    i_begin = first_q <= 0 ? 0 : first_q / BM;
-  }
-  const int n_q = q_tiles > i_begin ? q_tiles - i_begin : 0;
+  const int diag = Lk - Lq;  // bottom-right alignment of the window (causal: j <= i + diag)
+  const int wl = p.win_left, wr = p.win_right;
+  int i_begin, n_q;          // query tiles i_begin .. i_begin + n_q - 1
+  query_tile_range(k0, min(k0 + BN - 1, Lk - 1), Lq, diag, wl, wr, BM, &i_begin, &n_q);
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(B_KV), 1);
@@ -336,9 +332,12 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t ph = (uint32_t)it & 1u;
       const int q0 = (i_begin + it) * BM;
       const float* vec = reinterpret_cast<const float*>(sgen + C::A_OFF_VEC + s * 2 * BM * 4);
-      const bool need_mask =
-          (k0 + BN > Lk) || (q0 + BM > Lq) || (p.causal && (k0 + BN - 1 > q0 + diag));
-      const int qmin = p.causal ? kg - diag - q0 : -1;  // allowed columns: c >= qmin
+      const bool need_mask = (k0 + BN > Lk) || (q0 + BM > Lq) ||
+                             (wr >= 0 && k0 + BN - 1 > q0 + diag + wr) ||
+                             (wl >= 0 && k0 < q0 + BM - 1 + diag - wl);
+      // allowed columns (query q0 + c): qmin <= c < qend
+      const int qmin = wr >= 0 ? kg - diag - wr - q0 : -1;
+      const int qend = wl >= 0 ? min(Lq - q0, kg - diag + wl - q0 + 1) : Lq - q0;
       mbar_wait(BAR(B_QFULL + s), (uint32_t)(it / ST) & 1u, abort_flag, p.status);
       mbar_wait(BAR(B_SFULL), ph, abort_flag, p.status);
       tc_fence_after();
@@ -364,9 +363,9 @@ __global__ void __launch_bounds__(384, 1)
         pv[4 * e4 + 3] = ex2_approx(x1.y);
       }
       if (need_mask) {
-        // allowed columns c: key in range, c >= qmin (causal), query row q0 + c < Lq
+        // allowed columns c: key in range, qmin <= c < qend (window and sequence end)
         const int lo = key_ok ? max(qmin, 0) - cbase : 64;
-        const int hi = min(Lq - q0, 128) - cbase;
+        const int hi = min(qend, 128) - cbase;
 #pragma unroll
         for (int e = 0; e < 64; ++e)
           if (e < lo || e >= hi) pv[e] = 0.f;
@@ -493,16 +492,13 @@ __global__ void __launch_bounds__(384, 1)
     Lq = Lk = p.N;
     bcoord = bz;
   }
-  const int tile = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  const int tile = p.reverse_tiles ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
   const int q0 = tile * BM;
   if (q0 >= Lq) return;
   const int diag = Lk - Lq;
-  const int kv_tiles_all = (Lk + BN - 1) / BN;
-  int n_kv = kv_tiles_all;
-  if (p.causal) {
-    const int j_last = min(q0 + BM - 1, Lq - 1) + diag;
-    n_kv = (j_last < 0) ? 0 : min(kv_tiles_all, j_last / BN + 1);
-  }
+  const int wl = p.win_left, wr = p.win_right;
+  int j0, n_kv;  // key tiles j0 .. j0 + n_kv - 1
+  key_tile_range(q0, min(q0 + BM - 1, Lq - 1), Lk, diag, wl, wr, BN, &j0, &n_kv);
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(B_QFULL), 1);
@@ -553,12 +549,12 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(BAR(B_KFULL + ks), C::TILE);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(&tmK, BAR(B_KFULL + ks), sbase + C::B_OFF_K + ks * C::TILE + c * C::CHUNK,
-                      c * 64, h, k_row0 + j * BN, bcoord);
+                      c * 64, h, k_row0 + (j0 + j) * BN, bcoord);
         mbar_wait(BAR(B_VEMPTY + s), ((uint32_t)(j / ST) & 1u) ^ 1u, abort_flag, p.status);
         mbar_arrive_expect_tx(BAR(B_VFULL + s), C::TILE);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(&tmV, BAR(B_VFULL + s), sbase + C::B_OFF_V + s * C::TILE + c * C::CHUNK,
-                      c * 64, h, k_row0 + j * BN, bcoord);
+                      c * 64, h, k_row0 + (j0 + j) * BN, bcoord);
       }
     }
     __syncwarp();
@@ -640,9 +636,13 @@ __global__ void __launch_bounds__(384, 1)
     const uint64_t nd2 = f2_pack(-dd, -dd);
     for (int j = 0; j < n_kv; ++j) {
       const int b = j & 1;
-      const int k0 = j * BN + 64 * half;  // first key of this thread's columns
-      const bool need_mask = (j * BN + BN > Lk) || (p.causal && (j * BN + BN - 1 > q0 + diag));
-      const int lim = min(Lk - k0, p.causal ? i + diag - k0 + 1 : 64);  // columns c < lim allowed
+      const int kt = (j0 + j) * BN;       // first key of the tile
+      const int k0 = kt + 64 * half;      // first key of this thread's columns
+      const bool need_mask = (kt + BN > Lk) || (wr >= 0 && kt + BN - 1 > q0 + diag + wr) ||
+                             (wl >= 0 && kt < q0 + BM - 1 + diag - wl);
+      // allowed columns: lo <= c < lim
+      const int lim = wr >= 0 ? min(Lk - k0, i + diag + wr - k0 + 1) : Lk - k0;
+      const int lo = wl >= 0 ? i + diag - wl - k0 : 0;
       mbar_wait(BAR(B_SFULL + b), (uint32_t)(j >> 1) & 1u, abort_flag, p.status);
       tc_fence_after();
       uint32_t sv[64];
@@ -664,7 +664,7 @@ __global__ void __launch_bounds__(384, 1)
       if (need_mask) {
 #pragma unroll
         for (int e = 0; e < 64; ++e)
-          if (e >= lim) pv[e] = 0.f;
+          if (e >= lim || e < lo) pv[e] = 0.f;
       }
       mbar_wait(BAR(B_DPFULL), (uint32_t)j & 1u, abort_flag, p.status);
       tc_fence_after();

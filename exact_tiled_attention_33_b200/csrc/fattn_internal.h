@@ -22,7 +22,9 @@ struct FwdParams {
   float scale;      // softmax scale
   float scale_log2; // |scale| * log2(e), > 0 (a tiny positive value when scale == 0)
   int negate_scores;// 1 when scale < 0: the S product negates Q
-  int causal;
+  int win_left;     // attention window (see key_tile_range); causal is (-1, 0)
+  int win_right;
+  int reverse_tiles;// launch the query tiles with the most key tiles first
   uint32_t* status; // device status word
 };
 
@@ -44,9 +46,49 @@ struct BwdParams {
   int total_q, total_k;
   float scale;
   float scale_log2;
-  int causal;
+  int win_left, win_right;  // attention window (see key_tile_range)
+  int reverse_tiles;        // dQ pass: launch the query tiles with the most key tiles first
   uint32_t* status;
 };
+
+// Attention window.  Within one sequence of Lq queries and Lk keys (diag = Lk - Lq, the
+// bottom-right alignment), key j is allowed for query i iff
+//   i + diag - win_left <= j <= i + diag + win_right   and 0 <= j < Lk,
+// a negative bound meaning no bound on that side: causal is (-1, 0), full is (-1, -1).
+// The callers keep every bound below the sequence lengths and Lq + Lk < 2^31, so none of
+// the sums below overflows.
+
+// Key tiles (of BN keys) that query rows [q_first, q_last] may see: tiles
+// [*begin, *begin + *count).
+__host__ __device__ inline void key_tile_range(int q_first, int q_last, int Lk, int diag,
+                                               int win_left, int win_right, int BN, int* begin,
+                                               int* count) {
+  const int hi = win_right >= 0 ? min(Lk - 1, q_last + diag + win_right) : Lk - 1;
+  const int lo = win_left >= 0 ? max(0, q_first + diag - win_left) : 0;
+  if (hi < lo) {
+    *begin = 0;
+    *count = 0;
+  } else {
+    *begin = lo / BN;
+    *count = hi / BN - lo / BN + 1;
+  }
+}
+
+// Query tiles (of BM rows) that may see keys [k_first, k_last]: tiles
+// [*begin, *begin + *count).
+__host__ __device__ inline void query_tile_range(int k_first, int k_last, int Lq, int diag,
+                                                 int win_left, int win_right, int BM, int* begin,
+                                                 int* count) {
+  const int lo = win_right >= 0 ? max(0, k_first - diag - win_right) : 0;
+  const int hi = win_left >= 0 ? min(Lq - 1, k_last - diag + win_left) : Lq - 1;
+  if (hi < lo) {
+    *begin = 0;
+    *count = 0;
+  } else {
+    *begin = lo / BM;
+    *count = hi / BM - lo / BM + 1;
+  }
+}
 
 enum class LaunchResult { kOk, kUnsupported, kCudaError };
 

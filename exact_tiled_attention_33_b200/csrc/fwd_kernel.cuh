@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(384, 1)
   // each head is launched first.
   const int h = blockIdx.y;
   const int bz = blockIdx.z;
-  const int tile = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  const int tile = p.reverse_tiles ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
     q_row0 = p.cu_q[bz];
@@ -109,13 +109,10 @@ __global__ void __launch_bounds__(384, 1)
   }
   const int q0 = tile * BM;
   if (q0 >= Lq) return;  // uniform for the whole CTA
-  const int diag = Lk - Lq;  // key j is allowed for row i iff j <= i + diag (causal)
-  const int kv_tiles_all = (Lk + BN - 1) / BN;
-  int n_kv = kv_tiles_all;
-  if (p.causal) {
-    const int j_last = min(q0 + BM - 1, Lq - 1) + diag;
-    n_kv = (j_last < 0) ? 0 : min(kv_tiles_all, j_last / BN + 1);
-  }
+  const int diag = Lk - Lq;  // bottom-right alignment of the window (causal: j <= i + diag)
+  const int wl = p.win_left, wr = p.win_right;
+  int j0, n_kv;               // key tiles j0 .. j0 + n_kv - 1
+  key_tile_range(q0, min(q0 + BM - 1, Lq - 1), Lk, diag, wl, wr, BN, &j0, &n_kv);
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
@@ -159,12 +156,12 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(BAR(C::B_KFULL + s), C::TILE);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(&tmK, BAR(C::B_KFULL + s), sbase + C::OFF_K + s * C::TILE + c * C::CHUNK,
-                      c * 64, h, k_row0 + j * BN, bcoord);
+                      c * 64, h, k_row0 + (j0 + j) * BN, bcoord);
         mbar_wait(BAR(C::B_VEMPTY + s), ph ^ 1u, abort_flag, p.status);
         mbar_arrive_expect_tx(BAR(C::B_VFULL + s), C::TILE);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(&tmV, BAR(C::B_VFULL + s), sbase + C::OFF_V + s * C::TILE + c * C::CHUNK,
-                      c * 64, h, k_row0 + j * BN, bcoord);
+                      c * 64, h, k_row0 + (j0 + j) * BN, bcoord);
       }
     }
     __syncwarp();
@@ -240,14 +237,17 @@ __global__ void __launch_bounds__(384, 1)
       tmem_wait_ld();
       reg_fence(sr);
 
-      const int k0 = j * BN + 64 * half;  // first key of this thread's columns
-      const bool need_mask = (j * BN + BN > Lk) || (p.causal && (j * BN + BN - 1 > q0 + diag));
+      const int kt = (j0 + j) * BN;       // first key of the tile
+      const int k0 = kt + 64 * half;      // first key of this thread's columns
+      const bool need_mask = (kt + BN > Lk) || (wr >= 0 && kt + BN - 1 > q0 + diag + wr) ||
+                             (wl >= 0 && kt < q0 + BM - 1 + diag - wl);
       if (need_mask) {
-        int lim = Lk - k0;  // columns e < lim are allowed
-        if (p.causal) lim = min(lim, i + diag - k0 + 1);
+        // allowed columns: lo <= e < lim
+        const int lim = wr >= 0 ? min(Lk - k0, i + diag + wr - k0 + 1) : Lk - k0;
+        const int lo = wl >= 0 ? i + diag - wl - k0 : 0;
 #pragma unroll
         for (int e = 0; e < 64; ++e)
-          if (e >= lim) sr[e] = __float_as_uint(-INFINITY);
+          if (e >= lim || e < lo) sr[e] = __float_as_uint(-INFINITY);
       }
       // partial row maximum (tree of 3-input maxima), combined with the other half's
       float t1[22];

@@ -46,6 +46,7 @@ class Workload:
     seqlens: Optional[tuple] = None  # varlen only
     qk_mult: float = 1.0
     scale: Optional[float] = None    # default 1/sqrt(d)
+    window: Optional[tuple] = None   # sliding window (left, right); None: `causal` decides
 
     @property
     def varlen(self) -> bool:
@@ -68,11 +69,12 @@ class Workload:
         return np.concatenate([[0], np.cumsum(self.seqlens)]).astype(np.int32)
 
     def fwd_flops(self) -> float:
-        """4·B·H·N²·d forward FLOPs, halved when causal; varlen sums per sequence."""
-        if self.varlen:
-            f = sum(4.0 * self.H * L * L * self.d for L in self.seqlens)
-        else:
-            f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        """4·B·H·N²·d forward FLOPs, halved when causal; varlen sums per sequence.  With a
+        sliding window: 4·d FLOPs per allowed (query, key) pair, counted exactly."""
+        lens = self.seqlens if self.varlen else (self.N,) * self.B
+        if self.window is not None:
+            return sum(4.0 * self.H * self.d * window_pairs(L, L, self.window) for L in lens)
+        f = sum(4.0 * self.H * L * L * self.d for L in lens)
         return f / 2 if self.causal else f
 
     def bwd_flops(self) -> float:
@@ -93,7 +95,22 @@ class Workload:
             out.update(B=self.B, N=self.N)
         if self.qk_mult != 1.0:
             out["qk_mult"] = self.qk_mult
+        if self.window is not None:
+            out["window"] = list(self.window)
         return out
+
+
+def window_pairs(Lq: int, Lk: int, window) -> int:
+    """Number of (query, key) pairs a sliding window (left, right) admits in one sequence
+    (bottom-right aligned; a negative bound is no bound).  Used to size FLOP counts."""
+    left, right = window
+    diag = Lk - Lq
+    total = 0
+    for i in range(Lq):
+        lo = 0 if left < 0 else max(0, i + diag - left)
+        hi = Lk - 1 if right < 0 else min(Lk - 1, i + diag + right)
+        total += max(0, hi - lo + 1)
+    return total
 
 
 def varlen_lengths_64(seed: int = 3) -> tuple:
@@ -128,6 +145,12 @@ def _registry():
                      seed=4))
         add(Workload(f"long_peaky_{c}", B=2, H=32, N=16384, d=128, dtype="bf16",
                      causal=causal, seed=4, qk_mult=4.0))
+    # sliding-window (local) attention at the long-context size: each query sees the 4096
+    # keys ending at its own position (a causal window of 4096), and a symmetric window
+    add(Workload("long_local_w4096", B=2, H=32, N=16384, d=128, dtype="bf16", causal=True,
+                 seed=4, window=(4095, 0)))
+    add(Workload("long_local_sym512", B=2, H=32, N=16384, d=128, dtype="bf16", causal=False,
+                 seed=4, window=(256, 256)))
     # profiling size of the long-context kernel path: inputs larger than L2 (4 x 67 MB),
     # about 1 GB on the device in total
     add(Workload("profile_causal_8k", B=1, H=32, N=8192, d=128, dtype="bf16", causal=True,
@@ -143,13 +166,15 @@ def get(name: str) -> Workload:
 
 
 def custom(name="custom", *, B=1, N=128, H=1, d=64, dtype="bf16", causal=False, seed=0,
-           seqlens=None, qk_mult=1.0, scale=None) -> Workload:
+           seqlens=None, qk_mult=1.0, scale=None, window=None) -> Workload:
     """An ad-hoc workload (ragged sizes, edge cases) built with the same recipe."""
+    window = None if window is None else (int(window[0]), int(window[1]))
     if seqlens is not None:
         return Workload(name, H=H, d=d, dtype=dtype, causal=causal, seed=seed,
-                        seqlens=tuple(int(x) for x in seqlens), qk_mult=qk_mult, scale=scale)
+                        seqlens=tuple(int(x) for x in seqlens), qk_mult=qk_mult, scale=scale,
+                        window=window)
     return Workload(name, B=B, N=N, H=H, d=d, dtype=dtype, causal=causal, seed=seed,
-                    qk_mult=qk_mult, scale=scale)
+                    qk_mult=qk_mult, scale=scale, window=window)
 
 
 def generate(w: Workload, with_grad_out: bool = True):

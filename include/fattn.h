@@ -81,8 +81,8 @@ int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* l
                   int max_seqlen_k, int H, int d, float scale, int causal, int num_seqs,
                   int total_q, int total_k, int dtype, void* stream);
 
-/* Workspace bytes the dense backward needs: an fp32 dQ accumulator [B,N,H,d] and
- * D = rowsum(dO ∘ O) [B,H,N] fp32, each 256-byte aligned. */
+/* Workspace bytes the dense backward needs: D = rowsum(dO ∘ O) [B,H,N] fp32, rounded up
+ * to a multiple of 256 bytes (dQ, dK and dV are written directly, with no atomics). */
 size_t fa_bwd_workspace_size(int B, int N, int H, int d);
 
 /* Dense backward: recomputes P from q, k and lse (as written by fa_fwd with the same
@@ -94,8 +94,8 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            float scale, int causal, void* workspace, size_t workspace_bytes, int dtype,
            void* stream);
 
-/* Workspace bytes the varlen backward needs (fp32 dQ accumulator [total_q,H,d] and D
- * [H,total_q]). */
+/* Workspace bytes the varlen backward needs: D [H,total_q] fp32, rounded up to a
+ * multiple of 256 bytes. */
 size_t fa_varlen_bwd_workspace_size(int total_q, int H, int d);
 
 /* Varlen backward; arguments as fa_varlen_fwd plus the gradient buffers. */
@@ -104,6 +104,46 @@ int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, co
                   const int* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k, int H, int d,
                   float scale, int causal, int num_seqs, int total_q, int total_k,
                   void* workspace, size_t workspace_bytes, int dtype, void* stream);
+
+/* ---------------------------------------------------------------- local attention
+ * Sliding-window (local) attention: the variant listed by the page "FlashAttention技术
+ * 深度解析" (pwwt.cn/news/595117) in its CUDA backend feature table and in its section on
+ * local attention, which give no parameters.  Read here as a window around the same
+ * bottom-right-aligned diagonal the causal mask uses: key j is allowed for query i iff
+ *
+ *     i + (Lk - Lq) - window_left  <=  j  <=  i + (Lk - Lq) + window_right,
+ *
+ * a negative bound meaning no bound on that side.  (-1, 0) is the causal mask, (-1, -1)
+ * full attention, (w, 0) causal attention over the last w + 1 keys.  Key tiles that no
+ * row of a query tile may see are skipped, so the work grows with the window, not with
+ * the sequence.  Rows whose window holds no key behave like fully masked causal rows
+ * (O = 0, LSE = +inf, no gradient contribution).  Bounds at or above the sequence
+ * lengths are the same as no bound.  With any bound other than the causal one,
+ * max_seqlen_q + max_seqlen_k (dense: 2N) must be < 2^31 (FA_ERR_UNSUPPORTED otherwise).
+ * Every other argument, layout, limit and error is that of the call without _local. */
+int fa_fwd_local(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N,
+                 int H, int d, float scale, int window_left, int window_right, int dtype,
+                 void* stream);
+
+int fa_varlen_fwd_local(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int max_seqlen_q,
+                        int max_seqlen_k, int H, int d, float scale, int window_left,
+                        int window_right, int num_seqs, int total_q, int total_k, int dtype,
+                        void* stream);
+
+/* Backward of fa_fwd_local: lse must come from fa_fwd_local with the same scale and
+ * window; workspace as for fa_bwd. */
+int fa_bwd_local(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d,
+                 float scale, int window_left, int window_right, void* workspace,
+                 size_t workspace_bytes, int dtype, void* stream);
+
+int fa_varlen_bwd_local(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int max_seqlen_q,
+                        int max_seqlen_k, int H, int d, float scale, int window_left,
+                        int window_right, int num_seqs, int total_q, int total_k,
+                        void* workspace, size_t workspace_bytes, int dtype, void* stream);
 
 /* Allocation-free dense backward (no counterpart on the source pages: an interface
  * addition).  Same arguments and results as fa_bwd, without the workspace: the D vector

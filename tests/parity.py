@@ -63,17 +63,18 @@ def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, scale_ref=None,
     return float(err.max() / max(ref_max, 1e-30))
 
 
-def o16_term_in_d(q, k, v, do, scale, causal, dtype):
+def o16_term_in_d(q, k, v, do, scale, causal, dtype, window=None):
     """First-order bound on what computing D = rowsum(dO ∘ O) from the 16-bit O (the only
     O the backward pass receives) changes in dQ and dK, per element.
 
     |δD_i| <= Σ_c |dO_ic| · ½ulp(O_ic);  δdS_ij = -P_ij δD_i, so
     |δdQ_ic| <= scale |δD_i| Σ_j P_ij |K_jc|  and  |δdK_jc| <= scale Σ_i P_ij |δD_i| |Q_ic|.
-    Only significant for degenerate sizes (N <= 2) where the exact gradient nearly cancels.
+    Only significant where the exact gradient nearly cancels: degenerate sizes (N <= 2) or
+    a window of one key per row, where every exact gradient of Q and K is zero.
     """
     import oracle
-    o, _ = oracle.attention_forward(q, k, v, scale, causal)
-    pm = oracle.softmax_probs(q, k, scale, causal)
+    o, _ = oracle.attention_forward(q, k, v, scale, causal, window=window)
+    pm = oracle.softmax_probs(q, k, scale, causal, window=window)
     dd = (np.abs(do) * half_ulp(o, dtype)).sum(axis=1)
     bq = abs(scale) * dd[:, None] * (pm @ np.abs(k))
     bk = abs(scale) * (pm * dd[:, None]).T @ np.abs(q)

@@ -104,3 +104,20 @@ def test_empty_problems_are_noops(lib):
     assert lib.fa_fwd(None, None, None, None, None, 1, 0, 1, 64, 0.1, 1, 1, None) == _lib.FA_OK
     assert lib.fa_varlen_fwd(None, None, None, None, None, None, None, 0, 0, 1, 64, 0.1, 0, 0, 0,
                              0, 0, None) == _lib.FA_OK
+
+
+def test_local_window_validation(lib):
+    # Windowed calls keep index sums in int32: a bounded window with 2N >= 2^31 is refused
+    # on the host before any CUDA call; zero sizes stay no-ops.
+    n = 1 << 30
+    assert lib.fa_fwd_local(P, P, P, P, P, 1, n, 1, 64, 0.1, 5, 0, 0, None) == \
+        _lib.FA_ERR_UNSUPPORTED
+    assert b"window" in lib.fa_last_error()
+    assert lib.fa_bwd_local(P, P, P, P, P, P, P, P, P, 1, n, 1, 64, 0.1, -1, 7, P, 1 << 40, 0,
+                            None) == _lib.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_local(None, None, None, None, None, 0, 128, 1, 64, 0.1, 3, 3, 0, None) == \
+        _lib.FA_OK
+    assert lib.fa_varlen_fwd_local(P, P, P, P, P, P, P, 10, 10, 1, 64, 0.1, 4, 4, -2, 10, 10, 0,
+                                   None) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_varlen_bwd_local(P, P, P, P, P, P, P, P, P, P, P, 10, 10, 1, 96, 0.1, 4, 4, 1,
+                                   10, 10, P, 1 << 20, 0, None) == _lib.FA_ERR_UNSUPPORTED

@@ -220,3 +220,29 @@ def test_fma_pipe_exp2_accuracy():
     assert np.all(np.abs(ys[~ok]) <= 2.0 ** -124)  # clamped / denormal boundary: ~1e-38
     cuda = torch.exp2(x).double().cpu().numpy()
     assert np.abs(ys[ok] / cuda[ok] - 1.0).max() <= 1.2e-4
+
+
+def test_call_from_fresh_host_thread():
+    # A host thread that has made no CUDA runtime call (as autograd worker threads may
+    # not have) can call the library: it makes the device context current itself.
+    import threading
+    w = wl.custom("thread", B=1, N=200, H=2, d=64, causal=True, seed=14)
+    t = wl.generate(w, with_grad_out=False)
+    q, k, v = (t[x].to(DEV) for x in ("q", "k", "v"))
+    o_ref, l_ref = fa.fwd(q, k, v, None, True)
+    o, lse = torch.empty_like(o_ref), torch.empty_like(l_ref)
+    torch.cuda.synchronize()
+    err = []
+
+    def worker():
+        try:
+            fa.fwd(q, k, v, None, True, out=o, lse=lse)
+        except Exception as e:  # reported to the main thread
+            err.append(e)
+
+    th = threading.Thread(target=worker)
+    th.start()
+    th.join()
+    assert not err, err
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)

@@ -236,3 +236,13 @@ def test_planted_window_mistakes_are_caught(monkeypatch):
                 caught += 1
         monkeypatch.setattr(ref, "allowed_mask", real)
         assert caught > 0, mutant.__name__
+
+
+@pytest.mark.parametrize("Lq,Lk,win", [(50, 50, (7, 0)), (30, 70, (5, 9)), (70, 30, (-1, 4)),
+                                       (40, 40, (-1, -1)), (25, 60, (3, -1))])
+def test_flop_count_pairs_match_mask(Lq, Lk, win):
+    # The workloads' FLOP sizing counts the same pairs the oracle's mask admits.
+    from exact_tiled_attention_33_b200 import workloads
+    from oracle.attn_ref import allowed_mask
+    assert workloads.window_pairs(Lq, Lk, win) == int(allowed_mask(np.arange(Lq), Lq, Lk,
+                                                                   False, win).sum())
