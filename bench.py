@@ -39,9 +39,11 @@ UNIT = "TFLOPS"
 FALLBACK_PEAK_TFLOPS = 1590.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
 BWD_SOURCES = ["exact_tiled_attention_33_b200/csrc/bwd_kernel.cuh",
-               "exact_tiled_attention_33_b200/csrc/sm100.cuh"]
+               "exact_tiled_attention_33_b200/csrc/sm100.cuh",
+               "exact_tiled_attention_33_b200/csrc/fattn_internal.h"]
 FWD_SOURCES = ["exact_tiled_attention_33_b200/csrc/fwd_kernel.cuh",
-               "exact_tiled_attention_33_b200/csrc/sm100.cuh"]
+               "exact_tiled_attention_33_b200/csrc/sm100.cuh",
+               "exact_tiled_attention_33_b200/csrc/fattn_internal.h"]
 
 
 # ------------------------------------------------------------------ helpers (CPU-testable)
@@ -347,7 +349,7 @@ def run_fattn(args, w):
         "bound": "tensor", "achieved": bwd_ach, "peak": peak_sust, "unit": "TFLOP/s",
         "frac": bwd_ach / peak_sust,
         "peak_source": f"bf16_tflops_sustained ({peak_src})",
-        "traffic": read_traffic("fa_bwd_kernel", wr.name, bwd_sha),
+        "traffic": read_traffic("fa_bwd", wr.name, bwd_sha),
         "flops_per_launch": 2.5 * f_fwd}
     fwd_roof = {"kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": fwd_ach,
                 "peak": peak_sust, "unit": "TFLOP/s", "frac": fwd_ach / peak_sust,
