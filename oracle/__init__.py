@@ -7,6 +7,8 @@ from .attn_ref import (  # noqa: F401
     attention_backward_bhsd,
     attention_forward,
     attention_forward_bhsd,
+    decode_attention,
+    kv_cache_gather,
     softmax_probs,
     varlen_attention_backward,
     varlen_attention_forward,

@@ -257,3 +257,56 @@ def varlen_attention_backward(q, k, v, do, cu_seqlens_q, cu_seqlens_k, scale, ca
                                          do[q0:q1, h], scale, causal, window=window)
             dq[q0:q1, h], dk[k0:k1, h], dv[k0:k1, h] = a, b, c
     return dq, dk, dv
+
+
+# ------------------------------------------------------------------ KV-cache decode
+# The pages list KV caches for incremental decoding and paged KV caches as supported
+# features without giving their interface (page "FlashAttention技术深度解析"
+# (pwwt.cn/news/595117): Hopper row of the CUDA backend feature table, the causal-mask
+# section on KV-cache updates and incremental decoding, and the section on KV-cache
+# management with paged caches).  Read here as: one decode step attends Nq new query
+# tokens per sequence to that sequence's cached keys and values; the new tokens are the
+# last Nq positions of the cache, so masks are bottom-right aligned as everywhere else.
+
+def kv_cache_gather(pages, block_table_row, length):
+    """Rows 0..length-1 of one sequence's cache, from a paged cache.
+
+    pages: [num_pages, page_size, H, d]; block_table_row[i] is the page that holds the
+    sequence's rows i*page_size .. (i+1)*page_size - 1.  Returns [length, H, d].
+    """
+    pages = np.asarray(pages)
+    page_size = pages.shape[1]
+    idx = np.arange(length, dtype=np.int64)
+    table = np.asarray(block_table_row, dtype=np.int64)
+    return pages[table[idx // page_size], idx % page_size]
+
+
+def decode_attention(q, k_cache, v_cache, cache_seqlens, scale, causal, block_table=None,
+                     window=None):
+    """One decode step over a KV cache: O [B, Nq, H, d] and LSE [B, H, Nq] (float64).
+
+    q: [B, Nq, H, d].  Contiguous cache (block_table None): k_cache, v_cache are
+    [B, capacity, H, d] and sequence b holds rows 0..cache_seqlens[b]-1.  Paged cache:
+    k_cache, v_cache are [num_pages, page_size, H, d] and block_table [B, max_blocks]
+    maps each sequence's logical pages to physical ones.  Rows of the cache at or past
+    cache_seqlens[b] are never read.  Query row r of sequence b sits at position
+    cache_seqlens[b] - Nq + r; `causal` / `window` are applied as in attention_forward.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, Nq, H, d = q.shape
+    out = np.zeros((B, Nq, H, d), dtype=np.float64)
+    lse = np.zeros((B, H, Nq), dtype=np.float64)
+    for b in range(B):
+        L = int(cache_seqlens[b])
+        if block_table is None:
+            kb = np.asarray(k_cache[b, :L], dtype=np.float64)
+            vb = np.asarray(v_cache[b, :L], dtype=np.float64)
+        else:
+            kb = np.asarray(kv_cache_gather(k_cache, block_table[b], L), dtype=np.float64)
+            vb = np.asarray(kv_cache_gather(v_cache, block_table[b], L), dtype=np.float64)
+        for h in range(H):
+            o, l = attention_forward(q[b, :, h], kb[:, h], vb[:, h], scale, causal,
+                                     window=window)
+            out[b, :, h] = o
+            lse[b, h] = l
+    return out, lse
