@@ -393,6 +393,212 @@ def run_fattn(args, w):
     return 0
 
 
+def run_decode_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from exact_tiled_attention_33_b200 import workloads as wl
+    g = wl.generate_decode(w)
+    n = 1
+    dt, _, _ = oracle_decode_seconds(w, g, n)
+    while dt < 0.5 and n < w.H:
+        n = min(w.H, n * 2)
+        dt, _, _ = oracle_decode_seconds(w, g, n)
+    reps = max(1, int(0.5 / max(dt, 1e-3)))
+    for _ in range(args.warmup):
+        oracle_decode_seconds(w, g, n, reps)
+    tot_t = tot_b = 0.0
+    threads = os.cpu_count()
+    for _ in range(args.steps):
+        dt, by, threads = oracle_decode_seconds(w, g, n, reps)
+        tot_t += dt
+        tot_b += by
+    value = tot_b / tot_t / 1e9
+    sample = (f"sequence 0 ({w.cache_lens[0]} cached rows), {n} heads x {reps} passes, "
+              f"fp64 oracle decode, per step")
+    print(json.dumps({"impl": "reference", "metric": DECODE_METRIC, "value": value,
+                      "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+                      "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                      "dtype": "f64", "data": "synthetic",
+                      "config": dict(w.describe(), parallelism=f"dp{world}"),
+                      "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads,
+                                       "kind": "oracle", "sample": sample},
+                      "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                              "d2h_bytes_per_step": 0}}), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ KV-cache decode arm
+DECODE_METRIC = "KV-cache decode: HBM GB/s of the cached K/V read (and attention TFLOPS)"
+DECODE_SOURCES = ["exact_tiled_attention_33_b200/csrc/decode_kernel.cuh",
+                  "exact_tiled_attention_33_b200/csrc/sm100.cuh",
+                  "exact_tiled_attention_33_b200/csrc/fattn_internal.h"]
+
+
+def oracle_decode_seconds(w, g, n_heads: int, reps: int = 1):
+    """fp64 oracle decode of sequence 0 for the first n_heads heads, `reps` times:
+    (seconds, algorithmic K/V bytes of that work, threads)."""
+    import oracle
+    import torch
+    L = w.cache_lens[0]
+    if w.page_size:
+        row = g["block_table"][0].numpy()
+        kb = torch.from_numpy(oracle.kv_cache_gather(g["k_pages"].view(torch.int16).numpy(),
+                                                     row, L)).view(g["q"].dtype)
+        vb = torch.from_numpy(oracle.kv_cache_gather(g["v_pages"].view(torch.int16).numpy(),
+                                                     row, L)).view(g["q"].dtype)
+    else:
+        kb, vb = g["k_cache"][0, :L], g["v_cache"][0, :L]
+    q = g["q"][0].double().numpy()
+    kb, vb = kb[:, :n_heads].double().numpy(), vb[:, :n_heads].double().numpy()
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        for h in range(n_heads):
+            oracle.attention_forward(q[:, h], kb[:, h], vb[:, h], w.softmax_scale, w.causal)
+    dt = time.perf_counter() - t0
+    return dt, 2.0 * L * n_heads * w.d * 2 * reps, os.cpu_count()
+
+
+def run_decode(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from exact_tiled_attention_33_b200 import _lib
+    from exact_tiled_attention_33_b200 import attention as fa
+    from exact_tiled_attention_33_b200 import workloads as wl
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    wr = wl.DecodeWorkload(**{**w.__dict__, "seed": w.seed + rank})
+    host = wl.generate_decode(wr)
+    lib = _lib.load()
+    q = host["q"].to(dev)
+    lens = host["cache_seqlens"].to(dev)
+    B, Nq, H, d = q.shape
+    max_len = max(wr.cache_lens)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    ws = fa.decode_workspace(B, Nq, H, d, max_len, dev)
+    wsp, wsn = (0, 0) if ws is None else (ws.data_ptr(), ws.numel())
+    dtype = _lib.FA_BF16 if wr.dtype == "bf16" else _lib.FA_FP16
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    if wr.page_size:
+        kc, vc = host["k_pages"].to(dev), host["v_pages"].to(dev)
+        bt = host["block_table"].to(dev)
+
+        def step():
+            _lib.check(lib.fa_decode_paged(q.data_ptr(), kc.data_ptr(), vc.data_ptr(),
+                                           o.data_ptr(), lse.data_ptr(), bt.data_ptr(),
+                                           lens.data_ptr(), B, Nq, H, d, wr.page_size,
+                                           kc.shape[0], bt.shape[1], max_len,
+                                           wr.softmax_scale, int(wr.causal), wsp, wsn, dtype, sh),
+                       "fa_decode_paged")
+    else:
+        kc, vc = host["k_cache"].to(dev), host["v_cache"].to(dev)
+
+        def step():
+            _lib.check(lib.fa_decode(q.data_ptr(), kc.data_ptr(), vc.data_ptr(), o.data_ptr(),
+                                     lse.data_ptr(), lens.data_ptr(), B, Nq, H, d, wr.capacity,
+                                     max_len, wr.softmax_scale, int(wr.causal), wsp, wsn, dtype,
+                                     sh), "fa_decode")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert lib.fa_get_device_status(sh) == 0, "device status after warm-up"
+    # ---- timed region: the cache (>= 1 GB) is far larger than the 126 MB L2
+    sampler = ClockSampler(local) if rank == 0 else None
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler is not None else None
+    assert lib.fa_get_device_status(sh) == 0, "device status in timed region"
+    max_s = max_over_ranks(t0.elapsed_time(t1) / 1e3, world)
+    per = statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3
+    nbytes = wr.bytes_moved()
+    value = nbytes * args.steps * world / max_s / 1e9
+    splits_ws = lib.fa_decode_workspace_size(B, Nq, H, d, max_len)
+
+    e2e = None
+    if not args.no_e2e:
+        # per step: H2D of the new tokens' q, the decode call, D2H of O and LSE (the cache
+        # stays resident on the device, as a KV cache does between steps)
+        hq = host["q"].pin_memory()
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        n_e2e = max(2, min(args.steps, 10))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_s = max_over_ranks(a.elapsed_time(b_) / 1e3, world)
+        e2e = {"value": nbytes * n_e2e * world / e2e_s / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": hq.numel() * hq.element_size(),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size() + hl.numel() * hl.element_size(),
+               "steps": n_e2e}
+
+    _, _, hbm, src = load_peaks()
+    sha = sources_sha(DECODE_SOURCES)
+    roofline = {"kernel": "fa_decode_kernel" + (" + fa_decode_combine_kernel" if splits_ws else ""),
+                "bound": "hbm", "achieved": nbytes / per / 1e9, "peak": hbm, "unit": "GB/s",
+                "frac": nbytes / per / 1e9 / hbm, "peak_source": f"hbm_gbs ({src})",
+                "traffic": read_traffic("fa_decode", wr.name, sha), "bytes_per_launch": nbytes}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        reps = 1
+        dt, by, threads = oracle_decode_seconds(wr, host, H, reps)
+        while dt < 5.0:
+            reps *= 2
+            dt, by, threads = oracle_decode_seconds(wr, host, H, reps)
+        cpu = {"value": by / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"sequence 0 ({wr.cache_lens[0]} cached rows), all {H} heads, "
+                         f"{reps} passes, fp64 oracle decode ({dt:.1f} s)"}
+    if rank == 0:
+        line = {"metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * max_s / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": wr.dtype, "data": "synthetic",
+                "config": dict(wr.describe(), seed=w.seed, parallelism=f"dp{world}",
+                               l2="cache larger than L2, no flush"),
+                "tflops": wr.flops() * args.steps * world / max_s / 1e12,
+                "gpu_launches": (2 if splits_ws else 1) * args.steps,
+                "roofline": roofline, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -405,6 +611,10 @@ def main(argv=None):
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3) if args.impl == "fattn" else args.warmup
     from exact_tiled_attention_33_b200 import workloads as wl
+    if args.workload in wl.DECODE_WORKLOADS:
+        if args.impl == "reference":
+            return run_decode_reference(args, wl.get_decode(args.workload))
+        return run_decode(args, wl.get_decode(args.workload))
     w = wl.get(args.workload)
     if args.impl == "reference":
         return run_reference(args, w)

@@ -40,6 +40,11 @@ SIGNATURES = {
                           _i, _vp, _sz, _i, _vp]),
     "fa_varlen_bwd_local": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
                                  _i, _i, _f, _i, _i, _i, _i, _i, _vp, _sz, _i, _vp]),
+    "fa_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "fa_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _sz, _i,
+                       _vp]),
+    "fa_decode_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                             _f, _i, _vp, _sz, _i, _vp]),
     "fa_get_device_status": (_i, [_vp]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
     "fa_last_error": (ctypes.c_char_p, []),

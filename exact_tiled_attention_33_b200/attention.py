@@ -263,6 +263,81 @@ def varlen_bwd_local(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seql
     return dq, dk, dv
 
 
+# ------------------------------------------------------------------ KV-cache decode
+# One incremental-decoding step over a KV cache (page "FlashAttention技术深度解析"
+# (pwwt.cn/news/595117): KV caches for incremental decoding, paged KV caches).  The Nq
+# new tokens are the last Nq positions of each sequence's cache.
+
+def decode_workspace(B, Nq, H, d, max_seqlen_k, device) -> Optional[torch.Tensor]:
+    n = _lib.load().fa_decode_workspace_size(B, Nq, H, d, max_seqlen_k)
+    return None if n == 0 else torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _check_seqlens(t, B, device, name):
+    if t.dtype != torch.int32 or t.device != device or not t.is_contiguous() or t.dim() != 1 \
+            or t.numel() != B:
+        raise ValueError(f"{name} must be a contiguous int32 [B] tensor on q's device")
+
+
+def decode(q, k_cache, v_cache, cache_seqlens, max_seqlen_k=None, softmax_scale=None,
+           causal=True, out=None, lse=None, workspace=None):
+    """Decode step over a contiguous cache (fa_decode).  q: [B, Nq, H, d];
+    k_cache, v_cache: [B, capacity, H, d]; cache_seqlens: int32 [B] on the device.
+    max_seqlen_k: host bound on the lengths (default: the capacity).
+    Returns (o [B, Nq, H, d], lse [B, H, Nq] fp32)."""
+    if q.dim() != 4 or k_cache.dim() != 4 or k_cache.shape != v_cache.shape or \
+            k_cache.shape[0] != q.shape[0] or k_cache.shape[2:] != q.shape[2:]:
+        raise ValueError("q must be [B, Nq, H, d] and the caches [B, capacity, H, d]")
+    dtype = _check(q, k_cache, v_cache)
+    B, Nq, H, d = q.shape
+    cap = k_cache.shape[1]
+    _check_seqlens(cache_seqlens, B, q.device, "cache_seqlens")
+    max_len = cap if max_seqlen_k is None else int(max_seqlen_k)
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
+    ws = decode_workspace(B, Nq, H, d, max_len, q.device) if workspace is None else workspace
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse_t),
+                           _ptr(cache_seqlens), B, Nq, H, d, cap, max_len, scale,
+                           int(bool(causal)), _ptr(ws), 0 if ws is None else ws.numel(), dtype,
+                           _stream(q))
+    _lib.check(st, "fa_decode")
+    return o, lse_t
+
+
+def decode_paged(q, k_pages, v_pages, block_table, cache_seqlens, max_seqlen_k=None,
+                 softmax_scale=None, causal=True, out=None, lse=None, workspace=None):
+    """Decode step over a paged cache (fa_decode_paged).  q: [B, Nq, H, d];
+    k_pages, v_pages: [num_pages, page_size, H, d]; block_table: int32 [B, max_blocks];
+    cache_seqlens: int32 [B].  Returns (o, lse) as decode()."""
+    if q.dim() != 4 or k_pages.dim() != 4 or k_pages.shape != v_pages.shape or \
+            k_pages.shape[2:] != q.shape[2:]:
+        raise ValueError("q must be [B, Nq, H, d] and the pages [num_pages, page_size, H, d]")
+    dtype = _check(q, k_pages, v_pages)
+    B, Nq, H, d = q.shape
+    num_pages, page_size = k_pages.shape[0], k_pages.shape[1]
+    if block_table.dtype != torch.int32 or block_table.device != q.device or \
+            block_table.dim() != 2 or block_table.shape[0] != B or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous int32 [B, max_blocks] tensor")
+    _check_seqlens(cache_seqlens, B, q.device, "cache_seqlens")
+    max_blocks = block_table.shape[1]
+    max_len = max_blocks * page_size if max_seqlen_k is None else int(max_seqlen_k)
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
+    ws = decode_workspace(B, Nq, H, d, max_len, q.device) if workspace is None else workspace
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(o), _ptr(lse_t),
+                                 _ptr(block_table), _ptr(cache_seqlens), B, Nq, H, d, page_size,
+                                 num_pages, max_blocks, max_len, scale, int(bool(causal)),
+                                 _ptr(ws), 0 if ws is None else ws.numel(), dtype, _stream(q))
+    _lib.check(st, "fa_decode_paged")
+    return o, lse_t
+
+
 def device_status(stream: Optional[int] = None) -> int:
     """Synchronise and return the library status word (0 = ok, 4 = a wait timed out)."""
     lib = _lib.load()

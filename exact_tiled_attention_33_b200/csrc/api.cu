@@ -497,6 +497,133 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                     (cudaStream_t)stream);
 }
 
+// ------------------------------------------------------------------ KV-cache decode
+namespace {
+
+// Split policy: enough CTAs for about eight waves of 148 SMs, whole 128-key tiles per
+// split.  A fixed function of (B, H, max_seqlen_k), so fa_decode_workspace_size can size
+// the partial results without a device.
+constexpr long long kDecodeTargetCtas = 8LL * 148;
+
+void decode_splits(long long B, long long H, long long max_len, int* splits, int* chunk) {
+  const long long tiles = max_len > 0 ? (max_len + 127) / 128 : 1;
+  long long want = (kDecodeTargetCtas + B * H - 1) / (B * H);
+  want = std::max(1LL, std::min(want, tiles));
+  const long long per = (tiles + want - 1) / want;  // tiles per split
+  *splits = (int)((tiles + per - 1) / per);
+  *chunk = (int)(per * 128);
+}
+
+size_t decode_workspace(long long B, long long Nq, long long H, long long d, long long max_len) {
+  int splits = 1, chunk = 128;
+  decode_splits(B, H, max_len, &splits, &chunk);
+  if (splits <= 1) return 0;
+  const size_t rows = (size_t)B * Nq * H * splits;
+  return align256(rows * d * 4) + align256(rows * 4);
+}
+
+int decode_common(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* block_table, const int* cache_seqlens, int B, int Nq, int H, int d,
+                  long long cache_rows, long long cache_batches, int box_rows, int max_len,
+                  int page_size, int max_blocks, int num_pages, float scale, int causal,
+                  void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  if (int e = check_ptrs({q, o, lse, cache_seqlens})) return e;
+  if (int e = check_ptrs({k, v})) return e;
+  if (block_table != nullptr)
+    if (int e = check_ptrs({block_table})) return e;
+  DecParams p{};
+  p.q = q;
+  p.o = o;
+  p.lse = lse;
+  p.seqlens = cache_seqlens;
+  p.block_table = block_table;
+  p.B = B;
+  p.Nq = Nq;
+  p.H = H;
+  p.max_len = max_len;
+  p.page_size = page_size;
+  p.max_blocks = max_blocks;
+  p.num_pages = num_pages;
+  decode_splits(B, H, max_len, &p.splits, &p.chunk);
+  const size_t need = decode_workspace(B, Nq, H, d, max_len);
+  if (need > 0) {
+    if (workspace == nullptr) return fail(FA_ERR_INVALID_ARG, "decode needs a workspace");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(FA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (workspace_bytes < need)
+      return fail(FA_ERR_INVALID_ARG, "workspace too small (need " + std::to_string(need) + " bytes)");
+    const size_t rows = (size_t)B * Nq * H * p.splits;
+    p.o_part = static_cast<float*>(workspace);
+    p.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(rows * d * 4));
+  }
+  p.scale_log2 = scale * kLog2e;
+  p.win_left = -1;
+  p.win_right = causal ? 0 : -1;
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  CUtensorMap mk, mv;
+  if (int e = make_map(&mk, k, d, H, cache_rows, cache_batches, box_rows)) return e;
+  if (int e = make_map(&mv, v, d, H, cache_rows, cache_batches, box_rows)) return e;
+  return launch_result(launch_decode(d, dtype == FA_BF16, block_table != nullptr, mk, mv, p,
+                                     (cudaStream_t)stream));
+}
+
+int decode_check(int B, int Nq, int H, int d, int max_seqlen_k, float scale, int dtype) {
+  if (int e = check_common(H, d, dtype, scale)) return e;
+  if (B < 0 || Nq < 0 || max_seqlen_k < 0) return fail(FA_ERR_INVALID_ARG, "sizes must be >= 0");
+  if (Nq > kDecodeMaxQueries)
+    return fail(FA_ERR_UNSUPPORTED, "decode takes at most " + std::to_string(kDecodeMaxQueries) +
+                                        " query rows per sequence");
+  if (B > 65535) return fail(FA_ERR_UNSUPPORTED, "B must be <= 65535");
+  return FA_OK;
+}
+
+}  // namespace
+
+size_t fa_decode_workspace_size(int B, int Nq, int H, int d, int max_seqlen_k) {
+  if (B <= 0 || Nq <= 0 || H <= 0 || d <= 0 || max_seqlen_k < 0) return 0;
+  return decode_workspace(B, Nq, H, d, max_seqlen_k);
+}
+
+int fa_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+              const int* cache_seqlens, int B, int Nq, int H, int d, int cache_capacity,
+              int max_seqlen_k, float scale, int causal, void* workspace, size_t workspace_bytes,
+              int dtype, void* stream) {
+  g_last_error.clear();
+  if (int e = decode_check(B, Nq, H, d, max_seqlen_k, scale, dtype)) return e;
+  if (cache_capacity < 0) return fail(FA_ERR_INVALID_ARG, "cache_capacity must be >= 0");
+  if (max_seqlen_k > cache_capacity)
+    return fail(FA_ERR_INVALID_ARG, "max_seqlen_k exceeds cache_capacity");
+  if (B == 0 || Nq == 0 || H == 0) return FA_OK;
+  // An empty cache is never read; any aligned buffer stands in for the tensor map.
+  const bool empty = cache_capacity == 0;
+  return decode_common(q, empty ? q : k_cache, empty ? q : v_cache, o, lse, nullptr,
+                       cache_seqlens, B, Nq, H, d, empty ? 1 : cache_capacity, empty ? 1 : B,
+                       128, max_seqlen_k, 0, 0, 0, scale, causal, workspace, workspace_bytes,
+                       dtype, stream);
+}
+
+int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* o, float* lse,
+                    const int* block_table, const int* cache_seqlens, int B, int Nq, int H, int d,
+                    int page_size, int num_pages, int max_blocks_per_seq, int max_seqlen_k,
+                    float scale, int causal, void* workspace, size_t workspace_bytes, int dtype,
+                    void* stream) {
+  g_last_error.clear();
+  if (int e = decode_check(B, Nq, H, d, max_seqlen_k, scale, dtype)) return e;
+  if (page_size < 16 || (page_size & (page_size - 1)) != 0)
+    return fail(FA_ERR_UNSUPPORTED, "page_size must be a power of two >= 16");
+  if (num_pages <= 0 || max_blocks_per_seq <= 0)
+    return fail(FA_ERR_INVALID_ARG, "num_pages and max_blocks_per_seq must be >= 1");
+  if ((long long)max_blocks_per_seq * page_size < max_seqlen_k)
+    return fail(FA_ERR_INVALID_ARG, "max_seqlen_k exceeds max_blocks_per_seq * page_size");
+  if (B == 0 || Nq == 0 || H == 0) return FA_OK;
+  if (block_table == nullptr) return fail(FA_ERR_INVALID_ARG, "null pointer argument");
+  return decode_common(q, k_pages, v_pages, o, lse, block_table, cache_seqlens, B, Nq, H, d,
+                       page_size, num_pages, std::min(page_size, 128), max_seqlen_k, page_size,
+                       max_blocks_per_seq, num_pages, scale, causal, workspace, workspace_bytes,
+                       dtype, stream);
+}
+
 int fa_get_device_status(void* stream) {
   g_last_error.clear();
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
@@ -511,6 +638,9 @@ int fa_get_device_status(void* stream) {
     e = cudaMemcpy(sp, &zero, sizeof(zero), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(e, "clear status word");
     if (word & kDevTimeout) return fail(FA_ERR_TIMEOUT, "a kernel wait timed out");
+    if (word & kDevBadCache)
+      return fail(FA_ERR_INVALID_ARG,
+                  "a decode call saw a cache length above its bounds or a page id out of range");
     if (word & kDevSmemAlign)
       return fail(FA_ERR_UNSUPPORTED, "dynamic shared memory base not 1024-byte alignable");
   }

@@ -1,0 +1,417 @@
+// KV-cache decode for sm_100a: a few new query tokens per sequence attend to the keys and
+// values that sequence has cached, in a contiguous cache [B, capacity, H, d] or a paged
+// cache [num_pages, page_size, H, d] addressed through a block table.
+//
+// Method (what is computed): the same exact softmax attention as the forward kernel, with
+// the running maximum and rescaled running sum of the page "FlashAttention实战：如何在
+// A100上实现3倍加速的Transformer训练" §3.1 applied twice: across the key tiles a CTA
+// streams, and across the CTAs ("splits") that share one sequence's cache, whose partial
+// results are merged by the same rule in log-sum-exp form.  KV caches for incremental
+// decoding and paged KV caches are features the page "FlashAttention技术深度解析"
+// (pwwt.cn/news/595117) lists without an interface; the new tokens are read as the last
+// Nq positions of the cache (bottom-right alignment, as for causal masking).
+//
+// How it maps to B200.  Each cached key and value is read once and used for Nq·d
+// multiply-adds, so the kernel is bound by HBM bandwidth, not by the tensor cores: the
+// arithmetic runs on the CUDA cores and the design goal is to keep enough bytes in
+// flight.
+//   * grid (splits, H, B): a CTA takes one contiguous range of keys (a split, a multiple
+//     of 128 keys) of one (sequence, head), so that short batches still cover all SMs;
+//   * warp 4 streams 128-key K and V tiles by TMA (128-byte swizzle) through a ring of
+//     STAGES stages (192 KB of shared memory in flight per SM);
+//   * warps 0..3 compute.  Scores: thread t owns key t of the tile and forms its dot
+//     product with every query row (query rows in shared memory as fp32, read as
+//     broadcasts; several independent partial sums per row so the FMAs do not wait on
+//     each other).  Online softmax: the tile maximum of each row by warp shuffles and an
+//     exchange of the four warps' maxima through shared memory; every thread then holds
+//     the same running maximum, exponentiates its own key's scores and keeps its own
+//     partial row sum (summed once at the end).  P·V: warp w takes keys 32w..32w+31 of
+//     the tile, lane l the columns d/32·l ..; the four warps' partial outputs of the same
+//     rows are added once at the end;
+//   * one split: the CTA writes O and LSE; several: each writes its normalised partial O
+//     (fp32) and log2-domain LSE to the caller's workspace and fa_decode_combine_kernel
+//     merges them, O = Σ_s 2^(LSE_s − LSE) O_s with LSE = log2 Σ_s 2^LSE_s.
+// Keys past a sequence's length are never multiplied into O (cache rows there may hold
+// anything), and a paged tile loads only the pages that hold the sequence's keys.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "fattn_internal.h"
+#include "sm100.cuh"
+
+namespace fattn {
+
+template <int D>
+struct DecCfg {
+  static constexpr int BN = 128;                   // keys per tile
+  static constexpr int STAGES = (D == 128) ? 3 : 6;
+  static constexpr int KCH = D / 64;               // 64-column (128-byte) chunks per row
+  static constexpr int CHUNK = 128 * 128;          // one chunk of a 128-row tile
+  static constexpr int TILE = 128 * D * 2;         // a K or a V tile
+  static constexpr int NQ_MAX = kDecodeMaxQueries;
+  static constexpr int CPL = D / 32;               // output columns per lane in P·V
+  static constexpr int OFF_Q = 2 * STAGES * TILE;  // stage s: K at 2s·TILE, V at (2s+1)·TILE
+  static constexpr int OFF_S = OFF_Q + NQ_MAX * D * 4;        // fp32 [2][NQ_MAX][BN]: P
+  static constexpr int OFF_WM = OFF_S + 2 * NQ_MAX * BN * 4;  // fp32 [2][4][NQ_MAX]: warp maxima
+  static constexpr int OFF_L = OFF_WM + 2 * 4 * NQ_MAX * 4;   // fp32 [4][NQ_MAX]: warp sums
+  static constexpr int OFF_BAR = OFF_L + 4 * NQ_MAX * 4;
+  static constexpr int NBAR = 3 * STAGES;
+  static constexpr int SMEM_BYTES = OFF_BAR + 8 * NBAR + 16 + 1024;  // + alignment slack
+  static constexpr int THREADS = 160;  // warps 0-3 compute, warp 4 loads
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(4 * NQ_MAX * D * 4 <= 2 * STAGES * TILE, "final reduction fits in the ring");
+  static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
+};
+
+template <bool BF16>
+__device__ __forceinline__ float half_to_f32(uint16_t v) {
+  if constexpr (BF16) {
+    return __uint_as_float((uint32_t)v << 16);
+  } else {
+    return __half2float(__ushort_as_half(v));
+  }
+}
+
+// NQ: compile-time bound on the query rows (p.Nq <= NQ); rows past p.Nq are skipped.
+template <int D, bool BF16, bool PAGED, int NQ>
+__global__ void __launch_bounds__(160, 1)
+    fa_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const DecParams p) {
+  using C = DecCfg<D>;
+  constexpr int BN = C::BN, ST = C::STAGES, CPL = C::CPL;
+  enum { B_KFULL = 0, B_VFULL = ST, B_EMPTY = 2 * ST };
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * (uint32_t)i; };
+  volatile uint32_t* abort_flag =
+      reinterpret_cast<volatile uint32_t*>(sgen + C::OFF_BAR + 8 * C::NBAR);
+  float* qs = reinterpret_cast<float*>(sgen + C::OFF_Q);
+  float* S = reinterpret_cast<float*>(sgen + C::OFF_S);
+  float* WM = reinterpret_cast<float*>(sgen + C::OFF_WM);
+  float* LW = reinterpret_cast<float*>(sgen + C::OFF_L);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int Nq = p.Nq;
+  int L = p.seqlens[b];
+  if (L < 0 || L > p.max_len) {  // a length the caller's bounds do not cover: report, clamp
+    if (tid == 0) atomicOr(p.status, kDevBadCache);
+    L = L < 0 ? 0 : p.max_len;
+  }
+  const int wl = p.win_left, wr = p.win_right;
+  // keys any query row may see: [lo_all, L) (the last row's upper bound is >= L - 1)
+  const int lo_all = wl >= 0 ? max(0, L - Nq - wl) : 0;
+  const int k_first = max(split * p.chunk, lo_all) / BN * BN;
+  const int k_end = min(L, (split + 1) * p.chunk);
+  const int n_tiles = k_end > k_first ? (k_end - k_first + BN - 1) / BN : 0;
+
+  if (tid == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(BAR(B_KFULL + s), 1);
+      mbar_init(BAR(B_VFULL + s), 1);
+      mbar_init(BAR(B_EMPTY + s), 4);  // one arrival per compute warp
+    }
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (tid < 128) {  // query rows as fp32
+    const uint16_t* qg = reinterpret_cast<const uint16_t*>(p.q);
+    for (int e = tid; e < Nq * D; e += 128) {
+      const int r = e / D, c = e - r * D;
+      qs[r * D + c] = half_to_f32<BF16>(qg[((size_t)(b * Nq + r) * p.H + h) * D + c]);
+    }
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    // ============================================================ TMA producer
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % ST;
+        mbar_wait(BAR(B_EMPTY + s), ((uint32_t)(t / ST) & 1u) ^ 1u, abort_flag, p.status);
+        const int k0 = k_first + t * BN;
+        const uint32_t dK = sbase + (uint32_t)(2 * s) * C::TILE, dV = dK + C::TILE;
+        if constexpr (!PAGED) {
+          mbar_arrive_expect_tx(BAR(B_KFULL + s), C::TILE);
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_4d(&tmK, BAR(B_KFULL + s), dK + c * C::CHUNK, c * 64, h, k0, b);
+          mbar_arrive_expect_tx(BAR(B_VFULL + s), C::TILE);
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_4d(&tmV, BAR(B_VFULL + s), dV + c * C::CHUNK, c * 64, h, k0, b);
+        } else {
+          // boxes of min(page_size, 128) rows; only those holding keys below L are loaded
+          const int rows = min(p.page_size, BN);
+          const int nload = min(BN / rows, (L - k0 + rows - 1) / rows);
+          const uint32_t bytes = (uint32_t)(nload * rows * 128 * C::KCH);
+          mbar_arrive_expect_tx(BAR(B_KFULL + s), bytes);
+          mbar_arrive_expect_tx(BAR(B_VFULL + s), bytes);
+          for (int i = 0; i < nload; ++i) {
+            const int key = k0 + i * rows;
+            const int page = p.block_table[(size_t)b * p.max_blocks + key / p.page_size];
+            // an out-of-range page reads as zeros (TMA bounds) and is reported
+            if (page < 0 || page >= p.num_pages) atomicOr(p.status, kDevBadCache);
+            const int row = key % p.page_size;
+            const uint32_t off = (uint32_t)(i * rows * 128);
+            for (int c = 0; c < C::KCH; ++c) {
+              tma_load_4d(&tmK, BAR(B_KFULL + s), dK + c * C::CHUNK + off, c * 64, h, row, page);
+              tma_load_4d(&tmV, BAR(B_VFULL + s), dV + c * C::CHUNK + off, c * 64, h, row, page);
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    return;
+  }
+
+  // ============================================================== compute warps
+  // Every compute thread keeps the running maximum m of every query row (identical in all
+  // threads) and a partial row sum l over the keys it owned; O partials per warp.
+  float m_run[NQ], l_run[NQ];
+#pragma unroll
+  for (int r = 0; r < NQ; ++r) {
+    m_run[r] = -INFINITY;
+    l_run[r] = 0.f;
+  }
+  float o[NQ][CPL];
+#pragma unroll
+  for (int r = 0; r < NQ; ++r)
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) o[r][e] = 0.f;
+  const float c = p.scale_log2;
+  // independent partial dot products per row (breaks the FMA dependency chain)
+  constexpr int NACC = NQ == 1 ? 8 : (NQ <= 4 ? 4 : 2);
+  // this lane's P·V columns: chunk, 16-byte segment and byte offset inside it
+  const int col0 = lane * CPL;
+  const int vchunk = col0 >> 6, vseg = (col0 & 63) >> 3, vbyte = (col0 & 7) * 2;
+
+  for (int t = 0; t < n_tiles; ++t) {
+    const int s = t % ST;
+    const uint32_t ph = (uint32_t)(t / ST) & 1u;
+    const int buf = t & 1;
+    const int k0 = k_first + t * BN;
+    const uint8_t* Ks = sgen + (2 * s) * C::TILE;
+    const uint8_t* Vs = Ks + C::TILE;
+    float* Sb = S + buf * C::NQ_MAX * BN;
+    float* WMb = WM + buf * 4 * C::NQ_MAX;
+
+    // ---- scores x = c · q_r·k_j (thread = key j), masked keys -inf
+    mbar_wait(BAR(B_KFULL + s), ph, abort_flag, p.status);
+    const int j = k0 + tid;
+    float x[NQ];
+    {
+      float acc[NQ][NACC];
+#pragma unroll
+      for (int r = 0; r < NQ; ++r)
+#pragma unroll
+        for (int a = 0; a < NACC; ++a) acc[r][a] = 0.f;
+      if (j < L) {
+#pragma unroll
+        for (int cc = 0; cc < C::KCH; ++cc) {
+          const uint8_t* krow = Ks + cc * C::CHUNK + tid * 128;
+#pragma unroll
+          for (int seg = 0; seg < 8; ++seg) {
+            const uint4 kv = *reinterpret_cast<const uint4*>(krow + ((seg ^ (tid & 7)) << 4));
+            const float2 k01 = unpack2<BF16>(kv.x), k23 = unpack2<BF16>(kv.y);
+            const float2 k45 = unpack2<BF16>(kv.z), k67 = unpack2<BF16>(kv.w);
+            const float kf[8] = {k01.x, k01.y, k23.x, k23.y, k45.x, k45.y, k67.x, k67.y};
+#pragma unroll
+            for (int r = 0; r < NQ; ++r) {
+              if (r < Nq) {
+                const float4 qa = *reinterpret_cast<const float4*>(qs + r * D + cc * 64 + seg * 8);
+                const float4 qb =
+                    *reinterpret_cast<const float4*>(qs + r * D + cc * 64 + seg * 8 + 4);
+                const float qf[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  acc[r][e % NACC] = fmaf(qf[e], kf[e], acc[r][e % NACC]);
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < NQ; ++r) {
+        float a = 0.f;
+#pragma unroll
+        for (int u = 0; u < NACC; ++u) a += acc[r][u];
+        const int pos = L - Nq + r;  // this query row's position in the sequence
+        const bool ok =
+            r < Nq && j < L && (wr < 0 || j <= pos + wr) && (wl < 0 || j >= pos - wl);
+        x[r] = ok ? a * c : -INFINITY;
+      }
+    }
+    // ---- tile maximum per row: warp shuffles, then the four warps through shared memory
+#pragma unroll
+    for (int r = 0; r < NQ; ++r) {
+      if (r < Nq) {
+        float mx = x[r];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) WMb[warp * C::NQ_MAX + r] = mx;
+      }
+    }
+    named_barrier_sync(1, 128);
+    // ---- p = 2^(x - m_new) for this thread's key; alpha rescales l and O
+    float alpha[NQ];
+#pragma unroll
+    for (int r = 0; r < NQ; ++r) {
+      alpha[r] = 1.f;
+      if (r < Nq) {
+        const float mt = fmaxf(fmaxf(WMb[r], WMb[C::NQ_MAX + r]),
+                               fmaxf(WMb[2 * C::NQ_MAX + r], WMb[3 * C::NQ_MAX + r]));
+        const float m_new = fmaxf(m_run[r], mt);
+        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+        alpha[r] = ex2_approx(m_run[r] - mu);  // 0 while the row had no key yet
+        const float pr = ex2_approx(x[r] - mu);
+        l_run[r] = l_run[r] * alpha[r] + pr;
+        m_run[r] = m_new;
+        Sb[r * BN + tid] = pr;
+      }
+    }
+    named_barrier_sync(1, 128);
+
+    // ---- O = alpha·O + P V (warp = 32 keys, lane = CPL columns); keys past L skipped
+    mbar_wait(BAR(B_VFULL + s), ph, abort_flag, p.status);
+#pragma unroll
+    for (int r = 0; r < NQ; ++r) {
+      if (r < Nq) {
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) o[r][e] *= alpha[r];
+      }
+    }
+    const uint8_t* vcol = Vs + vchunk * C::CHUNK + vbyte;
+    const int jb = warp * 32;
+    const int je = min(jb + 32, L - k0);
+    auto pv_key = [&](int jj) {
+      const uint8_t* vp = vcol + jj * 128 + ((vseg ^ (jj & 7)) << 4);
+      float vf[CPL];
+      if constexpr (CPL == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(vp);
+        const float2 a = unpack2<BF16>(w.x), bb = unpack2<BF16>(w.y);
+        vf[0] = a.x; vf[1] = a.y; vf[2] = bb.x; vf[3] = bb.y;
+      } else {
+        const float2 a = unpack2<BF16>(*reinterpret_cast<const uint32_t*>(vp));
+        vf[0] = a.x; vf[1] = a.y;
+      }
+#pragma unroll
+      for (int r = 0; r < NQ; ++r) {
+        if (r < Nq) {
+          const float pr = Sb[r * BN + jj];
+#pragma unroll
+          for (int e = 0; e < CPL; ++e) o[r][e] = fmaf(pr, vf[e], o[r][e]);
+        }
+      }
+    };
+    if (je == jb + 32) {
+#pragma unroll 8
+      for (int jj = jb; jj < jb + 32; ++jj) pv_key(jj);
+    } else {
+      for (int jj = jb; jj < je; ++jj) pv_key(jj);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(BAR(B_EMPTY + s));
+  }
+
+  // ---- add the four warps' partial O and the 128 threads' partial l, then write
+  named_barrier_sync(1, 128);
+  float* red = reinterpret_cast<float*>(sgen);  // [4][NQ_MAX][D] over the drained K/V ring
+#pragma unroll
+  for (int r = 0; r < NQ; ++r) {
+    if (r < Nq) {
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) red[(warp * C::NQ_MAX + r) * D + col0 + e] = o[r][e];
+      float l = l_run[r];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+      if (lane == 0) LW[warp * C::NQ_MAX + r] = l;
+    }
+  }
+  named_barrier_sync(1, 128);
+  for (int e = tid; e < Nq * D; e += 128) {
+    const int r = e / D, cc = e - r * D;
+    const float sum = (red[(0 * C::NQ_MAX + r) * D + cc] + red[(1 * C::NQ_MAX + r) * D + cc]) +
+                      (red[(2 * C::NQ_MAX + r) * D + cc] + red[(3 * C::NQ_MAX + r) * D + cc]);
+    float m = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < NQ; ++u)
+      if (u == r) m = m_run[u];
+    const float l = (LW[r] + LW[C::NQ_MAX + r]) + (LW[2 * C::NQ_MAX + r] + LW[3 * C::NQ_MAX + r]);
+    const float val = l > 0.f ? sum / l : 0.f;
+    if (p.splits == 1) {
+      uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + ((size_t)(b * Nq + r) * p.H + h) * D;
+      orow[cc] = (uint16_t)(pack2<BF16>(val, 0.f) & 0xFFFFu);
+      if (cc == 0)
+        p.lse[((size_t)b * p.H + h) * Nq + r] =
+            l > 0.f ? (m + lg2_approx(l)) * 0.69314718055994530942f : INFINITY;
+    } else {
+      const size_t row = ((size_t)(b * Nq + r) * p.H + h) * p.splits + split;
+      p.o_part[row * D + cc] = val;
+      if (cc == 0) p.lse_part[row] = l > 0.f ? m + lg2_approx(l) : -INFINITY;
+    }
+  }
+}
+
+// Merge of the splits' partial results, one warp per (sequence, query row, head).
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_decode_combine_kernel(const DecParams p) {
+  constexpr int CPL = D / 32;
+  const int gw = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= p.B * p.Nq * p.H) return;
+  const int S = p.splits;
+  const float* lp = p.lse_part + (size_t)gw * S;
+  float M = -INFINITY;
+  for (int s = lane; s < S; s += 32) M = fmaxf(M, lp[s]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  const int h = gw % p.H, br = gw / p.H;
+  const int r = br % p.Nq, b = br / p.Nq;
+  uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + (size_t)gw * D + lane * CPL;
+  float* lse = p.lse + ((size_t)b * p.H + h) * p.Nq + r;
+  if (M == -INFINITY) {  // no split saw a key: O = 0, LSE = +inf
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) orow[e] = 0;
+    if (lane == 0) *lse = INFINITY;
+    return;
+  }
+  float W = 0.f;
+  for (int s = lane; s < S; s += 32) W += ex2_approx(lp[s] - M);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+  float acc[CPL];
+#pragma unroll
+  for (int e = 0; e < CPL; ++e) acc[e] = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float w = ex2_approx(lp[s] - M);
+    const float* op = p.o_part + ((size_t)gw * S + s) * D + lane * CPL;
+    if constexpr (CPL == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(op);
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+      acc[2] = fmaf(w, v.z, acc[2]);
+      acc[3] = fmaf(w, v.w, acc[3]);
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(op);
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+    }
+  }
+  const float inv = 1.f / W;
+  if constexpr (CPL == 4) {
+    *reinterpret_cast<uint2*>(orow) =
+        make_uint2(pack2<BF16>(acc[0] * inv, acc[1] * inv), pack2<BF16>(acc[2] * inv, acc[3] * inv));
+  } else {
+    *reinterpret_cast<uint32_t*>(orow) = pack2<BF16>(acc[0] * inv, acc[1] * inv);
+  }
+  if (lane == 0) *lse = (M + lg2_approx(W)) * 0.69314718055994530942f;
+}
+
+}  // namespace fattn

@@ -90,6 +90,25 @@ __host__ __device__ inline void query_tile_range(int k_first, int k_last, int Lq
   }
 }
 
+// KV-cache decode parameters (see decode_kernel.cuh).
+constexpr int kDecodeMaxQueries = 16;  // query rows per sequence in one decode call
+struct DecParams {
+  const void* q;           // [B, Nq, H, D] 16-bit
+  void* o;                 // [B, Nq, H, D] 16-bit
+  float* lse;              // [B, H, Nq] fp32, natural log
+  const int* seqlens;      // [B] cached rows per sequence (device)
+  const int* block_table;  // paged: [B, max_blocks] page ids; contiguous: nullptr
+  float* o_part;           // splits > 1: [B, Nq, H, splits, D] fp32 partial outputs
+  float* lse_part;         // splits > 1: [B, Nq, H, splits] log2-domain partial LSE
+  int B, Nq, H;
+  int max_len;             // bound on every seqlens[b] (larger values are clamped, reported)
+  int page_size, max_blocks, num_pages;  // paged only
+  int splits, chunk;       // CTAs per (sequence, head) and keys per split (multiple of 128)
+  float scale_log2;        // scale * log2(e), any sign
+  int win_left, win_right; // window as for the forward kernel (causal: -1, 0)
+  uint32_t* status;
+};
+
 enum class LaunchResult { kOk, kUnsupported, kCudaError };
 
 // Forward launch for one problem.  Tensor maps are built by the caller (api.cu).
@@ -99,6 +118,10 @@ LaunchResult launch_fwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensor
 
 // Forward grid: x = query-tile pairs, y = heads, z = batch (dense) or sequences (varlen).
 int fwd_rows_per_cta();
+
+// Decode launch: the split kernel and, when p.splits > 1, the merge kernel.
+LaunchResult launch_decode(int d, bool bf16, bool paged, const CUtensorMap& tmK,
+                           const CUtensorMap& tmV, const DecParams& p, cudaStream_t stream);
 
 // Backward launch: D preprocess, dK/dV pass, dQ pass.  q_rows = B*N (dense) or total_q
 // (varlen); batches = B (dense) or num_seqs (varlen).

@@ -15,7 +15,7 @@ namespace fattn {
 
 // ------------------------------------------------------------------ status word
 // Error codes a kernel can leave in the device status word (see fa_get_device_status).
-enum : uint32_t { kDevOk = 0u, kDevTimeout = 1u, kDevSmemAlign = 2u };
+enum : uint32_t { kDevOk = 0u, kDevTimeout = 1u, kDevSmemAlign = 2u, kDevBadCache = 4u };
 
 // Upper bound on a single mbarrier wait, in nanoseconds of %globaltimer.  A wait that
 // runs out records kDevTimeout and makes every later wait in the same CTA return at

@@ -199,6 +199,124 @@ def generate(w: Workload, with_grad_out: bool = True):
     return out
 
 
+# ------------------------------------------------------------------ KV-cache decode
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """One decode step: Nq new query tokens per sequence against its cached K/V.
+
+    Recipe: a CPU torch.Generator seeded with `seed`; randn fp32 in the order q, K cache,
+    V cache, cast to the dtype.  Contiguous caches are [B, capacity, H, d]; paged caches
+    are [num_pages, page_size, H, d] with a block table that is a seeded permutation of
+    the pages (numpy default_rng(seed + 1)), two spare pages left unused.  Cache rows past
+    a sequence's length, and unused pages, hold NaN: a correct kernel never reads them.
+    """
+    name: str
+    B: int
+    Nq: int
+    H: int
+    d: int
+    dtype: str
+    causal: bool
+    seed: int
+    cache_lens: tuple
+    capacity: int
+    page_size: int = 0               # 0: contiguous cache
+    scale: Optional[float] = None
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float16
+
+    @property
+    def max_blocks(self) -> int:
+        return -(-self.capacity // self.page_size) if self.page_size else 0
+
+    def window(self):
+        return (-1, 0) if self.causal else (-1, -1)
+
+    def flops(self) -> float:
+        """4·d FLOPs per allowed (query, key) pair, summed over sequences and heads."""
+        w = self.window()
+        return sum(4.0 * self.H * self.d * window_pairs(self.Nq, L, w) for L in self.cache_lens)
+
+    def bytes_moved(self) -> float:
+        """Algorithmic HBM bytes of one step: the cached K and V rows of every sequence
+        (read once), q read, O written, LSE written."""
+        el = 2
+        kv = 2 * sum(self.cache_lens) * self.H * self.d * el
+        qo = 2 * self.B * self.Nq * self.H * self.d * el
+        return float(kv + qo + 4 * self.B * self.H * self.Nq)
+
+    def describe(self) -> dict:
+        out = {"workload": self.name, "B": self.B, "Nq": self.Nq, "H": self.H, "d": self.d,
+               "dtype": self.dtype, "causal": self.causal, "seed": self.seed,
+               "scale": self.softmax_scale, "capacity": self.capacity,
+               "cache_tokens": int(sum(self.cache_lens)),
+               "max_cache_len": int(max(self.cache_lens))}
+        out["layout"] = f"paged (page_size {self.page_size})" if self.page_size else "contiguous"
+        return out
+
+
+def generate_decode(w: DecodeWorkload) -> dict:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    q = torch.randn((w.B, w.Nq, w.H, w.d), generator=g, dtype=torch.float32).to(w.torch_dtype)
+    lens = torch.tensor(w.cache_lens, dtype=torch.int32)
+    k = torch.randn((w.B, w.capacity, w.H, w.d), generator=g, dtype=torch.float32)
+    v = torch.randn((w.B, w.capacity, w.H, w.d), generator=g, dtype=torch.float32)
+    for b, L in enumerate(w.cache_lens):
+        k[b, L:] = float("nan")
+        v[b, L:] = float("nan")
+    k, v = k.to(w.torch_dtype), v.to(w.torch_dtype)
+    out = {"q": q, "cache_seqlens": lens}
+    if not w.page_size:
+        out["k_cache"], out["v_cache"] = k, v
+        return out
+    ps, mb = w.page_size, w.max_blocks
+    num_pages = w.B * mb + 2
+    perm = np.random.default_rng(w.seed + 1).permutation(num_pages)[:w.B * mb].reshape(w.B, mb)
+    pad = mb * ps - w.capacity
+    kp = torch.full((num_pages, ps, w.H, w.d), float("nan"), dtype=w.torch_dtype)
+    vp = torch.full((num_pages, ps, w.H, w.d), float("nan"), dtype=w.torch_dtype)
+    kk = torch.nn.functional.pad(k, (0, 0, 0, 0, 0, pad), value=float("nan")) if pad else k
+    vv = torch.nn.functional.pad(v, (0, 0, 0, 0, 0, pad), value=float("nan")) if pad else v
+    idx = torch.from_numpy(perm.reshape(-1).astype(np.int64))
+    kp[idx] = kk.reshape(w.B * mb, ps, w.H, w.d)
+    vp[idx] = vv.reshape(w.B * mb, ps, w.H, w.d)
+    out["k_pages"], out["v_pages"] = kp, vp
+    out["block_table"] = torch.from_numpy(perm.astype(np.int32))
+    return out
+
+
+def _decode_registry():
+    w = {}
+    lens16 = tuple(int(x) for x in np.random.default_rng(5).integers(1, 16385, size=16))
+    for x in (
+        # long-context single-token decode, contiguous cache (B=8, H=32, d=128, 16K cached)
+        DecodeWorkload("decode_b8_l16k", B=8, Nq=1, H=32, d=128, dtype="bf16", causal=True,
+                       seed=6, cache_lens=(16384,) * 8, capacity=16384),
+        # paged cache, ragged lengths uniform on [1, 16384], pages of 256 tokens
+        DecodeWorkload("decode_paged_ragged", B=16, Nq=1, H=32, d=128, dtype="bf16",
+                       causal=True, seed=7, cache_lens=lens16, capacity=16384, page_size=256),
+        # four new tokens per step (causal among themselves), 8K cached
+        DecodeWorkload("decode_q4_l8k", B=8, Nq=4, H=32, d=128, dtype="bf16", causal=True,
+                       seed=8, cache_lens=(8192,) * 8, capacity=8192),
+    ):
+        w[x.name] = x
+    return w
+
+
+DECODE_WORKLOADS = _decode_registry()
+
+
+def get_decode(name: str) -> DecodeWorkload:
+    return DECODE_WORKLOADS[name]
+
+
 def sample_rows(n_rows: int, k: int, seed: int) -> np.ndarray:
     """Sorted seeded subset of query/key rows, always containing the tile and causal
     boundaries 0, 1, 127, 128 and n_rows-1 (when they exist)."""

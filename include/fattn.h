@@ -56,7 +56,8 @@ extern "C" {
 
 typedef enum {
   FA_OK = 0,
-  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad cu_seqlens count */
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad cu_seqlens count,
+                             decode cache bounds exceeded on the device */
   FA_ERR_UNSUPPORTED = 2, /* head_dim other than 64/128, unknown dtype, size limits */
   FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (see fa_last_error) */
   FA_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (fa_get_device_status) */
@@ -144,6 +145,46 @@ int fa_varlen_bwd_local(const void* q, const void* k, const void* v, const void*
                         int max_seqlen_k, int H, int d, float scale, int window_left,
                         int window_right, int num_seqs, int total_q, int total_k,
                         void* workspace, size_t workspace_bytes, int dtype, void* stream);
+
+/* ---------------------------------------------------------------- KV-cache decode
+ * One incremental-decoding step: Nq new query tokens per sequence (1 <= Nq <= 16) attend
+ * to the keys and values that sequence has cached.  KV caches for incremental decoding
+ * and paged KV caches are features the page "FlashAttention技术深度解析"
+ * (pwwt.cn/news/595117) lists (CUDA backend feature table; sections on causal masking
+ * with KV-cache updates and incremental decoding, and on KV-cache management) without an
+ * interface.  Read here as: sequence b has cache_seqlens[b] cached rows (the new tokens'
+ * own keys and values already appended), and query row r sits at position
+ * cache_seqlens[b] - Nq + r, so `causal` uses the same bottom-right alignment as fa_fwd.
+ * Computes O and LSE exactly as fa_fwd would over that sequence's cached rows; rows of
+ * the cache at or past cache_seqlens[b] are never used (they may hold anything).
+ *
+ * Layouts: q, o [B, Nq, H, d]; lse [B, H, Nq] fp32; cache_seqlens device int32 [B].
+ *   fa_decode:       k_cache, v_cache [B, cache_capacity, H, d]
+ *   fa_decode_paged: k_pages, v_pages [num_pages, page_size, H, d]; block_table device
+ *                    int32 [B, max_blocks_per_seq]: logical page i of sequence b
+ *                    (rows i*page_size ..) is physical page block_table[b][i].
+ *                    page_size: a power of two >= 16.
+ * max_seqlen_k: host-side bound on every cache_seqlens[b] (<= cache_capacity, or
+ * <= max_blocks_per_seq * page_size); it sizes the split of each sequence over CTAs.
+ * A device length above its bound, or a page id outside [0, num_pages), cannot be seen
+ * on the host: the kernel clamps the length (reads nothing out of bounds, an invalid page
+ * reads as zeros) and fa_get_device_status then returns FA_ERR_INVALID_ARG.
+ * workspace: fa_decode_workspace_size(B, Nq, H, d, max_seqlen_k) bytes, 256-byte aligned
+ * (fp32 partial results of the splits); may be NULL when that size is 0.
+ * The arithmetic runs on the CUDA cores: the step is bound by reading the cache from HBM.
+ * Same dtype, alignment, stream and error conventions as fa_fwd. */
+size_t fa_decode_workspace_size(int B, int Nq, int H, int d, int max_seqlen_k);
+
+int fa_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+              const int* cache_seqlens, int B, int Nq, int H, int d, int cache_capacity,
+              int max_seqlen_k, float scale, int causal, void* workspace,
+              size_t workspace_bytes, int dtype, void* stream);
+
+int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* o,
+                    float* lse, const int* block_table, const int* cache_seqlens, int B, int Nq,
+                    int H, int d, int page_size, int num_pages, int max_blocks_per_seq,
+                    int max_seqlen_k, float scale, int causal, void* workspace,
+                    size_t workspace_bytes, int dtype, void* stream);
 
 /* Allocation-free dense backward (no counterpart on the source pages: an interface
  * addition).  Same arguments and results as fa_bwd, without the workspace: the D vector

@@ -121,3 +121,24 @@ def test_local_window_validation(lib):
                                    None) == _lib.FA_ERR_INVALID_ARG
     assert lib.fa_varlen_bwd_local(P, P, P, P, P, P, P, P, P, P, P, 10, 10, 1, 96, 0.1, 4, 4, 1,
                                    10, 10, P, 1 << 20, 0, None) == _lib.FA_ERR_UNSUPPORTED
+
+
+def test_decode_validation(lib):
+    # host-side checks of the decode calls (nothing is launched)
+    assert lib.fa_decode(P, P, P, P, P, P, 1, 17, 1, 128, 64, 64, 0.1, 1, None, 0, 0, None) == \
+        _lib.FA_ERR_UNSUPPORTED                      # Nq > 16
+    assert lib.fa_decode(P, P, P, P, P, P, 1, 1, 1, 128, 64, 65, 0.1, 1, None, 0, 0, None) == \
+        _lib.FA_ERR_INVALID_ARG                      # max_seqlen_k > capacity
+    assert lib.fa_decode(None, None, None, None, None, None, 0, 1, 1, 128, 64, 64, 0.1, 1, None,
+                         0, 0, None) == _lib.FA_OK   # B = 0
+    assert lib.fa_decode_paged(P, P, P, P, P, P, P, 1, 1, 1, 128, 24, 4, 4, 64, 0.1, 1, None, 0,
+                               0, None) == _lib.FA_ERR_UNSUPPORTED   # page size not 2^k
+    assert lib.fa_decode_paged(P, P, P, P, P, P, P, 1, 1, 1, 128, 16, 4, 2, 64, 0.1, 1, None, 0,
+                               0, None) == _lib.FA_ERR_INVALID_ARG   # 2 blocks x 16 < 64
+    # split policy: one split once B*H fills ~8 waves of CTAs, else a workspace for the
+    # fp32 partial outputs and log-sum-exps of every split
+    assert lib.fa_decode_workspace_size(40, 1, 32, 128, 16384) == 0
+    n = lib.fa_decode_workspace_size(8, 1, 32, 128, 16384)
+    splits = 5  # ceil(1184 / 256) = 5 splits of ceil(128 / 5) = 26 tiles (5 x 26 >= 128)
+    rows = 8 * 1 * 32 * splits
+    assert n == -(-rows * 128 * 4 // 256) * 256 + -(-rows * 4 // 256) * 256
