@@ -6,7 +6,7 @@ namespace fattn {
 template <int D, bool BF16, bool PAGED, int NQ>
 static LaunchResult launch_decode_t(const CUtensorMap& tmK, const CUtensorMap& tmV,
                                     const DecParams& p, cudaStream_t stream) {
-  using C = DecCfg<D>;
+  using C = DecCfg<D, NQ>;
   auto kern = fa_decode_kernel<D, BF16, PAGED, NQ>;
   static bool configured[64] = {};
   int dev = 0;

@@ -17,9 +17,12 @@
 // flight.
 //   * grid (splits, H, B): a CTA takes one contiguous range of keys (a split, a multiple
 //     of 128 keys) of one (sequence, head), so that short batches still cover all SMs;
-//   * warp 4 streams 128-key K and V tiles by TMA (128-byte swizzle) through a ring of
+//   * the last warp streams 128-key K and V tiles by TMA (128-byte swizzle) through a ring of
 //     STAGES stages (192 KB of shared memory in flight per SM);
-//   * warps 0..3 compute.  Scores: thread t owns key t of the tile and forms its dot
+//   * compute warps in groups of four (two groups when Nq <= 4, so each SM
+//     sub-partition has two compute warps to hide latency; group g takes tiles g, g + G,
+//     ... with its own softmax state, merged at the end).  Scores: thread t of a group
+//     owns key t of the tile and forms its dot
 //     product with every query row (query rows in shared memory as fp32, read as
 //     broadcasts; several independent partial sums per row so the FMAs do not wait on
 //     each other).  Online softmax: the tile maximum of each row by warp shuffles and an
@@ -43,26 +46,28 @@
 
 namespace fattn {
 
-template <int D>
+template <int D, int NQ>
 struct DecCfg {
   static constexpr int BN = 128;                   // keys per tile
   static constexpr int STAGES = (D == 128) ? 3 : 6;
   static constexpr int KCH = D / 64;               // 64-column (128-byte) chunks per row
   static constexpr int CHUNK = 128 * 128;          // one chunk of a 128-row tile
   static constexpr int TILE = 128 * D * 2;         // a K or a V tile
-  static constexpr int NQ_MAX = kDecodeMaxQueries;
   static constexpr int CPL = D / 32;               // output columns per lane in P·V
+  // consumer groups of four warps; group g takes tiles g, g + G, ...  Two groups give
+  // each SM sub-partition two compute warps; sixteen query rows need the room for one.
+  static constexpr int G = NQ <= 4 ? 2 : 1;
   static constexpr int OFF_Q = 2 * STAGES * TILE;  // stage s: K at 2s·TILE, V at (2s+1)·TILE
-  static constexpr int OFF_S = OFF_Q + NQ_MAX * D * 4;        // fp32 [2][NQ_MAX][BN]: P
-  static constexpr int OFF_WM = OFF_S + 2 * NQ_MAX * BN * 4;  // fp32 [2][4][NQ_MAX]: warp maxima
-  static constexpr int OFF_L = OFF_WM + 2 * 4 * NQ_MAX * 4;   // fp32 [4][NQ_MAX]: warp sums
-  static constexpr int OFF_BAR = OFF_L + 4 * NQ_MAX * 4;
+  static constexpr int OFF_S = OFF_Q + NQ * D * 4;          // fp32 [G][2][NQ][BN]: P
+  static constexpr int OFF_WM = OFF_S + G * 2 * NQ * BN * 4;  // fp32 [G][2][4][NQ]: warp maxima
+  static constexpr int OFF_L = OFF_WM + G * 2 * 4 * NQ * 4;   // fp32 [G][4][NQ]: warp sums
+  static constexpr int OFF_M = OFF_L + G * 4 * NQ * 4;        // fp32 [G][NQ]: group maxima
+  static constexpr int OFF_BAR = (OFF_M + G * NQ * 4 + 7) / 8 * 8;
   static constexpr int NBAR = 3 * STAGES;
   static constexpr int SMEM_BYTES = OFF_BAR + 8 * NBAR + 16 + 1024;  // + alignment slack
-  static constexpr int THREADS = 160;  // warps 0-3 compute, warp 4 loads
+  static constexpr int THREADS = 128 * G + 32;  // compute warps, then one load warp
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-  static_assert(4 * NQ_MAX * D * 4 <= 2 * STAGES * TILE, "final reduction fits in the ring");
-  static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
+  static_assert(G * 4 * NQ * D * 4 <= 2 * STAGES * TILE, "final reduction fits in the ring");
 };
 
 template <bool BF16>
@@ -76,11 +81,12 @@ __device__ __forceinline__ float half_to_f32(uint16_t v) {
 
 // NQ: compile-time bound on the query rows (p.Nq <= NQ); rows past p.Nq are skipped.
 template <int D, bool BF16, bool PAGED, int NQ>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(DecCfg<D, NQ>::THREADS, 1)
     fa_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const DecParams p) {
-  using C = DecCfg<D>;
-  constexpr int BN = C::BN, ST = C::STAGES, CPL = C::CPL;
+  using C = DecCfg<D, NQ>;
+  constexpr int BN = C::BN, ST = C::STAGES, CPL = C::CPL, G = C::G;
+  constexpr int NCOMP = 128 * G;  // compute threads
   enum { B_KFULL = 0, B_VFULL = ST, B_EMPTY = 2 * ST };
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -90,9 +96,6 @@ __global__ void __launch_bounds__(160, 1)
   volatile uint32_t* abort_flag =
       reinterpret_cast<volatile uint32_t*>(sgen + C::OFF_BAR + 8 * C::NBAR);
   float* qs = reinterpret_cast<float*>(sgen + C::OFF_Q);
-  float* S = reinterpret_cast<float*>(sgen + C::OFF_S);
-  float* WM = reinterpret_cast<float*>(sgen + C::OFF_WM);
-  float* LW = reinterpret_cast<float*>(sgen + C::OFF_L);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -114,21 +117,21 @@ __global__ void __launch_bounds__(160, 1)
     for (int s = 0; s < ST; ++s) {
       mbar_init(BAR(B_KFULL + s), 1);
       mbar_init(BAR(B_VFULL + s), 1);
-      mbar_init(BAR(B_EMPTY + s), 4);  // one arrival per compute warp
+      mbar_init(BAR(B_EMPTY + s), 4);  // one arrival per warp of the consuming group
     }
     *abort_flag = 0u;
     fence_barrier_init();
   }
-  if (tid < 128) {  // query rows as fp32
+  if (tid < NCOMP) {  // query rows as fp32
     const uint16_t* qg = reinterpret_cast<const uint16_t*>(p.q);
-    for (int e = tid; e < Nq * D; e += 128) {
+    for (int e = tid; e < Nq * D; e += NCOMP) {
       const int r = e / D, c = e - r * D;
       qs[r * D + c] = half_to_f32<BF16>(qg[((size_t)(b * Nq + r) * p.H + h) * D + c]);
     }
   }
   __syncthreads();
 
-  if (warp == 4) {
+  if (warp == 4 * G) {
     // ============================================================ TMA producer
     if (lane == 0 && n_tiles > 0) {
       tma_prefetch_desc(&tmK);
@@ -171,9 +174,17 @@ __global__ void __launch_bounds__(160, 1)
     return;
   }
 
-  // ============================================================== compute warps
-  // Every compute thread keeps the running maximum m of every query row (identical in all
-  // threads) and a partial row sum l over the keys it owned; O partials per warp.
+  // ============================================================== compute groups
+  // Group g (warps 4g..4g+3) takes tiles g, g + G, ...  Within a group every thread keeps
+  // the running maximum m of every query row (identical in all its threads) and a partial
+  // row sum l over the keys it owned; O partials per warp.  Groups merge at the end.
+  const int g = warp >> 2, gw = warp & 3;  // group, warp within the group
+  const int gt = tid & 127;                // thread within the group = key of the tile
+  float* S = reinterpret_cast<float*>(sgen + C::OFF_S) + g * 2 * NQ * BN;
+  float* WM = reinterpret_cast<float*>(sgen + C::OFF_WM) + g * 2 * 4 * NQ;
+  float* LW = reinterpret_cast<float*>(sgen + C::OFF_L) + g * 4 * NQ;
+  float* MG = reinterpret_cast<float*>(sgen + C::OFF_M);
+  const uint32_t gbar = 1u + (uint32_t)g;  // named barrier of this group
   float m_run[NQ], l_run[NQ];
 #pragma unroll
   for (int r = 0; r < NQ; ++r) {
@@ -192,19 +203,19 @@ __global__ void __launch_bounds__(160, 1)
   const int col0 = lane * CPL;
   const int vchunk = col0 >> 6, vseg = (col0 & 63) >> 3, vbyte = (col0 & 7) * 2;
 
-  for (int t = 0; t < n_tiles; ++t) {
+  for (int t = g, u = 0; t < n_tiles; t += G, ++u) {
     const int s = t % ST;
     const uint32_t ph = (uint32_t)(t / ST) & 1u;
-    const int buf = t & 1;
+    const int buf = u & 1;
     const int k0 = k_first + t * BN;
     const uint8_t* Ks = sgen + (2 * s) * C::TILE;
     const uint8_t* Vs = Ks + C::TILE;
-    float* Sb = S + buf * C::NQ_MAX * BN;
-    float* WMb = WM + buf * 4 * C::NQ_MAX;
+    float* Sb = S + buf * NQ * BN;
+    float* WMb = WM + buf * 4 * NQ;
 
     // ---- scores x = c · q_r·k_j (thread = key j), masked keys -inf
     mbar_wait(BAR(B_KFULL + s), ph, abort_flag, p.status);
-    const int j = k0 + tid;
+    const int j = k0 + gt;
     float x[NQ];
     {
       float acc[NQ][NACC];
@@ -215,10 +226,10 @@ __global__ void __launch_bounds__(160, 1)
       if (j < L) {
 #pragma unroll
         for (int cc = 0; cc < C::KCH; ++cc) {
-          const uint8_t* krow = Ks + cc * C::CHUNK + tid * 128;
+          const uint8_t* krow = Ks + cc * C::CHUNK + gt * 128;
 #pragma unroll
           for (int seg = 0; seg < 8; ++seg) {
-            const uint4 kv = *reinterpret_cast<const uint4*>(krow + ((seg ^ (tid & 7)) << 4));
+            const uint4 kv = *reinterpret_cast<const uint4*>(krow + ((seg ^ (gt & 7)) << 4));
             const float2 k01 = unpack2<BF16>(kv.x), k23 = unpack2<BF16>(kv.y);
             const float2 k45 = unpack2<BF16>(kv.z), k67 = unpack2<BF16>(kv.w);
             const float kf[8] = {k01.x, k01.y, k23.x, k23.y, k45.x, k45.y, k67.x, k67.y};
@@ -241,42 +252,41 @@ __global__ void __launch_bounds__(160, 1)
       for (int r = 0; r < NQ; ++r) {
         float a = 0.f;
 #pragma unroll
-        for (int u = 0; u < NACC; ++u) a += acc[r][u];
+        for (int v = 0; v < NACC; ++v) a += acc[r][v];
         const int pos = L - Nq + r;  // this query row's position in the sequence
         const bool ok =
             r < Nq && j < L && (wr < 0 || j <= pos + wr) && (wl < 0 || j >= pos - wl);
         x[r] = ok ? a * c : -INFINITY;
       }
     }
-    // ---- tile maximum per row: warp shuffles, then the four warps through shared memory
+    // ---- tile maximum per row: warp shuffles, then the group's four warps in shared memory
 #pragma unroll
     for (int r = 0; r < NQ; ++r) {
       if (r < Nq) {
         float mx = x[r];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        if (lane == 0) WMb[warp * C::NQ_MAX + r] = mx;
+        if (lane == 0) WMb[gw * NQ + r] = mx;
       }
     }
-    named_barrier_sync(1, 128);
+    named_barrier_sync(gbar, 128);
     // ---- p = 2^(x - m_new) for this thread's key; alpha rescales l and O
     float alpha[NQ];
 #pragma unroll
     for (int r = 0; r < NQ; ++r) {
       alpha[r] = 1.f;
       if (r < Nq) {
-        const float mt = fmaxf(fmaxf(WMb[r], WMb[C::NQ_MAX + r]),
-                               fmaxf(WMb[2 * C::NQ_MAX + r], WMb[3 * C::NQ_MAX + r]));
+        const float mt = fmaxf(fmaxf(WMb[r], WMb[NQ + r]), fmaxf(WMb[2 * NQ + r], WMb[3 * NQ + r]));
         const float m_new = fmaxf(m_run[r], mt);
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
         alpha[r] = ex2_approx(m_run[r] - mu);  // 0 while the row had no key yet
         const float pr = ex2_approx(x[r] - mu);
         l_run[r] = l_run[r] * alpha[r] + pr;
         m_run[r] = m_new;
-        Sb[r * BN + tid] = pr;
+        Sb[r * BN + gt] = pr;
       }
     }
-    named_barrier_sync(1, 128);
+    named_barrier_sync(gbar, 128);
 
     // ---- O = alpha·O + P V (warp = 32 keys, lane = CPL columns); keys past L skipped
     mbar_wait(BAR(B_VFULL + s), ph, abort_flag, p.status);
@@ -288,7 +298,7 @@ __global__ void __launch_bounds__(160, 1)
       }
     }
     const uint8_t* vcol = Vs + vchunk * C::CHUNK + vbyte;
-    const int jb = warp * 32;
+    const int jb = gw * 32;
     const int je = min(jb + 32, L - k0);
     auto pv_key = [&](int jj) {
       const uint8_t* vp = vcol + jj * 128 + ((vseg ^ (jj & 7)) << 4);
@@ -320,41 +330,50 @@ __global__ void __launch_bounds__(160, 1)
     if (lane == 0) mbar_arrive(BAR(B_EMPTY + s));
   }
 
-  // ---- add the four warps' partial O and the 128 threads' partial l, then write
-  named_barrier_sync(1, 128);
-  float* red = reinterpret_cast<float*>(sgen);  // [4][NQ_MAX][D] over the drained K/V ring
+  // ---- merge: groups' maxima, then the warps' partial O and the threads' partial l, each
+  // weighted by 2^(m_group - M) (exactly 1 for a single group)
+  named_barrier_sync(3, NCOMP);  // every tile consumed: the ring may be reused
+  float* red = reinterpret_cast<float*>(sgen);  // [G][4][NQ][D] over the drained K/V ring
 #pragma unroll
   for (int r = 0; r < NQ; ++r) {
     if (r < Nq) {
 #pragma unroll
-      for (int e = 0; e < CPL; ++e) red[(warp * C::NQ_MAX + r) * D + col0 + e] = o[r][e];
+      for (int e = 0; e < CPL; ++e) red[((g * 4 + gw) * NQ + r) * D + col0 + e] = o[r][e];
       float l = l_run[r];
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-      if (lane == 0) LW[warp * C::NQ_MAX + r] = l;
+      if (lane == 0) LW[gw * NQ + r] = l;
+      if (gt == 0) MG[g * NQ + r] = m_run[r];
     }
   }
-  named_barrier_sync(1, 128);
-  for (int e = tid; e < Nq * D; e += 128) {
+  named_barrier_sync(3, NCOMP);
+  float* LWall = reinterpret_cast<float*>(sgen + C::OFF_L);
+  for (int e = tid; e < Nq * D; e += NCOMP) {
     const int r = e / D, cc = e - r * D;
-    const float sum = (red[(0 * C::NQ_MAX + r) * D + cc] + red[(1 * C::NQ_MAX + r) * D + cc]) +
-                      (red[(2 * C::NQ_MAX + r) * D + cc] + red[(3 * C::NQ_MAX + r) * D + cc]);
-    float m = -INFINITY;
+    float M = -INFINITY;
 #pragma unroll
-    for (int u = 0; u < NQ; ++u)
-      if (u == r) m = m_run[u];
-    const float l = (LW[r] + LW[C::NQ_MAX + r]) + (LW[2 * C::NQ_MAX + r] + LW[3 * C::NQ_MAX + r]);
+    for (int q = 0; q < G; ++q) M = fmaxf(M, MG[q * NQ + r]);
+    const float Mu = (M == -INFINITY) ? 0.f : M;
+    float sum = 0.f, l = 0.f;
+#pragma unroll
+    for (int q = 0; q < G; ++q) {
+      const float wq = ex2_approx(MG[q * NQ + r] - Mu);  // 0 for a group that saw no key
+      const float* rq = red + (q * 4 * NQ + r) * D + cc;
+      sum += wq * ((rq[0] + rq[NQ * D]) + (rq[2 * NQ * D] + rq[3 * NQ * D]));
+      const float* lq = LWall + q * 4 * NQ + r;
+      l += wq * ((lq[0] + lq[NQ]) + (lq[2 * NQ] + lq[3 * NQ]));
+    }
     const float val = l > 0.f ? sum / l : 0.f;
     if (p.splits == 1) {
       uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + ((size_t)(b * Nq + r) * p.H + h) * D;
       orow[cc] = (uint16_t)(pack2<BF16>(val, 0.f) & 0xFFFFu);
       if (cc == 0)
         p.lse[((size_t)b * p.H + h) * Nq + r] =
-            l > 0.f ? (m + lg2_approx(l)) * 0.69314718055994530942f : INFINITY;
+            l > 0.f ? (M + lg2_approx(l)) * 0.69314718055994530942f : INFINITY;
     } else {
       const size_t row = ((size_t)(b * Nq + r) * p.H + h) * p.splits + split;
       p.o_part[row * D + cc] = val;
-      if (cc == 0) p.lse_part[row] = l > 0.f ? m + lg2_approx(l) : -INFINITY;
+      if (cc == 0) p.lse_part[row] = l > 0.f ? M + lg2_approx(l) : -INFINITY;
     }
   }
 }
