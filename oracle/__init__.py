@@ -7,7 +7,9 @@ from .attn_ref import (  # noqa: F401
     attention_backward_bhsd,
     attention_forward,
     attention_forward_bhsd,
+    attention_forward_fp8,
     decode_attention,
+    e4m3_to_float,
     kv_cache_gather,
     softmax_probs,
     varlen_attention_backward,

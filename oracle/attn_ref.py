@@ -310,3 +310,33 @@ def decode_attention(q, k_cache, v_cache, cache_seqlens, scale, causal, block_ta
             out[b, :, h] = o
             lse[b, h] = l
     return out, lse
+
+
+# ------------------------------------------------------------------ FP8 (e4m3) inputs
+# The pages credit FP8 tensor-core support to Hopper and quote FP8 attention at over 1.2
+# PFLOPS with an 8-bit quantization strategy (page "FlashAttention实战：如何在A100上实现3倍
+# 加速的Transformer训练" §7; page "Flash Attention V3：大模型训练加速与显存优化技术解析"
+# §2.1; page "FlashAttention技术深度解析", CUDA backend feature table) without fixing a
+# format or scaling.  Read here as the OCP FP8 E4M3 format the tensor cores take, one
+# dequantisation factor per tensor: the attention inputs are q = sq·Q8, k = sk·K8, v = sv·V8.
+
+def e4m3_to_float(codes):
+    """Decode FP8 E4M3 bytes to float64: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa
+    bits; exponent 0 is subnormal (m · 2^-9); no infinities; S.1111.111 is NaN.
+    Largest finite magnitude 448."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def attention_forward_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale, causal,
+                          rows=None, window=None):
+    """Attention of dequantised FP8 inputs: attention_forward(sq·Q8, sk·K8, sv·V8)."""
+    q = e4m3_to_float(q8) * float(q_descale)
+    k = e4m3_to_float(k8) * float(k_descale)
+    v = e4m3_to_float(v8) * float(v_descale)
+    return attention_forward(q, k, v, scale, causal, rows=rows, window=window)
