@@ -429,6 +429,191 @@ def run_decode_reference(args, w):
     return 0
 
 
+# ------------------------------------------------------------------ FP8 forward arm
+FP8_METRIC = "FP8 (E4M3) attention forward TFLOPS and % of B200 FP8 tensor peak"
+
+
+def oracle_fp8_seconds(w, host, rows: int, reps: int = 1):
+    """fp64 oracle forward of the last `rows` query rows of head (0, 0), FP8 inputs."""
+    import numpy as np
+    import oracle
+    from exact_tiled_attention_33_b200 import workloads as wl
+    q8, k8, v8 = (host[x][0, :, 0].view(torch_uint8()).numpy() for x in ("q8", "k8", "v8"))
+    N = q8.shape[0]
+    r = np.arange(N - rows, N)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.attention_forward_fp8(q8, k8, v8, host["q_descale"], host["k_descale"],
+                                     host["v_descale"], w.softmax_scale, w.causal, rows=r)
+    dt = time.perf_counter() - t0
+    win = (-1, 0) if w.causal else (-1, -1)
+    return dt, 4.0 * w.d * wl.window_pairs(rows, N, win) * reps, os.cpu_count()
+
+
+def run_fp8_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from exact_tiled_attention_33_b200 import workloads as wl
+    host = wl.generate(w, with_grad_out=False)
+    rows = 64
+    dt, _, _ = oracle_fp8_seconds(w, host, rows)
+    while dt < 0.5 and rows < w.N:
+        rows = min(w.N, rows * 2)
+        dt, _, _ = oracle_fp8_seconds(w, host, rows)
+    for _ in range(args.warmup):
+        oracle_fp8_seconds(w, host, rows)
+    tot_t = tot_f = 0.0
+    threads = os.cpu_count()
+    for _ in range(args.steps):
+        dt, fl, threads = oracle_fp8_seconds(w, host, rows)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = (f"last {rows} query rows of head (b=0,h=0) of {w.name} against all {w.N} keys, "
+              f"fp64 oracle forward of the dequantised FP8 inputs, per step")
+    print(json.dumps({"impl": "reference", "metric": FP8_METRIC, "value": value, "unit": UNIT,
+                      "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                      "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
+                      "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                      "data": "synthetic", "config": dict(w.describe(), parallelism=f"dp{world}"),
+                      "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads,
+                                       "kind": "oracle", "sample": sample},
+                      "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                              "d2h_bytes_per_step": 0}}), flush=True)
+    return 0
+
+
+def torch_uint8():
+    import torch
+    return torch.uint8
+
+
+def run_fp8(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from exact_tiled_attention_33_b200 import _lib
+    from exact_tiled_attention_33_b200 import workloads as wl
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    lib = _lib.load()
+    wr = wl.Workload(**{**w.__dict__, "seed": w.seed + rank})
+    host = wl.generate(wr, with_grad_out=False)
+    B, N, H, d = wr.B, wr.N, wr.H, wr.d
+    q8, k8, v8 = (host[x].to(dev) for x in ("q8", "k8", "v8"))
+    sq, sk, sv = host["q_descale"], host["k_descale"], host["v_descale"]
+    odt = _lib.FA_BF16 if wr.dtype == "bf16" else _lib.FA_FP16
+    o = torch.empty(q8.shape, dtype=torch.bfloat16 if wr.dtype == "bf16" else torch.float16,
+                    device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+
+    def step():
+        _lib.check(lib.fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), o.data_ptr(),
+                                  lse.data_ptr(), B, N, H, d, wr.softmax_scale, sq, sk, sv,
+                                  int(wr.causal), odt, sh), "fa_fwd_fp8")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert lib.fa_get_device_status(sh) == 0, "device status after warm-up"
+    # timed region: the inputs (134 MB per tensor) are larger than the 126 MB L2
+    sampler = ClockSampler(local) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler is not None else None
+    assert lib.fa_get_device_status(sh) == 0, "device status in timed region"
+    max_s = max_over_ranks(t0.elapsed_time(t1) / 1e3, world)
+    f = wr.fwd_flops()
+    value = throughput_tflops(f, args.steps, world, max_s)
+    per = statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3
+
+    e2e = None
+    if not args.no_e2e:
+        hin = [host[x].view(torch.uint8).pin_memory() for x in ("q8", "k8", "v8")]
+        dins = [x.view(torch.uint8) for x in (q8, k8, v8)]
+        hout = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (o, lse)]
+        n_e2e = max(2, min(args.steps, 5))
+
+        def e2e_step():
+            for hs, dd in zip(hin, dins):
+                dd.copy_(hs, non_blocking=True)
+            step()
+            for ds, hd in zip((o, lse), hout):
+                hd.copy_(ds, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_s = max_over_ranks(a.elapsed_time(b_) / 1e3, world)
+        e2e = {"value": throughput_tflops(f, n_e2e, world, e2e_s), "unit": UNIT,
+               "h2d_bytes_per_step": sum(x.numel() for x in hin),
+               "d2h_bytes_per_step": sum(x.numel() * x.element_size() for x in hout),
+               "steps": n_e2e}
+
+    burst, sust, _, src = load_peaks()
+    # no measured FP8 peak: the measured bf16 figure times the nominal FP8/BF16 ratio (2)
+    peak_b, peak_s = 2 * burst, 2 * sust
+    ach = f / per / 1e12
+    sha = sources_sha(FWD_SOURCES)
+    roofline = {"kernel": "fa_fwd_kernel<128, bf16 out, fp8>", "bound": "tensor",
+                "achieved": ach, "peak": peak_s, "unit": "TFLOP/s", "frac": ach / peak_s,
+                "frac_of_burst_peak": ach / peak_b,
+                "peak_source": f"2 x bf16_tflops_sustained ({src}; nominal fp8/bf16 ratio)",
+                "traffic": read_traffic("fa_fwd_kernel_fp8", wr.name, sha),
+                "flops_per_launch": f}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = 256
+        dt, fl, threads = oracle_fp8_seconds(wr, host, rows)
+        while dt < 5.0 and rows < N:
+            rows = min(N, rows * 2)
+            dt, fl, threads = oracle_fp8_seconds(wr, host, rows)
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"last {rows} query rows of head (b=0,h=0) against all {N} keys, "
+                         f"fp64 oracle forward of the dequantised FP8 inputs ({dt:.1f} s)"}
+    if rank == 0:
+        line = {"metric": FP8_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * max_s / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (bf16 out)",
+                "data": "synthetic",
+                "config": dict(wr.describe(), seed=w.seed, parallelism=f"dp{world}",
+                               l2="inputs larger than L2 (134 MB per tensor), no flush"),
+                "gpu_launches": args.steps, "roofline": roofline, "clocks": clocks,
+                "e2e": e2e, "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 # ------------------------------------------------------------------ KV-cache decode arm
 DECODE_METRIC = "KV-cache decode: HBM GB/s of the cached K/V read (and attention TFLOPS)"
 DECODE_SOURCES = ["exact_tiled_attention_33_b200/csrc/decode_kernel.cuh",
@@ -616,6 +801,10 @@ def main(argv=None):
             return run_decode_reference(args, wl.get_decode(args.workload))
         return run_decode(args, wl.get_decode(args.workload))
     w = wl.get(args.workload)
+    if w.fp8:
+        if args.impl == "reference":
+            return run_fp8_reference(args, w)
+        return run_fp8(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_fattn(args, w)

@@ -40,6 +40,9 @@ SIGNATURES = {
                           _i, _vp, _sz, _i, _vp]),
     "fa_varlen_bwd_local": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
                                  _i, _i, _f, _i, _i, _i, _i, _i, _vp, _sz, _i, _vp]),
+    "fa_fwd_fp8": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _f, _f, _f, _i, _i, _vp]),
+    "fa_varlen_fwd_fp8": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _f, _f, _f,
+                               _i, _i, _i, _i, _i, _vp]),
     "fa_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "fa_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _sz, _i,
                        _vp]),

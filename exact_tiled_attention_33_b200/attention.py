@@ -263,6 +263,65 @@ def varlen_bwd_local(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seql
     return dq, dk, dv
 
 
+# ------------------------------------------------------------------ FP8 forward
+# 8-bit (E4M3) inputs with per-tensor dequantisation factors (pages: FP8 attention with an
+# 8-bit quantization strategy on Hopper tensor cores).
+
+def _check_fp8(*ts):
+    dev = ts[0].device
+    if dev.type != "cuda":
+        raise ValueError("attention tensors must be CUDA tensors")
+    for t in ts:
+        if t.dtype not in (torch.float8_e4m3fn, torch.uint8) or t.device != dev or \
+                not t.is_contiguous():
+            raise ValueError("FP8 inputs must be contiguous float8_e4m3fn (or uint8) tensors "
+                             "on one device")
+
+
+def fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, softmax_scale=None, causal=False,
+            out_dtype=torch.bfloat16, out=None, lse=None):
+    """Dense FP8 forward (fa_fwd_fp8): q8, k8, v8 [B, N, H, 128] E4M3.
+    Returns (o [B,N,H,128] out_dtype, lse [B,H,N] fp32)."""
+    if q8.dim() != 4 or k8.shape != q8.shape or v8.shape != q8.shape:
+        raise ValueError("q, k, v must all be [B, N, H, d] with equal shapes")
+    _check_fp8(q8, k8, v8)
+    B, N, H, d = q8.shape
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    o = torch.empty(q8.shape, dtype=out_dtype, device=q8.device) if out is None else out
+    lse_t = torch.empty((B, H, N), device=q8.device, dtype=torch.float32) if lse is None else lse
+    lib = _lib.load()
+    with torch.cuda.device(q8.device):
+        st = lib.fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(o), _ptr(lse_t), B, N, H, d, scale,
+                            float(q_descale), float(k_descale), float(v_descale),
+                            int(bool(causal)), _DTYPES[o.dtype], _stream(q8))
+    _lib.check(st, "fa_fwd_fp8")
+    return o, lse_t
+
+
+def varlen_fwd_fp8(q8, k8, v8, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                   q_descale, k_descale, v_descale, softmax_scale=None, causal=False,
+                   out_dtype=torch.bfloat16, out=None, lse=None):
+    """Packed FP8 forward (fa_varlen_fwd_fp8). Returns (o, lse) as varlen_fwd."""
+    if q8.dim() != 3 or k8.dim() != 3 or k8.shape != v8.shape or q8.shape[1:] != k8.shape[1:]:
+        raise ValueError("q must be [total_q, H, d] and k, v [total_k, H, d]")
+    _check_fp8(q8, k8, v8)
+    total_q, H, d = q8.shape
+    total_k = k8.shape[0]
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    o = torch.empty(q8.shape, dtype=out_dtype, device=q8.device) if out is None else out
+    lse_t = torch.empty((H, total_q), device=q8.device, dtype=torch.float32) if lse is None else lse
+    lib = _lib.load()
+    with torch.cuda.device(q8.device):
+        st = lib.fa_varlen_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(o), _ptr(lse_t),
+                                   _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q),
+                                   int(max_seqlen_k), H, d, scale, float(q_descale),
+                                   float(k_descale), float(v_descale), int(bool(causal)),
+                                   cu_seqlens_q.numel() - 1, total_q, total_k,
+                                   _DTYPES[o.dtype], _stream(q8))
+    _lib.check(st, "fa_varlen_fwd_fp8")
+    return o, lse_t
+
+
 # ------------------------------------------------------------------ KV-cache decode
 # One incremental-decoding step over a KV cache (page "FlashAttention技术深度解析"
 # (pwwt.cn/news/595117): KV caches for incremental decoding, paged KV caches).  The Nq

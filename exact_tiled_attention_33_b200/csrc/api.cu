@@ -70,20 +70,24 @@ int ensure_context() {
   return e == cudaSuccess ? FA_OK : cuda_fail(e, "making the device context current");
 }
 
-// Tensor map over a [batches, rows, H, d] 16-bit tensor, dims listed innermost first
-// (d, H, rows, batches); box = 64 elements of d (one 128-byte swizzle row) x 1 head x
-// box_rows rows.  Out-of-range rows read as zero.
+// Tensor map over a [batches, rows, H, d] tensor of 16-bit (elem_bytes 2) or 8-bit
+// (elem_bytes 1) elements, dims listed innermost first (d, H, rows, batches); box = one
+// 128-byte swizzle row of d (64 or 128 elements) x 1 head x box_rows rows.  Out-of-range
+// rows read as zero.
 int make_map(CUtensorMap* map, const void* base, int d, int H, long long rows, long long batches,
-             int box_rows) {
+             int box_rows, int elem_bytes = 2) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   if (int e = ensure_context()) return e;
+  const cuuint64_t eb = (cuuint64_t)elem_bytes;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)batches};
-  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2,
-                           (cuuint64_t)rows * H * d * 2};
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  cuuint64_t strides[3] = {(cuuint64_t)d * eb, (cuuint64_t)H * d * eb,
+                           (cuuint64_t)rows * H * d * eb};
+  cuuint32_t box[4] = {(cuuint32_t)(128 / elem_bytes), 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(base), dims, strides,
+  const CUtensorMapDataType dt =
+      elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+  CUresult r = enc(map, dt, 4, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
@@ -144,6 +148,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // every finite score maps to x = 0 exactly in fp32 (uniform weights) while masked
 // scores (-inf) stay -inf.
 void set_fwd_scale(FwdParams& p, float scale) {
+  p.v_descale = 1.f;
   p.negate_scores = scale < 0.f ? 1 : 0;
   const float c = std::fabs(scale) * kLog2e;
   p.scale_log2 = c > 1e-30f ? c : 1e-30f;
@@ -308,6 +313,108 @@ int fa_varlen_fwd_local(const void* q, const void* k, const void* v, void* o, fl
   return fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, H,
                     d, scale, window_left, window_right, num_seqs, total_q, total_k, dtype,
                     stream);
+}
+
+// ------------------------------------------------------------------ FP8 forward
+namespace {
+
+int fp8_check(int d, float scale, float q_descale, float k_descale, float v_descale,
+              int out_dtype) {
+  if (d != 128) return fail(FA_ERR_UNSUPPORTED, "FP8 forward takes head_dim 128");
+  if (out_dtype != FA_BF16 && out_dtype != FA_FP16) return fail(FA_ERR_UNSUPPORTED, "unknown dtype");
+  if (!std::isfinite(scale) || scale < 0.f)
+    return fail(FA_ERR_UNSUPPORTED, "FP8 forward takes a finite scale >= 0");
+  for (float s : {q_descale, k_descale, v_descale})
+    if (!std::isfinite(s) || s <= 0.f)
+      return fail(FA_ERR_INVALID_ARG, "descale factors must be finite and > 0");
+  return FA_OK;
+}
+
+void set_fp8_scale(FwdParams& p, float scale, float q_descale, float k_descale,
+                   float v_descale) {
+  set_fwd_scale(p, scale * q_descale * k_descale);
+  p.v_descale = v_descale;
+}
+
+}  // namespace
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N,
+               int H, int d, float scale, float q_descale, float k_descale, float v_descale,
+               int causal, int out_dtype, void* stream) {
+  g_last_error.clear();
+  if (int e = fp8_check(d, scale, q_descale, k_descale, v_descale, out_dtype)) return e;
+  if (H < 0 || H > 65535) return fail(FA_ERR_UNSUPPORTED, "H must be in [0, 65535]");
+  if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
+  if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
+  if (B == 0 || N == 0 || H == 0) return FA_OK;
+  if (int e = check_grid(B, H, N)) return e;
+  if (int e = check_ptrs({q, k, v, o, lse})) return e;
+  CUtensorMap mq, mk, mv;
+  if (int e = make_map(&mq, q, d, H, N, B, 128, 1)) return e;
+  if (int e = make_map(&mk, k, d, H, N, B, 128, 1)) return e;
+  if (int e = make_map(&mv, v, d, H, N, B, 128, 1)) return e;
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.N = N;
+  p.H = H;
+  p.total_q = B * N;
+  p.scale = scale;
+  set_fp8_scale(p, scale, q_descale, k_descale, v_descale);
+  p.win_left = -1;
+  p.win_right = causal ? 0 : -1;
+  p.reverse_tiles = reverse_tiles(p.win_left, p.win_right);
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  const int rows = fwd_rows_per_cta();
+  dim3 grid((N + rows - 1) / rows, H, B);
+  return launch_result(
+      launch_fwd_fp8(d, out_dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+}
+
+int fa_varlen_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                      const int* cu_seqlens_q, const int* cu_seqlens_k, int max_seqlen_q,
+                      int max_seqlen_k, int H, int d, float scale, float q_descale,
+                      float k_descale, float v_descale, int causal, int num_seqs, int total_q,
+                      int total_k, int out_dtype, void* stream) {
+  g_last_error.clear();
+  if (int e = fp8_check(d, scale, q_descale, k_descale, v_descale, out_dtype)) return e;
+  if (H < 0 || H > 65535) return fail(FA_ERR_UNSUPPORTED, "H must be in [0, 65535]");
+  if (num_seqs < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
+    return fail(FA_ERR_INVALID_ARG, "sizes must be >= 0");
+  if (num_seqs > 65535) return fail(FA_ERR_UNSUPPORTED, "num_seqs must be <= 65535");
+  if (max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return fail(FA_ERR_INVALID_ARG, "max_seqlen exceeds the total token count");
+  if (num_seqs == 0 || total_q == 0 || H == 0 || max_seqlen_q == 0) return FA_OK;
+  if (int e = check_grid(num_seqs, H, std::max(max_seqlen_q, max_seqlen_k))) return e;
+  if (int e = check_ptrs({q, o, lse, cu_seqlens_q, cu_seqlens_k})) return e;
+  if (total_k > 0)
+    if (int e = check_ptrs({k, v})) return e;
+  CUtensorMap mq, mk, mv;
+  if (int e = make_map(&mq, q, d, H, total_q, 1, 128, 1)) return e;
+  const void* kb = total_k > 0 ? k : q;
+  const void* vb = total_k > 0 ? v : q;
+  const long long kr = total_k > 0 ? total_k : total_q;
+  if (int e = make_map(&mk, kb, d, H, kr, 1, 128, 1)) return e;
+  if (int e = make_map(&mv, vb, d, H, kr, 1, 128, 1)) return e;
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.H = H;
+  p.total_q = total_q;
+  p.scale = scale;
+  set_fp8_scale(p, scale, q_descale, k_descale, v_descale);
+  p.win_left = -1;
+  p.win_right = causal ? 0 : -1;
+  p.reverse_tiles = reverse_tiles(p.win_left, p.win_right);
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  const int rows = fwd_rows_per_cta();
+  dim3 grid((max_seqlen_q + rows - 1) / rows, H, num_seqs);
+  return launch_result(
+      launch_fwd_fp8(d, out_dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int N, int H, int d) {

@@ -22,6 +22,7 @@ struct FwdParams {
   float scale;      // softmax scale
   float scale_log2; // |scale| * log2(e), > 0 (a tiny positive value when scale == 0)
   int negate_scores;// 1 when scale < 0: the S product negates Q
+  float v_descale;  // O is multiplied by it (FP8 inputs; 1 otherwise)
   int win_left;     // attention window (see key_tile_range); causal is (-1, 0)
   int win_right;
   int reverse_tiles;// launch the query tiles with the most key tiles first
@@ -115,6 +116,10 @@ enum class LaunchResult { kOk, kUnsupported, kCudaError };
 LaunchResult launch_fwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                         const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
                         cudaStream_t stream);
+// FP8 (E4M3) operands, d = 128; bf16 selects the output format.
+LaunchResult launch_fwd_fp8(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                            const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
+                            cudaStream_t stream);
 
 // Forward grid: x = query-tile pairs, y = heads, z = batch (dense) or sequences (varlen).
 int fwd_rows_per_cta();

@@ -5,12 +5,12 @@ namespace fattn {
 
 int fwd_rows_per_cta() { return FwdCfg<128>::BM; }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool FP8 = false>
 static LaunchResult launch_fwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                  const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
                                  cudaStream_t stream) {
-  using C = FwdCfg<D>;
-  auto kern = fa_fwd_kernel<D, BF16>;
+  using C = FwdCfg<D, FP8>;
+  auto kern = fa_fwd_kernel<D, BF16, FP8>;
   static bool configured[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LaunchResult::kCudaError;
@@ -36,6 +36,14 @@ LaunchResult launch_fwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensor
                 : launch_fwd_t<64, false>(tmQ, tmK, tmV, p, grid, stream);
   }
   return LaunchResult::kUnsupported;
+}
+
+LaunchResult launch_fwd_fp8(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                            const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
+                            cudaStream_t stream) {
+  if (d != 128) return LaunchResult::kUnsupported;
+  return bf16 ? launch_fwd_t<128, true, true>(tmQ, tmK, tmV, p, grid, stream)
+              : launch_fwd_t<128, false, true>(tmQ, tmK, tmV, p, grid, stream);
 }
 
 }  // namespace fattn

@@ -32,14 +32,17 @@
 
 namespace fattn {
 
-template <int D>
+// FP8: E4M3 operands (1 byte) and 8-bit MMAs (32 elements of K per instruction).
+template <int D, bool FP8 = false>
 struct FwdCfg {
   static constexpr int BM = 128;  // query rows per tile = tensor-memory lanes
   static constexpr int BN = 128;  // keys per K/V tile
-  static constexpr int STAGES = (D == 128) ? 2 : 4;
-  static constexpr int KCH = D / 64;   // 128-byte (64-element) column chunks per row
+  static constexpr int EB = FP8 ? 1 : 2;        // operand bytes
+  static constexpr int KSTEP = FP8 ? 32 : 16;   // K elements per MMA instruction
+  static constexpr int STAGES = FP8 ? 4 : ((D == 128) ? 2 : 4);
+  static constexpr int KCH = D * EB / 128;      // 128-byte column chunks per row
   static constexpr int CHUNK = 128 * 128;
-  static constexpr int TILE = 128 * D * 2;
+  static constexpr int TILE = 128 * D * EB;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + TILE;
   static constexpr int OFF_V = OFF_K + STAGES * TILE;
@@ -61,18 +64,27 @@ struct FwdCfg {
   static constexpr uint32_t TM_O = 256;
   // pairs of every 16 (per 32-column chunk) whose exponentials use exp2_poly2
   static constexpr int kPolyPairs = 4;
-  // packed 16-bit P column for keys 16*kk .. 16*kk+15 of a 128-key tile: half 0 packs into
-  // columns 0..31 of its S buffer, half 1 into 64..95
+  // packed P column for the kk-th K step of a 128-key tile.  16-bit P (16 keys per step,
+  // 2 per column): half 0 packs into columns 0..31 of its S buffer, half 1 into 64..95.
+  // 8-bit P (32 keys per step, 4 per column): half 0 into 0..15, half 1 into 64..79.
   __device__ static constexpr uint32_t packed_col(int kk) {
-    return (uint32_t)(kk * 8 + (kk >= 4 ? 32 : 0));
+    return FP8 ? (uint32_t)((kk >> 1) * 64 + (kk & 1) * 8)
+               : (uint32_t)(kk * 8 + (kk >= 4 ? 32 : 0));
   }
 };
 
-template <int D, bool BF16>
+// BF16: 16-bit format of the output (and of the operands unless FP8).
+template <int D, bool BF16, bool FP8 = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, FP8>;
+  constexpr int EL = 128 / C::EB;  // elements per 128-byte chunk (TMA x step)
+  // 8-bit P is scaled by 2^8 (p = 2^(x - m + 8)) so that it spans the normal E4M3 range,
+  // and the reference maximum is refreshed as soon as the row maximum grows by 0.5 so that
+  // p stays below 2^8.5 < 448; 16-bit P keeps p = 2^(x - m) with the lazy threshold 8.
+  constexpr float POFF = FP8 ? 8.f : 0.f;
+  constexpr float LAZY = FP8 ? 0.5f : 8.f;
   constexpr int BM = C::BM, BN = C::BN, ST = C::STAGES;
 
   extern __shared__ uint8_t smem_raw[];
@@ -147,7 +159,7 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(BAR(C::B_QFULL), C::TILE);
       for (int c = 0; c < C::KCH; ++c)
-        tma_load_4d(&tmQ, BAR(C::B_QFULL), sbase + C::OFF_Q + c * C::CHUNK, c * 64, h, q_row0 + q0,
+        tma_load_4d(&tmQ, BAR(C::B_QFULL), sbase + C::OFF_Q + c * C::CHUNK, c * EL, h, q_row0 + q0,
                     bcoord);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % ST;
@@ -156,12 +168,12 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(BAR(C::B_KFULL + s), C::TILE);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(&tmK, BAR(C::B_KFULL + s), sbase + C::OFF_K + s * C::TILE + c * C::CHUNK,
-                      c * 64, h, k_row0 + (j0 + j) * BN, bcoord);
+                      c * EL, h, k_row0 + (j0 + j) * BN, bcoord);
         mbar_wait(BAR(C::B_VEMPTY + s), ph ^ 1u, abort_flag, p.status);
         mbar_arrive_expect_tx(BAR(C::B_VFULL + s), C::TILE);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(&tmV, BAR(C::B_VFULL + s), sbase + C::OFF_V + s * C::TILE + c * C::CHUNK,
-                      c * 64, h, k_row0 + (j0 + j) * BN, bcoord);
+                      c * EL, h, k_row0 + (j0 + j) * BN, bcoord);
       }
     }
     __syncwarp();
@@ -170,9 +182,10 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0 && n_kv > 0) {
       // S = Q Kᵀ: A = Q (K-major), B = K (K-major).  O += P V: A = P (tensor memory),
       // B = V stored [key][d], i.e. N-contiguous (MN-major).
-      constexpr uint32_t ID_S0 = idesc_f16_f32acc(BF16, BM, BN, false, false);
+      // (format code 0 is f16 for .kind::f16 and E4M3 for .kind::f8f6f4)
+      constexpr uint32_t ID_S0 = idesc_f16_f32acc(BF16 && !FP8, BM, BN, false, false);
       const uint32_t ID_S = ID_S0 | (p.negate_scores ? (1u << 13) : 0u);  // bit 13: negate A
-      constexpr uint32_t ID_O = idesc_f16_f32acc(BF16, BM, D, false, true);
+      constexpr uint32_t ID_O = idesc_f16_f32acc(BF16 && !FP8, BM, D, false, true);
       // Descriptors built once; each MMA only adds a compile-time offset.
       const uint64_t dQ = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
       const uint64_t dK0 = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
@@ -184,9 +197,14 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t db = sdesc_adv(dK0, (uint32_t)(s * C::TILE));
         const uint32_t dst = tmem + 128u * (uint32_t)(j & 1);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(dst, sdesc_adv(dQ, (kk >> 2) * C::CHUNK + (kk & 3) * 32),
-                 sdesc_adv(db, (kk >> 2) * C::CHUNK + (kk & 3) * 32), ID_S, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < D / C::KSTEP; ++kk) {
+          // K step kk starts kk * 32 bytes into the rows: chunk kk / 4, byte (kk % 4) * 32
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          if constexpr (FP8)
+            mma_ss_f8(dst, sdesc_adv(dQ, off), sdesc_adv(db, off), ID_S, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(dst, sdesc_adv(dQ, off), sdesc_adv(db, off), ID_S, kk > 0 ? 1u : 0u);
+        }
         mma_commit(BAR(C::B_SFULL + (j & 1)));
         mma_commit(BAR(C::B_KEMPTY + s));
       };
@@ -201,9 +219,15 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t db = sdesc_adv(dV0, (uint32_t)(s * C::TILE));
         const uint32_t src = tmem + 128u * (uint32_t)(j & 1);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + C::TM_O, src + C::packed_col(kk), sdesc_adv(db, kk * 16 * 128), ID_O,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BN / C::KSTEP; ++kk) {
+          // V rows kk * KSTEP .. of the tile: 128-byte rows, so KSTEP * 128 bytes per step
+          if constexpr (FP8)
+            mma_ts_f8(tmem + C::TM_O, src + C::packed_col(kk),
+                      sdesc_adv(db, kk * C::KSTEP * 128), ID_O, (j > 0 || kk > 0) ? 1u : 0u);
+          else
+            mma_ts(tmem + C::TM_O, src + C::packed_col(kk), sdesc_adv(db, kk * C::KSTEP * 128),
+                   ID_O, (j > 0 || kk > 0) ? 1u : 0u);
+        }
         mma_commit(BAR(C::B_ODONE));
         mma_commit(BAR(C::B_VEMPTY + s));
         // S_{j+2} reuses the buffer of S_j, whose P the product above has just consumed
@@ -272,7 +296,7 @@ __global__ void __launch_bounds__(384, 1)
       float alpha = 1.f;
       if (m == -INFINITY) {
         m = mx;  // first allowed keys for this row: O and l are still exactly 0
-      } else if (mx - m > 8.f) {
+      } else if (mx - m > LAZY) {
         alpha = ex2_approx(m - mx);
         m = mx;
         rescale = true;
@@ -282,15 +306,16 @@ __global__ void __launch_bounds__(384, 1)
       // P·V product uses and normalises O, so numerator and denominator share the
       // rounding of P (under the lazy maximum the largest P of a row is 2^δ, not 1).
       const uint64_t c2 = f2_pack(c, c);
-      const uint64_t nm2 = f2_pack(-m_use, -m_use);
+      const uint64_t nm2 = f2_pack(POFF - m_use, POFF - m_use);
       uint64_t ls2 = 0ull, lr2 = 0ull;
       // A quarter of the exponentials run on the FMA pipe (tiles without masked keys), the
       // rest on the special-function unit; the choice is made once per tile so the loop
       // bodies stay branch-free.
       auto exp_pass = [&](auto use_poly) {
+        [[maybe_unused]] uint32_t pk8[16];  // 8-bit P: four keys per 32-bit column
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          uint32_t pk[16];
+          [[maybe_unused]] uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[q * 32 + 2 * e]),
@@ -306,13 +331,24 @@ __global__ void __launch_bounds__(384, 1)
               p0 = ex2_approx(xx.x);
               p1 = ex2_approx(xx.y);
             }
-            pk[e] = pack2<BF16>(p0, p1);
-            const float2 pr = unpack2<BF16>(pk[e]);
+            float2 pr;
+            if constexpr (FP8) {
+              const uint32_t h8 = pack2_e4m3(p0, p1);
+              pr = unpack2_e4m3(h8);
+              if (e & 1)
+                pk8[q * 8 + (e >> 1)] |= h8 << 16;
+              else
+                pk8[q * 8 + (e >> 1)] = h8;
+            } else {
+              pk[e] = pack2<BF16>(p0, p1);
+              pr = unpack2<BF16>(pk[e]);
+            }
             ls2 = f2_add(ls2, f2_pack(p0, p1));
             lr2 = f2_add(lr2, f2_pack(pr.x, pr.y));
           }
-          tmem_st16(tS + q * 16, pk);
+          if constexpr (!FP8) tmem_st16(tS + q * 16, pk);
         }
+        if constexpr (FP8) tmem_st16(tS, pk8);
       };
       if (need_mask)
         exp_pass(std::false_type{});
@@ -355,7 +391,7 @@ __global__ void __launch_bounds__(384, 1)
     const float L = l + red_sum[(0 * 2 + (half ^ 1)) * 128 + row];
     const float LR = l_r + red_sum[(1 * 2 + (half ^ 1)) * 128 + row];
     const bool valid = i < Lq;
-    const float inv_l = (LR > 0.f) ? 1.f / LR : 0.f;
+    const float inv_l = (LR > 0.f) ? p.v_descale / LR : 0.f;
     uint16_t* orow;
     if (p.cu_q != nullptr)
       orow = reinterpret_cast<uint16_t*>(p.o) + ((size_t)(q_row0 + i) * p.H + h) * D;
@@ -385,7 +421,8 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     if (valid && half == 0) {
-      const float lse = (L > 0.f) ? (m + lg2_approx(L)) * 0.69314718055994530942f : INFINITY;
+      const float lse =
+          (L > 0.f) ? (m - POFF + lg2_approx(L)) * 0.69314718055994530942f : INFINITY;
       if (p.cu_q != nullptr)
         p.lse[(size_t)h * p.total_q + q_row0 + i] = lse;
       else

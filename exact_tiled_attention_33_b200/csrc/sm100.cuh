@@ -230,6 +230,27 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// The same two products for 8-bit operands (.kind::f8f6f4; both operands E4M3 here, the
+// instruction descriptor's format code 0).  K per instruction is 32 elements (32 bytes).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05 async operation this thread issued so far
 // has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -384,6 +405,26 @@ __device__ __forceinline__ float2 exp2_poly2(float a, float b) {
   const uint32_t eb = (__float_as_uint(tf.y) - 0x4B400000u) << 23;
   return make_float2(__uint_as_float(__float_as_uint(pf.x) + ea),
                      __uint_as_float(__float_as_uint(pf.y) + eb));
+}
+
+// Round two fp32 values to E4M3 (nearest-even, saturating at ±448) and pack them into 16
+// bits, lo = first (lower byte).
+__device__ __forceinline__ uint32_t pack2_e4m3(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return (uint32_t)r;
+}
+// The two E4M3 values of the low 16 bits back to fp32 (exact), lo = first.
+__device__ __forceinline__ float2 unpack2_e4m3(uint32_t v) {
+  uint32_t h2;
+  const uint16_t b = (uint16_t)(v & 0xFFFFu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(b));
+  float lo, hi;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h2));
+  return make_float2(lo, hi);
 }
 
 // Unpack two 16-bit floats (lo = first) to fp32.

@@ -47,6 +47,7 @@ class Workload:
     qk_mult: float = 1.0
     scale: Optional[float] = None    # default 1/sqrt(d)
     window: Optional[tuple] = None   # sliding window (left, right); None: `causal` decides
+    fp8: bool = False                # q, k, v quantised to E4M3 (dtype: the output's format)
 
     @property
     def varlen(self) -> bool:
@@ -97,6 +98,8 @@ class Workload:
             out["qk_mult"] = self.qk_mult
         if self.window is not None:
             out["window"] = list(self.window)
+        if self.fp8:
+            out["inputs"] = "e4m3, per-tensor descale"
         return out
 
 
@@ -145,6 +148,11 @@ def _registry():
                      seed=4))
         add(Workload(f"long_peaky_{c}", B=2, H=32, N=16384, d=128, dtype="bf16",
                      causal=causal, seed=4, qk_mult=4.0))
+    # FP8 (E4M3) inputs at the long-context size, per-tensor scales
+    for causal in (False, True):
+        c = "causal" if causal else "noncausal"
+        add(Workload(f"fp8_long_{c}", B=2, H=32, N=16384, d=128, dtype="bf16", causal=causal,
+                     seed=4, fp8=True))
     # sliding-window (local) attention at the long-context size: each query sees the 4096
     # keys ending at its own position (a causal window of 4096), and a symmetric window
     add(Workload("long_local_w4096", B=2, H=32, N=16384, d=128, dtype="bf16", causal=True,
@@ -166,15 +174,15 @@ def get(name: str) -> Workload:
 
 
 def custom(name="custom", *, B=1, N=128, H=1, d=64, dtype="bf16", causal=False, seed=0,
-           seqlens=None, qk_mult=1.0, scale=None, window=None) -> Workload:
+           seqlens=None, qk_mult=1.0, scale=None, window=None, fp8=False) -> Workload:
     """An ad-hoc workload (ragged sizes, edge cases) built with the same recipe."""
     window = None if window is None else (int(window[0]), int(window[1]))
     if seqlens is not None:
         return Workload(name, H=H, d=d, dtype=dtype, causal=causal, seed=seed,
                         seqlens=tuple(int(x) for x in seqlens), qk_mult=qk_mult, scale=scale,
-                        window=window)
+                        window=window, fp8=fp8)
     return Workload(name, B=B, N=N, H=H, d=d, dtype=dtype, causal=causal, seed=seed,
-                    qk_mult=qk_mult, scale=scale, window=window)
+                    qk_mult=qk_mult, scale=scale, window=window, fp8=fp8)
 
 
 def generate(w: Workload, with_grad_out: bool = True):
@@ -196,6 +204,16 @@ def generate(w: Workload, with_grad_out: bool = True):
         out["do"] = torch.randn(shape, generator=g, dtype=torch.float32).to(w.torch_dtype)
     if w.varlen:
         out["cu_seqlens"] = torch.from_numpy(w.cu_seqlens())
+    if w.fp8:
+        # per-tensor scaling to the E4M3 range: descale = amax / 448, codes = x / descale
+        # rounded to nearest (PyTorch's float8_e4m3fn cast); the 16-bit q, k, v above are
+        # replaced by the exactly representable dequantised values
+        for name, x in (("q", q), ("k", k), ("v", v)):
+            descale = float(x.abs().max()) / 448.0
+            x8 = (x / descale).to(torch.float8_e4m3fn)
+            out[name + "8"] = x8
+            out[name + "_descale"] = descale
+            out[name] = (x8.to(torch.float32) * descale).to(w.torch_dtype)
     return out
 
 

@@ -146,6 +146,31 @@ int fa_varlen_bwd_local(const void* q, const void* k, const void* v, const void*
                         int window_right, int num_seqs, int total_q, int total_k,
                         void* workspace, size_t workspace_bytes, int dtype, void* stream);
 
+/* ---------------------------------------------------------------- FP8 forward
+ * Forward pass with 8-bit inputs: the pages credit FP8 tensor-core support to Hopper and
+ * quote FP8 attention at over 1.2 PFLOPS with an 8-bit quantization strategy (page
+ * "FlashAttention实战：如何在A100上实现3倍加速的Transformer训练" §7, page "Flash
+ * Attention V3：大模型训练加速与显存优化技术解析" §2.1) without fixing a format or scaling.
+ * Read here as: q, k, v hold OCP FP8 E4M3 bytes, one dequantisation factor per tensor, and
+ * the result is fa_fwd's O and LSE for the real inputs q_descale·Q8, k_descale·K8,
+ * v_descale·V8 (layouts as fa_fwd / fa_varlen_fwd with 1-byte elements).
+ * Both products run on the 8-bit tensor cores with fp32 accumulation; the softmax weights
+ * P are themselves rounded to E4M3 (scaled into its normal range) for the P·V product and
+ * O is normalised by the sum of the rounded weights, so O carries a relative error of at
+ * most 2^-4/(1 - 2^-4) of sum_j P_ij |v_j - O_i| (per element) beyond the 16-bit output
+ * rounding; LSE is computed from the unrounded weights (fa_fwd's accuracy).
+ * d must be 128; scale finite and >= 0; descale factors finite and > 0.  o is written in
+ * out_dtype (FA_BF16 or FA_FP16). */
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N,
+               int H, int d, float scale, float q_descale, float k_descale, float v_descale,
+               int causal, int out_dtype, void* stream);
+
+int fa_varlen_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                      const int* cu_seqlens_q, const int* cu_seqlens_k, int max_seqlen_q,
+                      int max_seqlen_k, int H, int d, float scale, float q_descale,
+                      float k_descale, float v_descale, int causal, int num_seqs, int total_q,
+                      int total_k, int out_dtype, void* stream);
+
 /* ---------------------------------------------------------------- KV-cache decode
  * One incremental-decoding step: Nq new query tokens per sequence (1 <= Nq <= 16) attend
  * to the keys and values that sequence has cached.  KV caches for incremental decoding

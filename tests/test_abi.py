@@ -142,3 +142,15 @@ def test_decode_validation(lib):
     splits = 5  # ceil(1184 / 256) = 5 splits of ceil(128 / 5) = 26 tiles (5 x 26 >= 128)
     rows = 8 * 1 * 32 * splits
     assert n == -(-rows * 128 * 4 // 256) * 256 + -(-rows * 4 // 256) * 256
+
+
+def test_fp8_validation(lib):
+    # FP8 forward: head_dim 128 only, scale >= 0, descale factors > 0
+    assert lib.fa_fwd_fp8(P, P, P, P, P, 1, 128, 1, 64, 0.1, 1.0, 1.0, 1.0, 0, 0, None) == \
+        _lib.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_fp8(P, P, P, P, P, 1, 128, 1, 128, -0.1, 1.0, 1.0, 1.0, 0, 0, None) == \
+        _lib.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_fp8(P, P, P, P, P, 1, 128, 1, 128, 0.1, 0.0, 1.0, 1.0, 0, 0, None) == \
+        _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_fp8(None, None, None, None, None, 0, 128, 1, 128, 0.1, 1.0, 1.0, 1.0, 0, 0,
+                          None) == _lib.FA_OK
