@@ -43,10 +43,14 @@ struct FwdCfg {
   static constexpr int KCH = D * EB / 128;      // 128-byte column chunks per row
   static constexpr int CHUNK = 128 * 128;
   static constexpr int TILE = 128 * D * EB;
+  // Each V stage carries one more 128-byte column chunk filled with ones: the P·V product
+  // then also yields, in O columns D..D+15, the row sum of the rounded P it used.
+  static constexpr int NO = D + 16;                    // O columns in tensor memory
+  static constexpr int VSTAGE = (KCH + 1) * CHUNK;     // V tile + the ones chunk
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + TILE;
   static constexpr int OFF_V = OFF_K + STAGES * TILE;
-  static constexpr int OFF_RED = OFF_V + STAGES * TILE;  // max exchange [2][2][128], sums [2][2][128]
+  static constexpr int OFF_RED = OFF_V + STAGES * VSTAGE;  // max exchange [2][2][128], sums [2][128]
   static constexpr int OFF_BAR = OFF_RED + 4 * 2 * 128 * 4;
   static constexpr int B_QFULL = 0;
   static constexpr int B_KFULL = 1;
@@ -63,7 +67,10 @@ struct FwdCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TM_O = 256;
   // pairs of every 16 (per 32-column chunk) whose exponentials use exp2_poly2
-  static constexpr int kPolyPairs = 4;
+#ifndef FATTN_POLY_PAIRS
+#define FATTN_POLY_PAIRS 2
+#endif
+  static constexpr int kPolyPairs = FATTN_POLY_PAIRS;
   // packed P column for the kk-th K step of a 128-key tile.  16-bit P (16 keys per step,
   // 2 per column): half 0 packs into columns 0..31 of its S buffer, half 1 into 64..95.
   // 8-bit P (32 keys per step, 4 per column): half 0 into 0..15, half 1 into 64..79.
@@ -80,11 +87,11 @@ __global__ void __launch_bounds__(384, 1)
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D, FP8>;
   constexpr int EL = 128 / C::EB;  // elements per 128-byte chunk (TMA x step)
-  // 8-bit P is scaled by 2^8 (p = 2^(x - m + 8)) so that it spans the normal E4M3 range,
-  // and the reference maximum is refreshed as soon as the row maximum grows by 0.5 so that
-  // p stays below 2^8.5 < 448; 16-bit P keeps p = 2^(x - m) with the lazy threshold 8.
-  constexpr float POFF = FP8 ? 8.f : 0.f;
-  constexpr float LAZY = FP8 ? 0.5f : 8.f;
+  // 8-bit P is scaled by 2^6 (p = 2^(x - m + 6)) so that it spans the normal E4M3 range,
+  // and the reference maximum is refreshed once the row maximum grows by more than 2.5, so
+  // that p stays below 2^8.5 < 448; 16-bit P keeps p = 2^(x - m) with the lazy threshold 8.
+  constexpr float POFF = FP8 ? 6.f : 0.f;
+  constexpr float LAZY = FP8 ? 2.5f : 8.f;
   constexpr int BM = C::BM, BN = C::BN, ST = C::STAGES;
 
   extern __shared__ uint8_t smem_raw[];
@@ -146,6 +153,16 @@ __global__ void __launch_bounds__(384, 1)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
+  {
+    // the ones chunk of every V stage (1.0 in the operand format), for the tensor core
+    const uint32_t one = FP8 ? 0x38383838u : (BF16 ? 0x3F803F80u : 0x3C003C00u);
+    for (int e = threadIdx.x; e < ST * (C::CHUNK / 16); e += C::THREADS) {
+      const int s = e / (C::CHUNK / 16), w = e % (C::CHUNK / 16);
+      *reinterpret_cast<uint4*>(sgen + C::OFF_V + s * C::VSTAGE + C::KCH * C::CHUNK + w * 16) =
+          make_uint4(one, one, one, one);
+    }
+    fence_proxy_async_smem();  // visible to the tensor core (async proxy)
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -172,7 +189,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_wait(BAR(C::B_VEMPTY + s), ph ^ 1u, abort_flag, p.status);
         mbar_arrive_expect_tx(BAR(C::B_VFULL + s), C::TILE);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_4d(&tmV, BAR(C::B_VFULL + s), sbase + C::OFF_V + s * C::TILE + c * C::CHUNK,
+          tma_load_4d(&tmV, BAR(C::B_VFULL + s), sbase + C::OFF_V + s * C::VSTAGE + c * C::CHUNK,
                       c * EL, h, k_row0 + (j0 + j) * BN, bcoord);
       }
     }
@@ -185,7 +202,7 @@ __global__ void __launch_bounds__(384, 1)
       // (format code 0 is f16 for .kind::f16 and E4M3 for .kind::f8f6f4)
       constexpr uint32_t ID_S0 = idesc_f16_f32acc(BF16 && !FP8, BM, BN, false, false);
       const uint32_t ID_S = ID_S0 | (p.negate_scores ? (1u << 13) : 0u);  // bit 13: negate A
-      constexpr uint32_t ID_O = idesc_f16_f32acc(BF16 && !FP8, BM, D, false, true);
+      constexpr uint32_t ID_O = idesc_f16_f32acc(BF16 && !FP8, BM, C::NO, false, true);
       // Descriptors built once; each MMA only adds a compile-time offset.
       const uint64_t dQ = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
       const uint64_t dK0 = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
@@ -216,7 +233,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_wait(BAR(C::B_PFULL), (uint32_t)j & 1u, abort_flag, p.status);
         mbar_wait(BAR(C::B_VFULL + s), (uint32_t)(j / ST) & 1u, abort_flag, p.status);
         tc_fence_after();
-        const uint64_t db = sdesc_adv(dV0, (uint32_t)(s * C::TILE));
+        const uint64_t db = sdesc_adv(dV0, (uint32_t)(s * C::VSTAGE));
         const uint32_t src = tmem + 128u * (uint32_t)(j & 1);
 #pragma unroll
         for (int kk = 0; kk < BN / C::KSTEP; ++kk) {
@@ -246,9 +263,9 @@ __global__ void __launch_bounds__(384, 1)
     const float c = p.scale_log2;      // > 0: scores are handled as x = s * |scale| * log2(e)
     float m = -INFINITY;               // reference maximum of x shared by l and O
     float l = 0.f;                     // Σ p over this half's columns (fp32), for the LSE
-    float l_r = 0.f;                   // Σ of the 16-bit P of this half (normalises O)
+    // (the row sum of the rounded P that normalises O accumulates in O's extra columns)
     float* red_max = red;              // [parity][half][row]
-    float* red_sum = red + 2 * 2 * 128;  // [2][half][row]: l, l_r at the end
+    float* red_sum = red + 2 * 2 * 128;  // [half][row]: l at the end
 
     for (int j = 0; j < n_kv; ++j) {
       const int b = j & 1;
@@ -302,15 +319,16 @@ __global__ void __launch_bounds__(384, 1)
         rescale = true;
       }
       const float m_use = (m == -INFINITY) ? 0.f : m;
-      // p = 2^(s*c - m).  l sums the fp32 p (log-sum-exp); l_r sums the 16-bit values the
-      // P·V product uses and normalises O, so numerator and denominator share the
-      // rounding of P (under the lazy maximum the largest P of a row is 2^δ, not 1).
+      // p = 2^(s*c - m).  l sums the fp32 p (log-sum-exp).  O is normalised by the row sum
+      // of the rounded P that the P·V product itself accumulates in O's extra columns, so
+      // numerator and denominator share the rounding of P (under the lazy maximum the
+      // largest P of a row is 2^δ, not 1).
       const uint64_t c2 = f2_pack(c, c);
       const uint64_t nm2 = f2_pack(POFF - m_use, POFF - m_use);
-      uint64_t ls2 = 0ull, lr2 = 0ull;
-      // A quarter of the exponentials run on the FMA pipe (tiles without masked keys), the
-      // rest on the special-function unit; the choice is made once per tile so the loop
-      // bodies stay branch-free.
+      uint64_t ls2 = 0ull;
+      // kPolyPairs of every 16 pairs of exponentials run on the FMA pipe (tiles without
+      // masked keys), the rest on the special-function unit; the choice is made once per
+      // tile so the loop bodies stay branch-free.
       auto exp_pass = [&](auto use_poly) {
         [[maybe_unused]] uint32_t pk8[16];  // 8-bit P: four keys per 32-bit column
 #pragma unroll
@@ -331,20 +349,16 @@ __global__ void __launch_bounds__(384, 1)
               p0 = ex2_approx(xx.x);
               p1 = ex2_approx(xx.y);
             }
-            float2 pr;
             if constexpr (FP8) {
               const uint32_t h8 = pack2_e4m3(p0, p1);
-              pr = unpack2_e4m3(h8);
               if (e & 1)
                 pk8[q * 8 + (e >> 1)] |= h8 << 16;
               else
                 pk8[q * 8 + (e >> 1)] = h8;
             } else {
               pk[e] = pack2<BF16>(p0, p1);
-              pr = unpack2<BF16>(pk[e]);
             }
             ls2 = f2_add(ls2, f2_pack(p0, p1));
-            lr2 = f2_add(lr2, f2_pack(pr.x, pr.y));
           }
           if constexpr (!FP8) tmem_st16(tS + q * 16, pk);
         }
@@ -354,9 +368,8 @@ __global__ void __launch_bounds__(384, 1)
         exp_pass(std::false_type{});
       else
         exp_pass(std::true_type{});
-      const float2 ls = f2_unpack(ls2), lr = f2_unpack(lr2);
+      const float2 ls = f2_unpack(ls2);
       l = l * alpha + (ls.x + ls.y);
-      l_r = l_r * alpha + (lr.x + lr.y);
 
       if (__any_sync(0xffffffffu, rescale)) {
         // O was last written by the P·V product of tile j-1: wait until it completed, then
@@ -374,6 +387,15 @@ __global__ void __launch_bounds__(384, 1)
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
           tmem_st32(tO + q * 32, o);
         }
+        if (half == 1) {  // the rounded-P row sum columns D..D+15 scale with O
+          uint32_t o[16];
+          tmem_ld16(tmem + lane_off + C::TM_O + D, o);
+          tmem_wait_ld();
+          reg_fence(o);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st16(tmem + lane_off + C::TM_O + D, o);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -385,11 +407,17 @@ __global__ void __launch_bounds__(384, 1)
       mbar_wait(BAR(C::B_ODONE), (uint32_t)(n_kv - 1) & 1u, abort_flag, p.status);
       tc_fence_after();
     }
-    red_sum[(0 * 2 + half) * 128 + row] = l;
-    red_sum[(1 * 2 + half) * 128 + row] = l_r;
+    red_sum[half * 128 + row] = l;
     named_barrier_sync(1, 256);
-    const float L = l + red_sum[(0 * 2 + (half ^ 1)) * 128 + row];
-    const float LR = l_r + red_sum[(1 * 2 + (half ^ 1)) * 128 + row];
+    const float L = l + red_sum[(half ^ 1) * 128 + row];
+    float LR = 0.f;  // row sum of the rounded P (O column D)
+    if (n_kv > 0) {
+      uint32_t o[16];
+      tmem_ld16(tmem + lane_off + C::TM_O + D, o);
+      tmem_wait_ld();
+      reg_fence(o);
+      LR = __uint_as_float(o[0]);
+    }
     const bool valid = i < Lq;
     const float inv_l = (LR > 0.f) ? p.v_descale / LR : 0.f;
     uint16_t* orow;
