@@ -107,14 +107,14 @@ struct BwdCfg {
   static constexpr int A_OFF_DO = A_OFF_Q + STAGES * TILE;
   static constexpr int A_OFF_VEC = A_OFF_DO + STAGES * TILE;  // per stage: -lse*log2e, D
   static constexpr int A_OFF_BAR = A_OFF_VEC + STAGES * 2 * BM * 4;
-  // dQ kernel: Q, dO resident; K streamed through 3 stages (it is needed from the S
-  // product two steps ahead until the dQ product), V through 2
+  // dQ kernel: Q and dO resident in tensor memory (the A operands of S and dP); K streamed
+  // through 3 stages (it is needed from the S product one step ahead until the dQ
+  // product), V through 3
   static constexpr int K_STAGES = 3;
-  static constexpr int B_OFF_Q = 0;
-  static constexpr int B_OFF_DO = B_OFF_Q + TILE;
-  static constexpr int B_OFF_K = B_OFF_DO + TILE;
+  static constexpr int V_STAGES = 3;
+  static constexpr int B_OFF_K = 0;
   static constexpr int B_OFF_V = B_OFF_K + K_STAGES * TILE;
-  static constexpr int B_OFF_BAR = B_OFF_V + STAGES * TILE;
+  static constexpr int B_OFF_BAR = B_OFF_V + V_STAGES * TILE;
   static constexpr int NBAR = 24;  // mbarrier slots reserved in either kernel
   static constexpr int SMEM_A = A_OFF_BAR + 8 * NBAR + 16 + 1024;
   static constexpr int SMEM_B = B_OFF_BAR + 8 * NBAR + 16 + 1024;
@@ -451,8 +451,12 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // ------------------------------------------------------------------ dQ
-// Tensor memory: S two buffers [0,128), [128,256) | dP [256,384) (dS packed into it) |
-// dQ [384, 384+D).
+// One CTA per 128-row query tile, walking the key tiles it can see.
+// Tensor memory: S [0,128) | dP [128,256) (dS packed into it) | dQ [256, 256+D) |
+// Q [384, 384+D/2) and dO [448, 448+D/2) packed 16-bit: the A operands of S = Q Kᵀ and
+// dP = dO Vᵀ come from tensor memory, so per step the tensor core reads only K (twice)
+// and V from shared memory.  S has one buffer, released as soon as the compute warps have
+// loaded it, so S of the next step is computed while they exponentiate.
 // Grid: x = query tile (fastest, sharing one head's K/V in L2; when causal the tile
 // that sees the most key tiles first), y = head, z = batch or sequence.
 template <int D, bool BF16>
@@ -461,12 +465,12 @@ __global__ void __launch_bounds__(384, 1)
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                      const BwdParams p) {
   using C = BwdCfg<D>;
-  constexpr int BM = C::BM, BN = C::BN, ST = C::STAGES;
-  constexpr uint32_t TM_DP = 256, TM_DQ = 384;
+  constexpr int BM = C::BM, BN = C::BN, VST = C::V_STAGES;
+  constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256, TM_QT = 384, TM_DOT = 448;
   constexpr int KST = C::K_STAGES;
-  enum { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KST, B_VFULL = B_KEMPTY + KST,
-         B_VEMPTY = B_VFULL + ST, B_SFULL = B_VEMPTY + ST, B_SEMPTY = B_SFULL + 2,
-         B_DPFULL = B_SEMPTY + 2, B_DSFULL, B_DONE };
+  enum { B_QTM = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KST, B_VFULL = B_KEMPTY + KST,
+         B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST, B_SEMPTY, B_DPFULL, B_DSFULL,
+         B_DONE };
   static_assert(B_DONE < C::NBAR, "mbarrier slots");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -501,19 +505,17 @@ __global__ void __launch_bounds__(384, 1)
   key_tile_range(q0, min(q0 + BM - 1, Lq - 1), Lk, diag, wl, wr, BN, &j0, &n_kv);
 
   if (threadIdx.x == 0) {
-    mbar_init(BAR(B_QFULL), 1);
+    mbar_init(BAR(B_QTM), 256);
     for (int s = 0; s < KST; ++s) {
       mbar_init(BAR(B_KFULL + s), 1);
       mbar_init(BAR(B_KEMPTY + s), 1);
     }
-    for (int s = 0; s < ST; ++s) {
+    for (int s = 0; s < VST; ++s) {
       mbar_init(BAR(B_VFULL + s), 1);
       mbar_init(BAR(B_VEMPTY + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(BAR(B_SFULL + b), 1);
-      mbar_init(BAR(B_SEMPTY + b), 256);
-    }
+    mbar_init(BAR(B_SFULL), 1);
+    mbar_init(BAR(B_SEMPTY), 256);
     mbar_init(BAR(B_DPFULL), 1);
     mbar_init(BAR(B_DSFULL), 256);
     mbar_init(BAR(B_DONE), 1);
@@ -532,25 +534,16 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 0) {
     // ============================================================ loads
     if (lane == 0 && n_kv > 0) {
-      tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      tma_prefetch_desc(&tmDO);
-      mbar_arrive_expect_tx(BAR(B_QFULL), 2 * C::TILE);
-      for (int c = 0; c < C::KCH; ++c) {
-        tma_load_4d(&tmQ, BAR(B_QFULL), sbase + C::B_OFF_Q + c * C::CHUNK, c * 64, h, q_row0 + q0,
-                    bcoord);
-        tma_load_4d(&tmDO, BAR(B_QFULL), sbase + C::B_OFF_DO + c * C::CHUNK, c * 64, h, q_row0 + q0,
-                    bcoord);
-      }
       for (int j = 0; j < n_kv; ++j) {
-        const int ks = j % KST, s = j % ST;
+        const int ks = j % KST, s = j % VST;
         mbar_wait(BAR(B_KEMPTY + ks), ((uint32_t)(j / KST) & 1u) ^ 1u, abort_flag, p.status);
         mbar_arrive_expect_tx(BAR(B_KFULL + ks), C::TILE);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(&tmK, BAR(B_KFULL + ks), sbase + C::B_OFF_K + ks * C::TILE + c * C::CHUNK,
                       c * 64, h, k_row0 + (j0 + j) * BN, bcoord);
-        mbar_wait(BAR(B_VEMPTY + s), ((uint32_t)(j / ST) & 1u) ^ 1u, abort_flag, p.status);
+        mbar_wait(BAR(B_VEMPTY + s), ((uint32_t)(j / VST) & 1u) ^ 1u, abort_flag, p.status);
         mbar_arrive_expect_tx(BAR(B_VFULL + s), C::TILE);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(&tmV, BAR(B_VFULL + s), sbase + C::B_OFF_V + s * C::TILE + c * C::CHUNK,
@@ -564,40 +557,44 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t ID_S = idesc_f16_f32acc(BF16, 128, 128, false, false);   // S, dP
       constexpr uint32_t ID_DQ = idesc_f16_f32acc(BF16, 128, D, false, true);     // dQ
       // Descriptors built once; each MMA only adds a compile-time offset.
-      const uint64_t dQ = sdesc_sw128(sbase + C::B_OFF_Q, 16, 1024);
-      const uint64_t dDO = sdesc_sw128(sbase + C::B_OFF_DO, 16, 1024);
       const uint64_t dKk = sdesc_sw128(sbase + C::B_OFF_K, 16, 1024);         // K-major
       const uint64_t dKm = sdesc_sw128(sbase + C::B_OFF_K, C::CHUNK, 1024);   // MN-major
       const uint64_t dVk = sdesc_sw128(sbase + C::B_OFF_V, 16, 1024);
-      auto issue_qt = [&](uint32_t dst, uint64_t da, uint64_t db) {
+      // X = A Bᵀ with A (queries x d) packed in tensor memory and B = [keys][d] in shared
+      // memory: K step kk covers d-elements 16kk.. = tensor-memory columns 8kk..
+      auto issue_qt = [&](uint32_t dst, uint32_t a_tm, uint64_t db) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + dst, sdesc_adv(da, off), sdesc_adv(db, off), ID_S, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ts(tmem + dst, tmem + a_tm + 8u * kk,
+                 sdesc_adv(db, (kk >> 2) * C::CHUNK + (kk & 3) * 32), ID_S, kk > 0 ? 1u : 0u);
       };
-      auto issue_s = [&](int j) {  // S_j = Q K_jᵀ into buffer j % 2
-        const int ks = j % KST, b = j & 1;
-        if (j >= 2) mbar_wait(BAR(B_SEMPTY + b), ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, p.status);
+      auto issue_s = [&](int j) {  // S_j = Q K_jᵀ
+        const int ks = j % KST;
         mbar_wait(BAR(B_KFULL + ks), (uint32_t)(j / KST) & 1u, abort_flag, p.status);
         tc_fence_after();
-        issue_qt(128u * b, dQ, sdesc_adv(dKk, ks * C::TILE));
-        mma_commit(BAR(B_SFULL + b));
+        issue_qt(TM_S, TM_QT, sdesc_adv(dKk, ks * C::TILE));
+        mma_commit(BAR(B_SFULL));
       };
       auto issue_dp = [&](int j) {  // dP_j = dO V_jᵀ; V_j is free once it completes
-        const int s = j % ST;
-        mbar_wait(BAR(B_VFULL + s), (uint32_t)(j / ST) & 1u, abort_flag, p.status);
+        const int s = j % VST;
+        mbar_wait(BAR(B_VFULL + s), (uint32_t)(j / VST) & 1u, abort_flag, p.status);
         tc_fence_after();
-        issue_qt(TM_DP, dDO, sdesc_adv(dVk, s * C::TILE));
+        issue_qt(TM_DP, TM_DOT, sdesc_adv(dVk, s * C::TILE));
         mma_commit(BAR(B_DPFULL));
         mma_commit(BAR(B_VEMPTY + s));
       };
-      mbar_wait(BAR(B_QFULL), 0, abort_flag, p.status);
+      mbar_wait(BAR(B_QTM), 0, abort_flag, p.status);  // Q and dO are in tensor memory
+      tc_fence_after();
       issue_s(0);
-      if (n_kv > 1) issue_s(1);
       issue_dp(0);
       for (int j = 0; j < n_kv; ++j) {
         const int ks = j % KST;
+        // S_{j+1} as soon as the compute warps have loaded S_j
+        if (j + 1 < n_kv) {
+          mbar_wait(BAR(B_SEMPTY), (uint32_t)j & 1u, abort_flag, p.status);
+          tc_fence_after();
+          issue_s(j + 1);
+        }
         // dQ += dS K_j  (A = dS in tensor memory; B = K_j as [d x keys], d-contiguous)
         mbar_wait(BAR(B_DSFULL), (uint32_t)j & 1u, abort_flag, p.status);
         tc_fence_after();
@@ -607,10 +604,8 @@ __global__ void __launch_bounds__(384, 1)
           mma_ts(tmem + TM_DQ, tmem + TM_DP + C::packed_col(kk), sdesc_adv(kb, kk * 2048), ID_DQ,
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(BAR(B_KEMPTY + ks));
-        // dP of the next step goes first (the compute warps wait for it); it overwrites
-        // dS_j only after the product above that reads it (in-order pipe).
+        // dP_{j+1} overwrites dS_j only after the product above that reads it (in-order)
         if (j + 1 < n_kv) issue_dp(j + 1);
-        if (j + 2 < n_kv) issue_s(j + 2);
       }
       mma_commit(BAR(B_DONE));
     }
@@ -622,7 +617,32 @@ __global__ void __launch_bounds__(384, 1)
     const int r = quarter * 32 + lane;  // query row within the tile
     const int i = q0 + r;               // query index within the sequence
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + TM_S + 64 * half;
     const uint32_t tDP = tmem + lane_off + TM_DP + 64 * half;
+    const size_t grow = (p.cu_q != nullptr) ? ((size_t)(q_row0 + i) * p.H + h) * D
+                                            : (((size_t)bcoord * p.N + i) * p.H + h) * D;
+    {
+      // this thread's row of Q (half 0) or dO (half 1) into tensor memory, packed 16-bit
+      const uint4* src = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const uint16_t*>(half == 0 ? p.q : p.dout) + grow);
+      const uint32_t dst = tmem + lane_off + (half == 0 ? TM_QT : TM_DOT);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t w[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = (i < Lq) ? src[c * 8 + u] : make_uint4(0u, 0u, 0u, 0u);
+          w[4 * u] = v.x;
+          w[4 * u + 1] = v.y;
+          w[4 * u + 2] = v.z;
+          w[4 * u + 3] = v.w;
+        }
+        tmem_st32(dst + 32u * c, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR(B_QTM));
+    }
     const float kLog2e = 1.4426950408889634f;
     float nl2 = -INFINITY, dd = 0.f;  // this row's -LSE·log2(e) and D
     if (i < Lq) {
@@ -635,7 +655,6 @@ __global__ void __launch_bounds__(384, 1)
     const uint64_t nl22 = f2_pack(nl2, nl2);
     const uint64_t nd2 = f2_pack(-dd, -dd);
     for (int j = 0; j < n_kv; ++j) {
-      const int b = j & 1;
       const int kt = (j0 + j) * BN;       // first key of the tile
       const int k0 = kt + 64 * half;      // first key of this thread's columns
       const bool need_mask = (kt + BN > Lk) || (wr >= 0 && kt + BN - 1 > q0 + diag + wr) ||
@@ -643,16 +662,15 @@ __global__ void __launch_bounds__(384, 1)
       // allowed columns: lo <= c < lim
       const int lim = wr >= 0 ? min(Lk - k0, i + diag + wr - k0 + 1) : Lk - k0;
       const int lo = wl >= 0 ? i + diag - wl - k0 : 0;
-      mbar_wait(BAR(B_SFULL + b), (uint32_t)(j >> 1) & 1u, abort_flag, p.status);
+      mbar_wait(BAR(B_SFULL), (uint32_t)j & 1u, abort_flag, p.status);
       tc_fence_after();
       uint32_t sv[64];
-      const uint32_t tS = tmem + lane_off + 128u * b + 64 * half;
       tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
       reg_fence(sv);
       tc_fence_before();
-      mbar_arrive(BAR(B_SEMPTY + b));  // the S buffer may be overwritten now
+      mbar_arrive(BAR(B_SEMPTY));  // S may be overwritten now
       float pv[64];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
