@@ -213,6 +213,73 @@ def run_reference(args, w):
     return 0
 
 
+# ------------------------------------------------------------------ N = 1K..4K sweep
+SWEEP = ["a100table_N1024", "a100table_N2048", "a100table_N4096", "llama_causal"]
+
+
+def sweep_small_n(lib, dev, reps: int = 10):
+    """Forward and forward+backward of the pages' smaller shapes (the A100-table B8 H16 d64
+    at N = 1K, 2K, 4K and the Llama-style B4 H32 d128 N=4K), one GPU.  Their inputs fit in
+    L2, so L2 is flushed (a 256 MB write) before every timed launch; each launch is timed
+    alone with CUDA events.  Reports TFLOPS and the forward's algorithmic HBM GB/s
+    (Q, K, V read once, O and LSE written once)."""
+    import torch
+    from exact_tiled_attention_33_b200 import _lib
+    from exact_tiled_attention_33_b200 import attention as fa
+    from exact_tiled_attention_33_b200 import workloads as wl
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    out = []
+    for name in SWEEP:
+        w = wl.get(name)
+        t = wl.generate(w)
+        q, k, v, do = (t[x].to(dev) for x in ("q", "k", "v", "do"))
+        B, N, H, d = q.shape
+        dt = _lib.FA_BF16 if w.dtype == "bf16" else _lib.FA_FP16
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = fa.bwd_workspace(B, N, H, d, dev)
+
+        def fwd():
+            _lib.check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  lse.data_ptr(), B, N, H, d, w.softmax_scale, int(w.causal), dt,
+                                  sh), "fa_fwd")
+
+        def bwd():
+            _lib.check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                  dv.data_ptr(), B, N, H, d, w.softmax_scale, int(w.causal),
+                                  ws.data_ptr(), ws.numel(), dt, sh), "fa_bwd")
+
+        def timed(fn):
+            ms = []
+            for _ in range(3):
+                fn()
+            for _ in range(reps):
+                flush.fill_(1)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize(dev)
+                ms.append(a.elapsed_time(b))
+            return statistics.median(ms)
+
+        f_ms, b_ms = timed(fwd), timed(bwd)
+        assert lib.fa_get_device_status(sh) == 0
+        f = w.fwd_flops()
+        e = q.numel() * q.element_size()
+        fwd_bytes = 4 * e + 4 * B * H * N
+        out.append({"workload": name, "B": B, "N": N, "H": H, "d": d, "causal": w.causal,
+                    "fwd_ms": f_ms, "bwd_ms": b_ms, "fwd_tflops": f / f_ms / 1e9,
+                    "fwd_bwd_tflops": 3.5 * f / (f_ms + b_ms) / 1e9,
+                    "fwd_hbm_gbs": fwd_bytes / f_ms / 1e6})
+    del flush
+    return out
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_fattn(args, w):
     import torch
@@ -357,6 +424,10 @@ def run_fattn(args, w):
                 "traffic": read_traffic("fa_fwd_kernel", wr.name, fwd_sha),
                 "flops_per_launch": f_fwd}
 
+    sweep = None
+    if rank == 0 and world == 1 and not args.no_sweep:
+        sweep = sweep_small_n(lib, dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = 512
@@ -385,7 +456,7 @@ def run_fattn(args, w):
                 "ms_fwd": fwd_avg, "ms_bwd": bwd_avg,
                 "gpu_launches": 4 * args.steps,
                 "roofline": roofline, "roofline_fwd": fwd_roof,
-                "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu}
+                "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "sweep_n1k_4k": sweep}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -793,6 +864,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="long_causal")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the N = 1K..4K sweep of the default bench line")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3) if args.impl == "fattn" else args.warmup
     from exact_tiled_attention_33_b200 import workloads as wl
