@@ -66,11 +66,16 @@ struct FwdCfg {
   static constexpr int THREADS = 384;  // warps 0 loads, 1 MMA, 2-3 idle, 4-11 softmax
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TM_O = 256;
-  // pairs of every 16 (per 32-column chunk) whose exponentials use exp2_poly2
+  // pairs of every 16 (per 32-column chunk) whose exponentials use exp2_poly2.  At d = 64
+  // a score carries half the tensor work of d = 128 for the same exponential, so a larger
+  // share moves to the FMA pipe there.
 #ifndef FATTN_POLY_PAIRS
 #define FATTN_POLY_PAIRS 2
 #endif
-  static constexpr int kPolyPairs = FATTN_POLY_PAIRS;
+#ifndef FATTN_POLY_PAIRS_D64
+#define FATTN_POLY_PAIRS_D64 6
+#endif
+  static constexpr int kPolyPairs = D == 64 ? FATTN_POLY_PAIRS_D64 : FATTN_POLY_PAIRS;
   // packed P column for the kk-th K step of a 128-key tile.  16-bit P (16 keys per step,
   // 2 per column): half 0 packs into columns 0..31 of its S buffer, half 1 into 64..95.
   // 8-bit P (32 keys per step, 4 per column): half 0 into 0..15, half 1 into 64..79.
