@@ -375,36 +375,81 @@ def run_fattn(args, w):
     fwd_avg = statistics.mean(fwd_ms)
     bwd_avg = statistics.mean(bwd_ms)
 
-    # ---- end to end through the C ABI with pinned host buffers (per step: H2D of q, k,
-    # v, dO; fwd; bwd; D2H of O, LSE, dQ, dK, dV)
+    # ---- end to end through the C ABI with pinned host buffers.  Every step copies its
+    # inputs q, k, v, dO host -> device, runs fwd + bwd and copies O, LSE, dQ, dK, dV back.
+    # Two device buffer sets and three streams pipeline the steps: the copies of one step
+    # overlap the compute of the previous / next step (H2D and D2H also run concurrently),
+    # as a training loop that feeds a GPU from host memory would.
     e2e = None
     if not args.no_e2e:
         hin = [host[x].pin_memory() for x in ("q", "k", "v", "do")]
-        hout = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (o, lse, dq, dk, dv)]
+        sets = []
+        for bset in range(2):
+            ins = [q, k, v, do] if bset == 0 else [torch.empty_like(x) for x in (q, k, v, do)]
+            outs = [o, lse, dq, dk, dv] if bset == 0 else [torch.empty_like(x)
+                                                          for x in (o, lse, dq, dk, dv)]
+            hout = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in outs]
+            wsb = ws if bset == 0 else fa.bwd_workspace(B, N, H, d, dev)
+            sets.append((ins, outs, hout, wsb))
         h2d = sum(x.numel() * x.element_size() for x in hin)
-        d2h = sum(x.numel() * x.element_size() for x in hout)
-        e2e_steps = max(2, min(args.steps, 5))
+        d2h = sum(x.numel() * x.element_size() for x in sets[0][2])
+        e2e_steps = max(4, min(args.steps, 8))
+        s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_cmp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            for hsrc, ddst in zip(hin, (q, k, v, do)):
-                ddst.copy_(hsrc, non_blocking=True)
-            step()
-            for dsrc, hdst in zip((o, lse, dq, dk, dv), hout):
-                hdst.copy_(dsrc, non_blocking=True)
+        def compute(ins, outs, wsb, hs):
+            qq, kk, vv, dd = (x.data_ptr() for x in ins)
+            oo, ll, gq, gk, gv = (x.data_ptr() for x in outs)
+            if wr.window is None:
+                _lib.check(lib.fa_fwd(qq, kk, vv, oo, ll, B, N, H, d, scale, causal, dtype, hs),
+                           "fa_fwd")
+                _lib.check(lib.fa_bwd(qq, kk, vv, oo, dd, ll, gq, gk, gv, B, N, H, d, scale,
+                                      causal, wsb.data_ptr(), wsb.numel(), dtype, hs), "fa_bwd")
+            else:
+                wl_, wr_ = wr.window
+                _lib.check(lib.fa_fwd_local(qq, kk, vv, oo, ll, B, N, H, d, scale, wl_, wr_,
+                                            dtype, hs), "fa_fwd_local")
+                _lib.check(lib.fa_bwd_local(qq, kk, vv, oo, dd, ll, gq, gk, gv, B, N, H, d,
+                                            scale, wl_, wr_, wsb.data_ptr(), wsb.numel(), dtype,
+                                            hs), "fa_bwd_local")
 
-        e2e_step()
+        def e2e_step(i):
+            ins, outs, hout, wsb = sets[i % 2]
+            b_ = i % 2
+            s_in.wait_event(ev_cmp[b_])            # inputs of this set consumed (step i - 2)
+            with torch.cuda.stream(s_in):
+                for hsrc, ddst in zip(hin, ins):
+                    ddst.copy_(hsrc, non_blocking=True)
+            ev_in[b_].record(s_in)
+            s_cmp.wait_event(ev_in[b_])
+            s_cmp.wait_event(ev_out[b_])           # outputs of this set copied out (step i - 2)
+            compute(ins, outs, wsb, s_cmp.cuda_stream)
+            ev_cmp[b_].record(s_cmp)
+            s_out.wait_event(ev_cmp[b_])
+            with torch.cuda.stream(s_out):
+                for dsrc, hdst in zip(outs, hout):
+                    hdst.copy_(dsrc, non_blocking=True)
+            ev_out[b_].record(s_out)
+
+        for i in range(2):                        # warm-up of the pipeline
+            e2e_step(i)
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        b.record(stream)
+        a.record(s_in)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        b.record(s_out)                           # after the last step's D2H (all in order)
         torch.cuda.synchronize(dev)
         e2e_s = max_over_ranks(a.elapsed_time(b) / 1e3, world)
         e2e = {"value": throughput_tflops(f_step, e2e_steps, world, e2e_s), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "pipelined": "2 buffer sets; H2D, compute, D2H on 3 streams"}
+        assert lib.fa_get_device_status(sh) == 0, "device status after e2e"
+        del sets
 
     peak_burst, peak_sust, hbm, peak_src = load_peaks()
     bwd_sha = sources_sha(BWD_SOURCES)
