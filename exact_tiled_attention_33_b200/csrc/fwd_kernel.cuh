@@ -22,7 +22,10 @@
 //     tile), update the reference maximum m identically, and keep partial row sums;
 //     each writes P over its own S columns as packed 16-bit values and rescales its half
 //     of O only when m grew by more than 2^8 (exact: O and l share the reference);
-//   * tensor memory: S_a | S_b | O (128 + 128 + D columns of 32 bits).
+//   * tensor memory: S_a | S_b | O (128 + 128 + D + 16 columns of 32 bits); the P·V
+//     product runs with 16 more columns of V that are all ones, so O's last 16 columns
+//     hold the row sum of the rounded P it used (the normaliser of O);
+//   * FP8 = true: E4M3 operands and 8-bit tensor-core products (d = 128).
 #pragma once
 
 #include <type_traits>
