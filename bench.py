@@ -224,7 +224,8 @@ SWEEP = ["a100table_N1024", "a100table_N2048", "a100table_N4096", "llama_causal"
 
 def sweep_small_n(lib, dev, reps: int = 10):
     """Forward and forward+backward of the pages' smaller shapes (the A100-table B8 H16 d64
-    at N = 1K, 2K, 4K and the Llama-style B4 H32 d128 N=4K), one GPU.  Their inputs fit in
+    at N = 1K, 2K, 4K, the Llama-style B4 H32 d128 N=4K and the 64-sequence packed varlen
+    batch), one GPU.  Their inputs fit in
     L2, so L2 is flushed (a 256 MB write) before every timed launch; each launch is timed
     alone with CUDA events.  Reports TFLOPS and the forward's algorithmic HBM GB/s
     (Q, K, V read once, O and LSE written once)."""
@@ -281,6 +282,29 @@ def sweep_small_n(lib, dev, reps: int = 10):
                     "fwd_ms": f_ms, "bwd_ms": b_ms, "fwd_tflops": f / f_ms / 1e9,
                     "fwd_bwd_tflops": 3.5 * f / (f_ms + b_ms) / 1e9,
                     "fwd_hbm_gbs": fwd_bytes / f_ms / 1e6})
+    # the packed variable-length batch: 64 sequences of 64..4096 tokens, H32 d128, causal
+    w = wl.get("varlen64")
+    t = wl.generate(w)
+    q, k, v, do = (t[x].to(dev) for x in ("q", "k", "v", "do"))
+    cu = t["cu_seqlens"].to(dev)
+    L = max(w.seqlens)
+    o, lse = fa.varlen_fwd(q, k, v, cu, cu, L, L, w.softmax_scale, True)
+    wsv = fa.varlen_bwd_workspace(q.shape[0], w.H, w.d, dev)
+
+    def vfwd():
+        fa.varlen_fwd(q, k, v, cu, cu, L, L, w.softmax_scale, True, out=o, lse=lse)
+
+    def vbwd():
+        fa.varlen_bwd(q, k, v, o, lse, do, cu, cu, L, L, w.softmax_scale, True, workspace=wsv)
+
+    f_ms, b_ms = timed(vfwd), timed(vbwd)
+    assert lib.fa_get_device_status(sh) == 0
+    f = w.fwd_flops()
+    e = q.numel() * q.element_size()
+    out.append({"workload": "varlen64", "num_seqs": len(w.seqlens), "total_tokens": w.total,
+                "H": w.H, "d": w.d, "causal": True, "fwd_ms": f_ms, "bwd_ms": b_ms,
+                "fwd_tflops": f / f_ms / 1e9, "fwd_bwd_tflops": 3.5 * f / (f_ms + b_ms) / 1e9,
+                "fwd_hbm_gbs": (4 * e + 4 * w.H * w.total) / f_ms / 1e6})
     del flush
     return out
 
