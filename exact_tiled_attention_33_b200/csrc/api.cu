@@ -236,6 +236,7 @@ int fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
   p.N = 0;
   p.H = H;
   p.total_q = total_q;
+  p.total_k = total_k;
   p.scale = scale;
   set_fwd_scale(p, scale);
   p.win_left = wl;
@@ -404,6 +405,7 @@ int fa_varlen_fwd_fp8(const void* q, const void* k, const void* v, void* o, floa
   p.cu_k = cu_seqlens_k;
   p.H = H;
   p.total_q = total_q;
+  p.total_k = total_k;
   p.scale = scale;
   set_fp8_scale(p, scale, q_descale, k_descale, v_descale);
   p.win_left = -1;
@@ -745,6 +747,10 @@ int fa_get_device_status(void* stream) {
     e = cudaMemcpy(sp, &zero, sizeof(zero), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(e, "clear status word");
     if (word & kDevTimeout) return fail(FA_ERR_TIMEOUT, "a kernel wait timed out");
+    if (word & kDevBadSeqlens)
+      return fail(FA_ERR_INVALID_ARG,
+                  "a varlen call saw cu_seqlens outside [0, total] or a sequence longer than "
+                  "max_seqlen (that sequence was skipped)");
     if (word & kDevBadCache)
       return fail(FA_ERR_INVALID_ARG,
                   "a decode call saw a cache length above its bounds or a page id out of range");

@@ -19,6 +19,7 @@ struct FwdParams {
   int N;            // dense sequence length
   int H;
   int total_q;      // varlen: rows of q/o (row stride of lse)
+  int total_k;      // varlen: rows of k/v
   float scale;      // softmax scale
   float scale_log2; // |scale| * log2(e), > 0 (a tiny positive value when scale == 0)
   int negate_scores;// 1 when scale < 0: the S product negates Q

@@ -15,7 +15,29 @@ namespace fattn {
 
 // ------------------------------------------------------------------ status word
 // Error codes a kernel can leave in the device status word (see fa_get_device_status).
-enum : uint32_t { kDevOk = 0u, kDevTimeout = 1u, kDevSmemAlign = 2u, kDevBadCache = 4u };
+enum : uint32_t {
+  kDevOk = 0u,
+  kDevTimeout = 1u,
+  kDevSmemAlign = 2u,
+  kDevBadCache = 4u,    // decode: cache length above its bound or page id out of range
+  kDevBadSeqlens = 8u,  // varlen: a segment outside [0, total) or longer than the grid
+};
+
+// Varlen segment bz read from device prefix sums, checked before any use: rows
+// [cu_q[bz], cu_q[bz+1]) must lie in [0, total_q) and keys likewise in [0, total_k), and the
+// segment must fit the rows (q_cover) or keys (k_cover) the grid covers (negative: not
+// checked).  A bad segment is reported in the status word and its CTA does nothing, so a
+// malformed cu_seqlens never leads to an out-of-bounds access.
+__device__ __forceinline__ bool varlen_segment_ok(const int* cu_q, const int* cu_k, int bz,
+                                                  int total_q, int total_k, long long q_cover,
+                                                  long long k_cover, uint32_t* status) {
+  const int q0 = cu_q[bz], q1 = cu_q[bz + 1], k0 = cu_k[bz], k1 = cu_k[bz + 1];
+  const bool ok = 0 <= q0 && q0 <= q1 && q1 <= total_q && 0 <= k0 && k0 <= k1 &&
+                  k1 <= total_k && (q_cover < 0 || q1 - q0 <= q_cover) &&
+                  (k_cover < 0 || k1 - k0 <= k_cover);
+  if (!ok && threadIdx.x == 0) atomicOr(status, kDevBadSeqlens);
+  return ok;
+}
 
 // Upper bound on a single mbarrier wait, in nanoseconds of %globaltimer.  A wait that
 // runs out records kDevTimeout and makes every later wait in the same CTA return at

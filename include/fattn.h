@@ -76,7 +76,11 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
  * Writes o [total_q,H,d] and lse [H,total_q].
  * max_seqlen_q / max_seqlen_k must be >= every sequence's length (they size the grid);
  * num_seqs, total_q, total_k are the host-side counts matching cu_seqlens (the host
- * cannot read device cu_seqlens without a synchronisation).  num_seqs <= 65535. */
+ * cannot read device cu_seqlens without a synchronisation).  num_seqs <= 65535.
+ * The kernels check every segment before using it: a segment outside [0, total_q) or
+ * [0, total_k), or longer than max_seqlen_q (forward, dQ) or max_seqlen_k (dK/dV), is
+ * skipped (its outputs are left unwritten) and fa_get_device_status then returns
+ * FA_ERR_INVALID_ARG; nothing is accessed out of bounds. */
 int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                   const int* cu_seqlens_q, const int* cu_seqlens_k, int max_seqlen_q,
                   int max_seqlen_k, int H, int d, float scale, int causal, int num_seqs,

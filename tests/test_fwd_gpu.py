@@ -246,3 +246,28 @@ def test_call_from_fresh_host_thread():
     assert not err, err
     torch.cuda.synchronize()
     assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
+
+
+def test_malformed_cu_seqlens_are_reported_not_followed():
+    # cu_seqlens live on the device, so the host cannot check them: a segment beyond the
+    # packed total, or longer than max_seqlen, is skipped by the kernels and reported as
+    # FA_ERR_INVALID_ARG; nothing is read or written out of bounds.
+    from exact_tiled_attention_33_b200 import _lib
+    H, d = 2, 64
+    q = torch.randn((300, H, d), device=DEV).to(torch.bfloat16)
+    k, v = torch.randn_like(q), torch.randn_like(q)
+    o, obuf = guarded_empty(q.shape, q.dtype, DEV)
+    lse, lbuf = guarded_empty((H, 300), torch.float32, DEV)
+    bad_total = torch.tensor([0, 100, 400], dtype=torch.int32, device=DEV)   # 400 > 300 rows
+    fa.varlen_fwd(q, k, v, bad_total, bad_total, 300, 300, None, True, out=o, lse=lse)
+    assert fa.device_status() == _lib.FA_ERR_INVALID_ARG
+    assert guard_intact(obuf, o.numel()) and guard_intact(lbuf, lse.numel())
+    short = torch.tensor([0, 100, 300], dtype=torch.int32, device=DEV)       # 200 > max 128
+    fa.varlen_fwd(q, k, v, short, short, 128, 128, None, True, out=o, lse=lse)
+    assert fa.device_status() == _lib.FA_ERR_INVALID_ARG
+    o2, lse2 = fa.varlen_fwd(q, k, v, short, short, 200, 200, None, True)
+    do = torch.randn_like(q)
+    fa.varlen_bwd(q, k, v, o2, lse2, do, bad_total, bad_total, 300, 300, None, True)
+    assert fa.device_status() == _lib.FA_ERR_INVALID_ARG
+    fa.varlen_bwd(q, k, v, o2, lse2, do, short, short, 200, 200, None, True)
+    assert fa.device_status() == 0  # well-formed again
