@@ -152,6 +152,30 @@ class ClockSampler:
 # ------------------------------------------------------------------ oracle timing
 _HEAD_CACHE = {}
 
+
+def oracle_threads() -> int:
+    """Threads the oracle runs on: its matrix products go to numpy's BLAS pool (the rest of
+    its numpy steps are single-threaded), so the BLAS pool size; the logical CPU count when
+    no BLAS pool is visible."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except ImportError:
+        pass
+    return os.cpu_count() or 1
+
+
+def host_cpus() -> dict:
+    """Physical and logical core counts of the host the oracle is timed on."""
+    try:
+        import psutil
+        phys = psutil.cpu_count(logical=False)
+    except ImportError:
+        phys = None
+    return {"physical_cores": phys, "logical_cores": os.cpu_count()}
+
 def oracle_sample_seconds(w, rows: int, head=(0, 0)):
     """Run the fp64 oracle forward + backward for the last `rows` query rows of one head
     against all keys; return (seconds, metric FLOPs of that share, threads)."""
@@ -180,8 +204,7 @@ def oracle_sample_seconds(w, rows: int, head=(0, 0)):
     win = w.window if w.window is not None else ((-1, 0) if w.causal else (-1, -1))
     keys = wl.window_pairs(rows, N, win)
     flops = 3.5 * 4.0 * float(keys) * w.d
-    threads = os.cpu_count()
-    return dt, flops, threads
+    return dt, flops, oracle_threads()
 
 
 def run_reference(args, w):
@@ -197,7 +220,7 @@ def run_reference(args, w):
     for _ in range(args.warmup):
         oracle_sample_seconds(w, rows)
     total_t, total_f = 0.0, 0.0
-    threads = os.cpu_count()
+    threads = oracle_threads()
     for _ in range(args.steps):
         dt, fl, threads = oracle_sample_seconds(w, rows)
         total_t += dt
@@ -210,25 +233,54 @@ def run_reference(args, w):
             "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": dict(w.describe(), parallelism=f"dp{world}"),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, **host_cpus(),
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
-# ------------------------------------------------------------------ N = 1K..4K sweep
-SWEEP = ["a100table_N1024", "a100table_N2048", "a100table_N4096", "llama_causal"]
+# ------------------------------------------------------------------ N = 128..4K sweep
+SWEEP = ["tiny_causal", "tiny_noncausal", "a100table_N1024", "a100table_N2048",
+         "a100table_N4096", "llama_causal", "varlen3", "varlen64"]
 
 
-def sweep_small_n(lib, dev, reps: int = 10):
-    """Forward and forward+backward of the pages' smaller shapes (the A100-table B8 H16 d64
-    at N = 1K, 2K, 4K, the Llama-style B4 H32 d128 N=4K and the 64-sequence packed varlen
-    batch), one GPU.  Their inputs fit in
-    L2, so L2 is flushed (a 256 MB write) before every timed launch; each launch is timed
-    alone with CUDA events.  Reports TFLOPS and the forward's algorithmic HBM GB/s
-    (Q, K, V read once, O and LSE written once)."""
+def _timed(fn, stream, dev, flush, reps):
+    """CUDA-event times (ms) of `reps` launches of fn, each alone: L2-flushed (a 256 MB
+    write before each) and L2-warm (back to back after one warm launch)."""
+    import torch
+    for _ in range(3):
+        fn()
+    cold, warm = [], []
+    for _ in range(reps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        cold.append(a.elapsed_time(b))
+    fn()
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        warm.append(a.elapsed_time(b))
+    return {"median": statistics.median(cold), "min": min(cold), "max": max(cold),
+            "warm_median": statistics.median(warm)}
+
+
+def sweep_small_n(lib, dev):
+    """Forward and backward of the pages' other shapes on one GPU: the tiny B1 H2 N128 d64
+    case, the A100-table B8 H16 d64 at N = 1K, 2K, 4K, the Llama-style B4 H32 d128 N=4K,
+    and the packed varlen batches (3 sequences / 896 tokens, 64 sequences).  Each launch is
+    timed alone with CUDA events, L2-flushed (inputs of these sizes fit in L2) and L2-warm;
+    200 launches for the microsecond-scale cases, 20 otherwise.  TFLOPS and the forward's
+    algorithmic HBM GB/s (Q, K, V read once, O and LSE written once) use the flushed
+    median."""
     import torch
     from exact_tiled_attention_33_b200 import _lib
     from exact_tiled_attention_33_b200 import attention as fa
@@ -241,70 +293,56 @@ def sweep_small_n(lib, dev, reps: int = 10):
         w = wl.get(name)
         t = wl.generate(w)
         q, k, v, do = (t[x].to(dev) for x in ("q", "k", "v", "do"))
-        B, N, H, d = q.shape
         dt = _lib.FA_BF16 if w.dtype == "bf16" else _lib.FA_FP16
         o = torch.empty_like(q)
-        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        ws = fa.bwd_workspace(B, N, H, d, dev)
+        if w.varlen:
+            cu = t["cu_seqlens"].to(dev)
+            L = max(w.seqlens)
+            lse = torch.empty((w.H, w.total), dtype=torch.float32, device=dev)
+            ws = fa.varlen_bwd_workspace(w.total, w.H, w.d, dev)
 
-        def fwd():
-            _lib.check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                  lse.data_ptr(), B, N, H, d, w.softmax_scale, int(w.causal), dt,
-                                  sh), "fa_fwd")
+            def fwd():
+                fa.varlen_fwd(q, k, v, cu, cu, L, L, w.softmax_scale, w.causal, out=o, lse=lse)
 
-        def bwd():
-            _lib.check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                  do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                                  dv.data_ptr(), B, N, H, d, w.softmax_scale, int(w.causal),
-                                  ws.data_ptr(), ws.numel(), dt, sh), "fa_bwd")
+            def bwd():
+                fa.varlen_bwd(q, k, v, o, lse, do, cu, cu, L, L, w.softmax_scale, w.causal,
+                              workspace=ws, dq=dq, dk=dk, dv=dv)
+            shape = {"num_seqs": len(w.seqlens), "total_tokens": w.total}
+            rows = w.total
+        else:
+            B, N, H, d = q.shape
+            lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+            ws = fa.bwd_workspace(B, N, H, d, dev)
 
-        def timed(fn):
-            ms = []
-            for _ in range(3):
-                fn()
-            for _ in range(reps):
-                flush.fill_(1)
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                fn()
-                b.record(stream)
-                torch.cuda.synchronize(dev)
-                ms.append(a.elapsed_time(b))
-            return statistics.median(ms)
+            def fwd():
+                _lib.check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      lse.data_ptr(), B, N, H, d, w.softmax_scale,
+                                      int(w.causal), dt, sh), "fa_fwd")
 
-        f_ms, b_ms = timed(fwd), timed(bwd)
+            def bwd():
+                _lib.check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+                                      dk.data_ptr(), dv.data_ptr(), B, N, H, d,
+                                      w.softmax_scale, int(w.causal), ws.data_ptr(),
+                                      ws.numel(), dt, sh), "fa_bwd")
+            shape = {"B": B, "N": N}
+            rows = B * N
+        small = w.fwd_flops() < 1e10
+        reps = 200 if small else 20
+        tf, tb = _timed(fwd, stream, dev, flush, reps), _timed(bwd, stream, dev, flush, reps)
         assert lib.fa_get_device_status(sh) == 0
         f = w.fwd_flops()
         e = q.numel() * q.element_size()
-        fwd_bytes = 4 * e + 4 * B * H * N
-        out.append({"workload": name, "B": B, "N": N, "H": H, "d": d, "causal": w.causal,
-                    "fwd_ms": f_ms, "bwd_ms": b_ms, "fwd_tflops": f / f_ms / 1e9,
-                    "fwd_bwd_tflops": 3.5 * f / (f_ms + b_ms) / 1e9,
-                    "fwd_hbm_gbs": fwd_bytes / f_ms / 1e6})
-    # the packed variable-length batch: 64 sequences of 64..4096 tokens, H32 d128, causal
-    w = wl.get("varlen64")
-    t = wl.generate(w)
-    q, k, v, do = (t[x].to(dev) for x in ("q", "k", "v", "do"))
-    cu = t["cu_seqlens"].to(dev)
-    L = max(w.seqlens)
-    o, lse = fa.varlen_fwd(q, k, v, cu, cu, L, L, w.softmax_scale, True)
-    wsv = fa.varlen_bwd_workspace(q.shape[0], w.H, w.d, dev)
-
-    def vfwd():
-        fa.varlen_fwd(q, k, v, cu, cu, L, L, w.softmax_scale, True, out=o, lse=lse)
-
-    def vbwd():
-        fa.varlen_bwd(q, k, v, o, lse, do, cu, cu, L, L, w.softmax_scale, True, workspace=wsv)
-
-    f_ms, b_ms = timed(vfwd), timed(vbwd)
-    assert lib.fa_get_device_status(sh) == 0
-    f = w.fwd_flops()
-    e = q.numel() * q.element_size()
-    out.append({"workload": "varlen64", "num_seqs": len(w.seqlens), "total_tokens": w.total,
-                "H": w.H, "d": w.d, "causal": True, "fwd_ms": f_ms, "bwd_ms": b_ms,
-                "fwd_tflops": f / f_ms / 1e9, "fwd_bwd_tflops": 3.5 * f / (f_ms + b_ms) / 1e9,
-                "fwd_hbm_gbs": (4 * e + 4 * w.H * w.total) / f_ms / 1e6})
+        fwd_bytes = 4 * e + 4 * w.H * rows
+        out.append(dict({"workload": name, "H": w.H, "d": w.d, "causal": w.causal}, **shape,
+                        fwd_us=1e3 * tf["median"], fwd_us_min=1e3 * tf["min"],
+                        fwd_us_max=1e3 * tf["max"], fwd_us_l2_warm=1e3 * tf["warm_median"],
+                        bwd_us=1e3 * tb["median"], bwd_us_min=1e3 * tb["min"],
+                        bwd_us_max=1e3 * tb["max"], bwd_us_l2_warm=1e3 * tb["warm_median"],
+                        fwd_tflops=f / tf["median"] / 1e9,
+                        fwd_bwd_tflops=3.5 * f / (tf["median"] + tb["median"]) / 1e9,
+                        fwd_hbm_gbs=fwd_bytes / tf["median"] / 1e6, reps=reps))
     del flush
     return out
 
@@ -510,10 +548,13 @@ def run_fattn(args, w):
         while dt < 5.0 and rows < wr.N:
             rows = min(wr.N, rows * 2)
             dt, fl, threads = oracle_sample_seconds(wr, rows)
-        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, **host_cpus(),
+               "kind": "oracle",
                "sample": f"last {rows} query rows of head (b=0,h=0) against all {wr.N} keys"
                          f"{'' if wr.window is None else ' (window ' + str(list(wr.window)) + ')'}"
-                         f", fp64 oracle fwd+bwd ({dt:.1f} s)"}
+                         f", fp64 oracle fwd+bwd ({dt:.1f} s)",
+               # one whole step (every head of every batch row) at the sample's rate
+               "full_step_seconds_extrapolated": f_step / (fl / dt)}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -530,7 +571,7 @@ def run_fattn(args, w):
                 "ms_fwd": fwd_avg, "ms_bwd": bwd_avg,
                 "gpu_launches": 4 * args.steps,
                 "roofline": roofline, "roofline_fwd": fwd_roof,
-                "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "sweep_n1k_4k": sweep}
+                "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "sweep_small_n": sweep}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -553,7 +594,7 @@ def run_decode_reference(args, w):
     for _ in range(args.warmup):
         oracle_decode_seconds(w, g, n, reps)
     tot_t = tot_b = 0.0
-    threads = os.cpu_count()
+    threads = oracle_threads()
     for _ in range(args.steps):
         dt, by, threads = oracle_decode_seconds(w, g, n, reps)
         tot_t += dt
@@ -568,6 +609,7 @@ def run_decode_reference(args, w):
                       "dtype": "f64", "data": "synthetic",
                       "config": dict(w.describe(), parallelism=f"dp{world}"),
                       "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads,
+                                       **host_cpus(),
                                        "kind": "oracle", "sample": sample},
                       "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
                               "d2h_bytes_per_step": 0}}), flush=True)
@@ -592,7 +634,7 @@ def oracle_fp8_seconds(w, host, rows: int, reps: int = 1):
                                      host["v_descale"], w.softmax_scale, w.causal, rows=r)
     dt = time.perf_counter() - t0
     win = (-1, 0) if w.causal else (-1, -1)
-    return dt, 4.0 * w.d * wl.window_pairs(rows, N, win) * reps, os.cpu_count()
+    return dt, 4.0 * w.d * wl.window_pairs(rows, N, win) * reps, oracle_threads()
 
 
 def run_fp8_reference(args, w):
@@ -609,7 +651,7 @@ def run_fp8_reference(args, w):
     for _ in range(args.warmup):
         oracle_fp8_seconds(w, host, rows)
     tot_t = tot_f = 0.0
-    threads = os.cpu_count()
+    threads = oracle_threads()
     for _ in range(args.steps):
         dt, fl, threads = oracle_fp8_seconds(w, host, rows)
         tot_t += dt
@@ -623,6 +665,7 @@ def run_fp8_reference(args, w):
                       "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                       "data": "synthetic", "config": dict(w.describe(), parallelism=f"dp{world}"),
                       "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads,
+                                       **host_cpus(),
                                        "kind": "oracle", "sample": sample},
                       "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                               "d2h_bytes_per_step": 0}}), flush=True)
@@ -739,7 +782,8 @@ def run_fp8(args, w):
         while dt < 5.0 and rows < N:
             rows = min(N, rows * 2)
             dt, fl, threads = oracle_fp8_seconds(wr, host, rows)
-        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, **host_cpus(),
+               "kind": "oracle",
                "sample": f"last {rows} query rows of head (b=0,h=0) against all {N} keys, "
                          f"fp64 oracle forward of the dequantised FP8 inputs ({dt:.1f} s)"}
     if rank == 0:
@@ -787,7 +831,7 @@ def oracle_decode_seconds(w, g, n_heads: int, reps: int = 1):
         for h in range(n_heads):
             oracle.attention_forward(q[:, h], kb[:, h], vb[:, h], w.softmax_scale, w.causal)
     dt = time.perf_counter() - t0
-    return dt, 2.0 * L * n_heads * w.d * 2 * reps, os.cpu_count()
+    return dt, 2.0 * L * n_heads * w.d * 2 * reps, oracle_threads()
 
 
 def run_decode(args, w):
@@ -909,7 +953,8 @@ def run_decode(args, w):
         while dt < 5.0:
             reps *= 2
             dt, by, threads = oracle_decode_seconds(wr, host, H, reps)
-        cpu = {"value": by / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+        cpu = {"value": by / dt / 1e9, "unit": "GB/s", "cores": threads, **host_cpus(),
+               "kind": "oracle",
                "sample": f"sequence 0 ({wr.cache_lens[0]} cached rows), all {H} heads, "
                          f"{reps} passes, fp64 oracle decode ({dt:.1f} s)"}
     if rank == 0:
@@ -939,7 +984,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true",
-                    help="skip the N = 1K..4K sweep of the default bench line")
+                    help="skip the small-shape sweep of the default bench line")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3) if args.impl == "fattn" else args.warmup
     from exact_tiled_attention_33_b200 import workloads as wl
