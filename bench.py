@@ -107,11 +107,44 @@ REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_powe
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clocks and throttle reasons sampled during the timed region: NVML (the library
+    nvidia-smi reads) polled every 20 ms from a thread, so even a region of a few hundred
+    milliseconds gets a dozen samples; nvidia-smi in a subprocess when NVML is missing."""
+
+    _BITS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+             "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+             "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+             "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
 
     def __init__(self, gpu_index: int):
+        self.rows = []          # (sm MHz, max sm MHz, [active reasons])
         self.proc = None
-        self.path = None
+        self.thread = None
+        self.source = None
+        try:
+            import threading
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(torch.cuda._get_nvml_device_index(gpu_index))
+            bits = {r: getattr(pynvml, n) for r, n in self._BITS.items()}
+            self.stop_flag = threading.Event()
+
+            def poll():
+                mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+                while True:
+                    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    why = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.rows.append((float(sm), float(mx),
+                                      [r for r, b in bits.items() if why & b]))
+                    if self.stop_flag.wait(0.02):
+                        return
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            self.source = "nvml, 20 ms"
+            return
+        except Exception:  # noqa: BLE001 - any NVML failure falls back to nvidia-smi
+            self.thread = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -119,34 +152,37 @@ class ClockSampler:
                  ",".join(f"clocks_event_reasons.{r}" for r in REASONS))
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200",
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "100",
                  "-i", str(gpu_index)], stdout=self.out, stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi, 100 ms"
         except (OSError, FileNotFoundError):
             self.proc = None
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.close()
+            for line in open(self.path):
+                r = [x.strip() for x in line.split(",")]
+                if len(r) == 4 + len(REASONS) and r[1].replace(".", "").isdigit():
+                    self.rows.append((float(r[1]), float(r[2]) if r[2].replace(".", "").isdigit()
+                                      else float("nan"),
+                                      [REASONS[i] for i in range(len(REASONS))
+                                       if r[4 + i].lower() == "active"]))
+            os.unlink(self.path)
+        if not self.rows:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.out.close()
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) == 4 + len(REASONS):
-                rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        active = sorted({REASONS[i] for r in rows for i in range(len(REASONS))
-                         if r[4 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": active, "samples": len(rows)}
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows),
+                "sm_max_mhz": max(r[1] for r in self.rows),
+                "reasons": sorted({x for r in self.rows for x in r[2]}),
+                "samples": len(self.rows), "source": self.source}
 
 
 # ------------------------------------------------------------------ oracle timing
@@ -248,7 +284,9 @@ SWEEP = ["tiny_causal", "tiny_noncausal", "a100table_N1024", "a100table_N2048",
 
 def _timed(fn, stream, dev, flush, reps):
     """CUDA-event times (ms) of `reps` launches of fn, each alone: L2-flushed (a 256 MB
-    write before each) and L2-warm (back to back after one warm launch)."""
+    write before each) and L2-warm (after a launch on the same data, with a ~100 us GPU
+    sleep in between that touches no memory).  The flush or the sleep keeps the GPU busy
+    while the host enqueues the launch, so the host's launch overhead is not timed."""
     import torch
     for _ in range(3):
         fn()
@@ -263,6 +301,7 @@ def _timed(fn, stream, dev, flush, reps):
         cold.append(a.elapsed_time(b))
     fn()
     for _ in range(reps):
+        torch.cuda._sleep(200_000)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()
