@@ -243,6 +243,24 @@ def oracle_sample_seconds(w, rows: int, head=(0, 0)):
     return dt, flops, oracle_threads()
 
 
+def oracle_full_seconds(name: str) -> dict:
+    """The fp64 oracle's forward + backward over every (batch, head) of a small workload,
+    timed directly (no sampling)."""
+    import oracle
+    from exact_tiled_attention_33_b200 import workloads as wl
+    w = wl.get(name)
+    t = wl.generate(w)
+    q, k, v, do = (wl.to_f64(t[x]) for x in ("q", "k", "v", "do"))
+    t0 = time.perf_counter()
+    for b in range(w.B):
+        for h in range(w.H):
+            a = (q[b, :, h], k[b, :, h], v[b, :, h])
+            oracle.attention_forward(*a, w.softmax_scale, w.causal)
+            oracle.attention_backward(*a, do[b, :, h], w.softmax_scale, w.causal)
+    dt = time.perf_counter() - t0
+    return {"workload": name, "seconds": dt, "gflops": 3.5 * w.fwd_flops() / dt / 1e9}
+
+
 def run_reference(args, w):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -288,7 +306,7 @@ def _timed(fn, stream, dev, flush, reps):
     sleep in between that touches no memory).  The flush or the sleep keeps the GPU busy
     while the host enqueues the launch, so the host's launch overhead is not timed."""
     import torch
-    for _ in range(3):
+    for _ in range(5):
         fn()
     cold, warm = [], []
     for _ in range(reps):
@@ -593,7 +611,8 @@ def run_fattn(args, w):
                          f"{'' if wr.window is None else ' (window ' + str(list(wr.window)) + ')'}"
                          f", fp64 oracle fwd+bwd ({dt:.1f} s)",
                # one whole step (every head of every batch row) at the sample's rate
-               "full_step_seconds_extrapolated": f_step / (fl / dt)}
+               "full_step_seconds_extrapolated": f_step / (fl / dt),
+               "full_runs": [oracle_full_seconds(n) for n in ("tiny_causal", "a100table_N1024")]}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
