@@ -499,6 +499,25 @@ def run_fattn(args, w):
     fwd_avg = statistics.mean(fwd_ms)
     bwd_avg = statistics.mean(bwd_ms)
 
+    # ---- the forward alone, as the pages' forward benchmarks time it: `steps` forward
+    # launches back to back on the same inputs (each tensor larger than the 126 MB L2),
+    # CUDA events around them on the launching stream, max over ranks
+    fsampler = ClockSampler(local) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    f_start = torch.cuda.Event(enable_timing=True)
+    f_end = torch.cuda.Event(enable_timing=True)
+    f_start.record(stream)
+    for _ in range(args.steps):
+        launch_fwd()
+    f_end.record(stream)
+    torch.cuda.synchronize(dev)
+    fclocks = fsampler.stop() if fsampler is not None else None
+    assert lib.fa_get_device_status(sh) == 0, "device status after the forward-only loop"
+    fo_s = max_over_ranks(f_start.elapsed_time(f_end) / 1e3, world)
+    fwd_only_tflops = throughput_tflops(f_fwd, args.steps, world, fo_s)
+
     # ---- end to end through the C ABI with pinned host buffers.  Every step copies its
     # inputs q, k, v, dO host -> device, runs fwd + bwd and copies O, LSE, dQ, dK, dV back.
     # Two device buffer sets and three streams pipeline the steps: the copies of one step
@@ -592,6 +611,10 @@ def run_fattn(args, w):
                 "frac_of_burst_peak": fwd_ach / peak_burst,
                 "traffic": read_traffic("fa_fwd_kernel", wr.name, fwd_sha),
                 "flops_per_launch": f_fwd}
+    fwd_only = {"ms": 1e3 * fo_s / args.steps, "tflops": fwd_only_tflops,
+                "frac_of_burst_peak": fwd_only_tflops / world / peak_burst,
+                "frac_of_sustained_peak": fwd_only_tflops / world / peak_sust,
+                "clocks": fclocks}
 
     sweep = None
     if rank == 0 and world == 1 and not args.no_sweep:
@@ -628,7 +651,7 @@ def run_fattn(args, w):
                                      "peak_tflops": peak_burst, "peak_source": peak_src},
                 "ms_fwd": fwd_avg, "ms_bwd": bwd_avg,
                 "gpu_launches": 4 * args.steps,
-                "roofline": roofline, "roofline_fwd": fwd_roof,
+                "roofline": roofline, "roofline_fwd": fwd_roof, "fwd_only": fwd_only,
                 "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "sweep_small_n": sweep}
         print(json.dumps(line), flush=True)
     if world > 1:
