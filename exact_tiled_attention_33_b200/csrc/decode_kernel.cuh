@@ -199,6 +199,9 @@ __global__ void __launch_bounds__(DecCfg<D, NQ>::THREADS, 1)
   const float c = p.scale_log2;
   // independent partial dot products per row (breaks the FMA dependency chain)
   constexpr int NACC = NQ == 1 ? 8 : (NQ <= 4 ? 4 : 2);
+  // up to four query rows: the score and P·V multiply-adds issue two lanes per instruction
+  // (fma.rn.f32x2); sixteen rows keep the scalar form, which fits the registers
+  constexpr bool PAIRED = NQ > 1 && NQ <= 4;
   // this lane's P·V columns: chunk, 16-byte segment and byte offset inside it
   const int col0 = lane * CPL;
   const int vchunk = col0 >> 6, vseg = (col0 & 63) >> 3, vbyte = (col0 & 7) * 2;
@@ -240,9 +243,23 @@ __global__ void __launch_bounds__(DecCfg<D, NQ>::THREADS, 1)
                 const float4 qb =
                     *reinterpret_cast<const float4*>(qs + r * D + cc * 64 + seg * 8 + 4);
                 const float qf[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+                if constexpr (!PAIRED) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                  acc[r][e % NACC] = fmaf(qf[e], kf[e], acc[r][e % NACC]);
+                  for (int e = 0; e < 8; ++e)
+                    acc[r][e % NACC] = fmaf(qf[e], kf[e], acc[r][e % NACC]);
+                } else {
+                  // two lanes per instruction (fma.rn.f32x2): element e still goes to
+                  // partial sum e % NACC, so the sums are those of the scalar form
+#pragma unroll
+                  for (int e = 0; e < 8; e += 2) {
+                    const int a = e % NACC;
+                    const float2 t = f2_unpack(f2_fma(f2_pack(qf[e], qf[e + 1]),
+                                                      f2_pack(kf[e], kf[e + 1]),
+                                                      f2_pack(acc[r][a], acc[r][a + 1])));
+                    acc[r][a] = t.x;
+                    acc[r][a + 1] = t.y;
+                  }
+                }
               }
             }
           }
@@ -293,8 +310,18 @@ __global__ void __launch_bounds__(DecCfg<D, NQ>::THREADS, 1)
 #pragma unroll
     for (int r = 0; r < NQ; ++r) {
       if (r < Nq) {
+        if constexpr (!PAIRED) {
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) o[r][e] *= alpha[r];
+          for (int e = 0; e < CPL; ++e) o[r][e] *= alpha[r];
+        } else {
+#pragma unroll
+          for (int e = 0; e < CPL; e += 2) {
+            const float2 t = f2_unpack(f2_mul(f2_pack(o[r][e], o[r][e + 1]),
+                                              f2_pack(alpha[r], alpha[r])));
+            o[r][e] = t.x;
+            o[r][e + 1] = t.y;
+          }
+        }
       }
     }
     const uint8_t* vcol = Vs + vchunk * C::CHUNK + vbyte;
@@ -315,8 +342,18 @@ __global__ void __launch_bounds__(DecCfg<D, NQ>::THREADS, 1)
       for (int r = 0; r < NQ; ++r) {
         if (r < Nq) {
           const float pr = Sb[r * BN + jj];
+          if constexpr (!PAIRED) {
 #pragma unroll
-          for (int e = 0; e < CPL; ++e) o[r][e] = fmaf(pr, vf[e], o[r][e]);
+            for (int e = 0; e < CPL; ++e) o[r][e] = fmaf(pr, vf[e], o[r][e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < CPL; e += 2) {
+              const float2 t = f2_unpack(f2_fma(f2_pack(pr, pr), f2_pack(vf[e], vf[e + 1]),
+                                                f2_pack(o[r][e], o[r][e + 1])));
+              o[r][e] = t.x;
+              o[r][e + 1] = t.y;
+            }
+          }
         }
       }
     };
