@@ -1,0 +1,97 @@
+"""CPU test of the kernels' tile scheduling: `key_tile_range` (which K/V tiles a query tile
+walks: forward and dQ pass) and `query_tile_range` (which query tiles a key tile walks: dK/dV
+pass), compiled for the host from the library's own header.  For every small shape, window
+and tile size, the tiles returned must be exactly the tiles that hold at least one allowed
+(query, key) pair of the oracle's mask: none missed (that would drop keys) and none extra
+(wasted work).  Tile sizes below 128 exercise many more tile boundaries than the kernels'
+128 while running the same arithmetic."""
+
+import ctypes
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "exact_tiled_attention_33_b200", "csrc")
+WINDOWS = [(-1, -1), (-1, 0), (0, 0), (0, -1), (1, 0), (2, 3), (5, 0), (0, 4), (-1, 2), (3, -1)]
+
+
+def _nvcc():
+    for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    return None
+
+
+@pytest.fixture(scope="module")
+def shim(tmp_path_factory):
+    nvcc = _nvcc()
+    if nvcc is None:
+        pytest.skip("nvcc not found")
+    out = tmp_path_factory.mktemp("shim") / "libtile_range_shim.so"
+    cmd = [nvcc, "-std=c++17", "-shared", "-Xcompiler", "-fPIC", "-I", CSRC,
+           "-gencode", "arch=compute_100a,code=sm_100a",
+           os.path.join(ROOT, "tests", "c", "tile_range_shim.cu"), "-o", str(out)]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    lib = ctypes.CDLL(str(out))
+    for f in (lib.shim_key_tile_range, lib.shim_query_tile_range):
+        f.argtypes = [ctypes.c_int] * 7 + [ctypes.POINTER(ctypes.c_int)] * 2
+        f.restype = None
+    return lib
+
+
+def _call(f, a0, a1, L, diag, wl, wr, T):
+    b, c = ctypes.c_int(-7), ctypes.c_int(-7)
+    f(a0, a1, L, diag, wl, wr, T, ctypes.byref(b), ctypes.byref(c))
+    assert c.value >= 0
+    return set(range(b.value, b.value + c.value))
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 128])
+def test_tile_ranges_match_the_mask(shim, T):
+    checked = 0
+    for Lq in range(1, 10):
+        for Lk in range(1, 10):
+            diag = Lk - Lq
+            for win in WINDOWS:
+                mask = oracle.allowed_mask(np.arange(Lq), Lq, Lk, False, window=win)
+                for q0 in range(0, Lq, T):      # query tiles, as the forward and dQ pass cut them
+                    q1 = min(q0 + T, Lq) - 1
+                    want = {int(j) // T for j in np.nonzero(mask[q0:q1 + 1].any(axis=0))[0]}
+                    got = _call(shim.shim_key_tile_range, q0, q1, Lk, diag, *win, T)
+                    assert got == want, (Lq, Lk, win, T, q0, got, want)
+                    checked += 1
+                for k0 in range(0, Lk, T):      # key tiles, as the dK/dV pass cuts them
+                    k1 = min(k0 + T, Lk) - 1
+                    want = {int(i) // T for i in np.nonzero(mask[:, k0:k1 + 1].any(axis=1))[0]}
+                    got = _call(shim.shim_query_tile_range, k0, k1, Lq, diag, *win, T)
+                    assert got == want, (Lq, Lk, win, T, k0, got, want)
+                    checked += 1
+    assert checked > 0
+
+
+def test_tile_ranges_at_kernel_sizes(shim):
+    # the kernels' 128-row tiles on the pages' shapes (16K causal, a 4096-key window, a
+    # decode-like 4 rows over 8192 keys, Lq != Lk with a two-sided window): sampled tiles of
+    # both kinds against the oracle's mask of those rows / keys
+    T = 128
+    for Lq, Lk, win in ((16384, 16384, (-1, 0)), (16384, 16384, (4096, 0)), (4, 8192, (-1, 0)),
+                        (1000, 3000, (100, 100))):
+        diag = Lk - Lq
+        nq, nk = (Lq + T - 1) // T, (Lk + T - 1) // T
+        for t in sorted({0, 1, nq // 3, nq // 2, nq - 2, nq - 1} & set(range(nq))):
+            q0, q1 = t * T, min(t * T + T, Lq) - 1
+            m = oracle.allowed_mask(np.arange(q0, q1 + 1), Lq, Lk, False, window=win)
+            want = {int(j) // T for j in np.nonzero(m.any(axis=0))[0]}
+            assert _call(shim.shim_key_tile_range, q0, q1, Lk, diag, *win, T) == want
+        full = oracle.allowed_mask(np.arange(Lq), Lq, Lk, False, window=win)
+        for t in sorted({0, 1, nk // 3, nk // 2, nk - 2, nk - 1} & set(range(nk))):
+            k0, k1 = t * T, min(t * T + T, Lk) - 1
+            want = {int(i) // T for i in np.nonzero(full[:, k0:k1 + 1].any(axis=1))[0]}
+            assert _call(shim.shim_query_tile_range, k0, k1, Lq, diag, *win, T) == want
