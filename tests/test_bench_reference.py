@@ -49,6 +49,19 @@ def test_reference_arm_windowed():
     _check_line(d, "long_local_sym512")
 
 
+def test_reference_arm_decode():
+    d = _run(["--impl", "reference", "--workload", "decode_q4_l8k", "--steps", "1",
+              "--warmup", "0"])
+    _check_line(d, "decode_q4_l8k")
+    assert d["unit"] == "GB/s"
+
+
+def test_reference_arm_fp8():
+    d = _run(["--impl", "reference", "--workload", "fp8_long_causal", "--steps", "1",
+              "--warmup", "0"])
+    _check_line(d, "fp8_long_causal")
+
+
 def test_host_helpers():
     assert bench.oracle_threads() >= 1
     h = bench.host_cpus()
