@@ -206,8 +206,10 @@ def generate(w: Workload, with_grad_out: bool = True):
         out["cu_seqlens"] = torch.from_numpy(w.cu_seqlens())
     if w.fp8:
         # per-tensor scaling to the E4M3 range: descale = amax / 448, codes = x / descale
-        # rounded to nearest (PyTorch's float8_e4m3fn cast); the 16-bit q, k, v above are
-        # replaced by the exactly representable dequantised values
+        # rounded to nearest (PyTorch's float8_e4m3fn cast).  The 16-bit q, k, v above are
+        # replaced by the dequantised values rounded to 16 bits, a view for callers that
+        # want one; the FP8 kernels take the codes and descales, and the parity tests give
+        # the oracle the codes and descales too (exact in fp64)
         for name, x in (("q", q), ("k", k), ("v", v)):
             descale = float(x.abs().max()) / 448.0
             x8 = (x / descale).to(torch.float8_e4m3fn)
