@@ -234,9 +234,16 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d,
                    float scale, int causal, int dtype, void* stream);
 
-/* Synchronises `stream`, returns FA_ERR_TIMEOUT if any kernel of this library on the
- * current device recorded a timed-out wait since the last call (FA_OK otherwise), and
- * clears the status word.  FA_ERR_CUDA if the synchronisation itself failed. */
+/* Synchronises `stream`, reads and clears the library's status word of the current
+ * device, and reports what its kernels recorded since the last call, in this order:
+ *   FA_ERR_TIMEOUT      a kernel's bounded wait ran out (its outputs are undefined);
+ *   FA_ERR_INVALID_ARG  a varlen call met a cu_seqlens segment outside [0, total] or
+ *                       longer than max_seqlen (that segment was skipped), or a decode
+ *                       call met a cache length above its bound or a page id out of range;
+ *   FA_ERR_UNSUPPORTED  the dynamic shared memory base could not be 1024-byte aligned;
+ *   FA_OK               nothing recorded.
+ * FA_ERR_CUDA if the synchronisation or the status read itself failed; fa_last_error then
+ * names the step. */
 int fa_get_device_status(void* stream);
 
 /* Static description of a status code. */
