@@ -56,7 +56,8 @@ extern "C" {
 
 typedef enum {
   FA_OK = 0,
-  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad cu_seqlens count,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad cu_seqlens count;
+                             from fa_get_device_status: a malformed cu_seqlens segment or
                              decode cache bounds exceeded on the device */
   FA_ERR_UNSUPPORTED = 2, /* head_dim other than 64/128, unknown dtype, size limits */
   FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (see fa_last_error) */
