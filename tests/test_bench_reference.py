@@ -73,3 +73,24 @@ def test_clock_sampler_without_gpu_returns_nothing_or_a_summary():
     s = bench.ClockSampler(0)
     out = s.stop()
     assert out is None or {"sm_mhz", "sm_max_mhz", "reasons", "samples"} <= set(out)
+
+
+def test_reference_arm_under_two_ranks_prints_once():
+    # launched like the multi-GPU bench (RANK / WORLD_SIZE in the environment): rank 0 runs
+    # the oracle and prints the one JSON line, rank 1 exits 0 without work or output
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    outs = []
+    for rank in (0, 1):
+        env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank),
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT="29531")
+        r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload",
+                            "tiny_causal", "--gpus", "2", "--steps", "1", "--warmup", "0"],
+                           cwd=root, env=env, capture_output=True, text=True, timeout=300)
+        assert r.returncode == 0, r.stderr
+        outs.append([x for x in r.stdout.splitlines() if x.startswith("{")])
+    assert len(outs[0]) == 1 and outs[1] == []
+    d = json.loads(outs[0][0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
