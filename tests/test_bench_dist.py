@@ -37,7 +37,7 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_max_and_throughput():
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()   # no fork of this (multi-threaded) process
     out = mgr.dict()
     mp.start_processes(_worker, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
     for rank in range(2):
