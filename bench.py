@@ -41,6 +41,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
 BWD_SOURCES = ["exact_tiled_attention_33_b200/csrc/bwd_kernel.cuh",
                "exact_tiled_attention_33_b200/csrc/sm100.cuh",
                "exact_tiled_attention_33_b200/csrc/fattn_internal.h"]
+BWD_KERNEL_DESC = "fa_bwd (D preprocess + dK/dV kernel + dQ kernel, timed as one call)"
 FWD_SOURCES = ["exact_tiled_attention_33_b200/csrc/fwd_kernel.cuh",
                "exact_tiled_attention_33_b200/csrc/sm100.cuh",
                "exact_tiled_attention_33_b200/csrc/fattn_internal.h"]
@@ -599,16 +600,22 @@ def run_fattn(args, w):
     fwd_sha = sources_sha(FWD_SOURCES)
     bwd_ach = 2.5 * f_fwd / (bwd_avg / 1e3) / 1e12
     fwd_ach = f_fwd / (fwd_avg / 1e3) / 1e12
+    # The timed region lasts well under the seconds a sustained (power-capped) measurement
+    # needs, so the fractions are taken against the burst peak; the fraction of the
+    # sustained figure is kept beside it, labelled.
+    timed_s = total_ms / 1e3
     roofline = {
-        "kernel": "fa_bwd (D preprocess + dK/dV kernel + dQ kernel, timed as one call)",
-        "bound": "tensor", "achieved": bwd_ach, "peak": peak_sust, "unit": "TFLOP/s",
-        "frac": bwd_ach / peak_sust,
-        "peak_source": f"bf16_tflops_sustained ({peak_src})",
+        "kernel": BWD_KERNEL_DESC,
+        "bound": "tensor", "achieved": bwd_ach, "peak": peak_burst, "unit": "TFLOP/s",
+        "frac": bwd_ach / peak_burst,
+        "peak_source": f"bf16_tflops burst ({peak_src}); timed region {timed_s:.2f} s",
+        "frac_of_sustained_peak": bwd_ach / peak_sust,
         "traffic": read_traffic("fa_bwd", wr.name, bwd_sha),
         "flops_per_launch": 2.5 * f_fwd}
     fwd_roof = {"kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": fwd_ach,
-                "peak": peak_sust, "unit": "TFLOP/s", "frac": fwd_ach / peak_sust,
-                "frac_of_burst_peak": fwd_ach / peak_burst,
+                "peak": peak_burst, "unit": "TFLOP/s", "frac": fwd_ach / peak_burst,
+                "peak_source": f"bf16_tflops burst ({peak_src})",
+                "frac_of_sustained_peak": fwd_ach / peak_sust,
                 "traffic": read_traffic("fa_fwd_kernel", wr.name, fwd_sha),
                 "flops_per_launch": f_fwd}
     fwd_only = {"ms": 1e3 * fo_s / args.steps, "tflops": fwd_only_tflops,

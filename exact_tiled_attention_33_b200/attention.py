@@ -64,6 +64,24 @@ def fwd(q, k, v, softmax_scale=None, causal=False, out=None, lse=None):
     return o, lse_t
 
 
+def fwd_f32out(q, k, v, softmax_scale=None, causal=False):
+    """Test hook: fa_fwd with O returned in fp32 before rounding (fa_selftest_fwd_f32).
+    Returns (o [B,N,H,d] fp32, lse [B,H,N] fp32)."""
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must all be [B, N, H, d] with equal shapes")
+    dtype = _check(q, k, v)
+    B, N, H, d = q.shape
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    o = torch.empty(q.shape, device=q.device, dtype=torch.float32)
+    lse_t = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_selftest_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, N, H,
+                                     d, scale, int(bool(causal)), dtype, _stream(q))
+    _lib.check(st, "fa_selftest_fwd_f32")
+    return o, lse_t
+
+
 def varlen_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
                softmax_scale=None, causal=False, out=None, lse=None):
     """Varlen forward. q: [total_q, H, d]; k, v: [total_k, H, d]; cu_seqlens int32 on device.

@@ -95,16 +95,38 @@ int make_map(CUtensorMap* map, const void* base, int d, int H, long long rows, l
   return FA_OK;
 }
 
-uint32_t* status_ptr() {
-  static uint32_t* ptrs[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return nullptr;
-  if (ptrs[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<uint32_t*>(p);
+// Device address of a module variable on the current device, looked up once per device
+// (std::call_once, so concurrent first calls from several host threads are safe).  The
+// host-side symbol is only a stand-in and must never be handed to a kernel.
+template <typename T>
+struct PerDeviceSymbol {
+  static constexpr int kMaxDevices = 64;
+  std::once_flag once[kMaxDevices];
+  T* ptr[kMaxDevices] = {};
+  cudaError_t err[kMaxDevices] = {};
+  // Returns the address (nullptr on failure, with the lookup's error in *e).
+  template <typename Sym>
+  T* get(const Sym& sym, int dev, cudaError_t* e) {
+    if (dev < 0 || dev >= kMaxDevices) {
+      *e = cudaErrorInvalidDevice;
+      return nullptr;
+    }
+    std::call_once(once[dev], [&] {
+      void* p = nullptr;
+      err[dev] = cudaGetSymbolAddress(&p, sym);
+      if (err[dev] == cudaSuccess) ptr[dev] = static_cast<T*>(p);
+    });
+    *e = err[dev];
+    return ptr[dev];
   }
-  return ptrs[dev];
+};
+
+uint32_t* status_ptr() {
+  static PerDeviceSymbol<uint32_t> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  cudaError_t e = cudaSuccess;
+  return cache.get(g_status_word, dev, &e);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -566,20 +588,17 @@ constexpr size_t kNoAllocScratchFloats = size_t(1) << 22;  // 16 MiB: B*H*N <= 4
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
 // Device address of the scratch array on the current device, looked up once per device
-// (the host-side symbol is only a stand-in and must never be handed to a kernel).
+// with that device current (the host-side symbol is only a stand-in and must never be
+// handed to a kernel).
 static int noalloc_scratch(float** out) {
-  static float* ptrs[64] = {};
+  static PerDeviceSymbol<float> cache;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev >= 64) return fail(FA_ERR_UNSUPPORTED, "device index >= 64");
-  if (ptrs[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
-    ptrs[dev] = static_cast<float*>(p);
-  }
-  *out = ptrs[dev];
+  if (dev >= PerDeviceSymbol<float>::kMaxDevices) return fail(FA_ERR_UNSUPPORTED, "device index >= 64");
+  float* p = cache.get(g_noalloc_scratch, dev, &e);
+  if (p == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+  *out = p;
   return FA_OK;
 }
 
@@ -782,6 +801,38 @@ int fa_selftest_exp2(const float* x, float* y, int n, void* stream) {
   selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, (cudaStream_t)stream>>>(x, y, n);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : cuda_fail(e, "selftest_exp2 launch");
+}
+
+int fa_selftest_fwd_f32(const void* q, const void* k, const void* v, float* o, float* lse, int B,
+                        int N, int H, int d, float scale, int causal, int dtype, void* stream) {
+  g_last_error.clear();
+  if (int e = check_common(H, d, dtype, scale)) return e;
+  if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
+  if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
+  if (B == 0 || N == 0 || H == 0) return FA_OK;
+  if (int e = check_grid(B, H, N)) return e;
+  if (int e = check_ptrs({q, k, v, o, lse})) return e;
+  CUtensorMap mq, mk, mv;
+  if (int e = make_map(&mq, q, d, H, N, B, 128)) return e;
+  if (int e = make_map(&mk, k, d, H, N, B, 128)) return e;
+  if (int e = make_map(&mv, v, d, H, N, B, 128)) return e;
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.N = N;
+  p.H = H;
+  p.total_q = B * N;
+  p.scale = scale;
+  set_fwd_scale(p, scale);
+  p.win_left = -1;
+  p.win_right = causal ? 0 : -1;
+  p.reverse_tiles = reverse_tiles(p.win_left, p.win_right);
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  const int rows = fwd_rows_per_cta();
+  dim3 grid((N + rows - 1) / rows, H, B);
+  return launch_result(
+      launch_fwd_f32out(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
 }
 
 int fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {

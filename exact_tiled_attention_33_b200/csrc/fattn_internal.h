@@ -122,6 +122,12 @@ LaunchResult launch_fwd_fp8(int d, bool bf16, const CUtensorMap& tmQ, const CUte
                             const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
                             cudaStream_t stream);
 
+// Test-only instance of the forward kernel that writes O in fp32 before rounding (p.o is
+// then a float buffer of the same shape).
+LaunchResult launch_fwd_f32out(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                               const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
+                               cudaStream_t stream);
+
 // Forward grid: x = query-tile pairs, y = heads, z = batch (dense) or sequences (varlen).
 int fwd_rows_per_cta();
 

@@ -5,12 +5,12 @@ namespace fattn {
 
 int fwd_rows_per_cta() { return FwdCfg<128>::BM; }
 
-template <int D, bool BF16, bool FP8 = false>
+template <int D, bool BF16, bool FP8 = false, bool F32O = false>
 static LaunchResult launch_fwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                  const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
                                  cudaStream_t stream) {
   using C = FwdCfg<D, FP8>;
-  auto kern = fa_fwd_kernel<D, BF16, FP8>;
+  auto kern = fa_fwd_kernel<D, BF16, FP8, F32O>;
   static bool configured[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LaunchResult::kCudaError;
@@ -44,6 +44,18 @@ LaunchResult launch_fwd_fp8(int d, bool bf16, const CUtensorMap& tmQ, const CUte
   if (d != 128) return LaunchResult::kUnsupported;
   return bf16 ? launch_fwd_t<128, true, true>(tmQ, tmK, tmV, p, grid, stream)
               : launch_fwd_t<128, false, true>(tmQ, tmK, tmV, p, grid, stream);
+}
+
+LaunchResult launch_fwd_f32out(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                               const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
+                               cudaStream_t stream) {
+  if (d == 128)
+    return bf16 ? launch_fwd_t<128, true, false, true>(tmQ, tmK, tmV, p, grid, stream)
+                : launch_fwd_t<128, false, false, true>(tmQ, tmK, tmV, p, grid, stream);
+  if (d == 64)
+    return bf16 ? launch_fwd_t<64, true, false, true>(tmQ, tmK, tmV, p, grid, stream)
+                : launch_fwd_t<64, false, false, true>(tmQ, tmK, tmV, p, grid, stream);
+  return LaunchResult::kUnsupported;
 }
 
 }  // namespace fattn

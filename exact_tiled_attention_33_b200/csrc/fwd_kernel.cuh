@@ -88,8 +88,10 @@ struct FwdCfg {
   }
 };
 
-// BF16: 16-bit format of the output (and of the operands unless FP8).
-template <int D, bool BF16, bool FP8 = false>
+// BF16: 16-bit format of the output (and of the operands unless FP8).  F32O: the output is
+// written in fp32 before any rounding (a test-only instance: the library's entry points
+// all write 16-bit O; fa_selftest_fwd_f32 exposes this one to the parity tests).
+template <int D, bool BF16, bool FP8 = false, bool F32O = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -431,11 +433,9 @@ __global__ void __launch_bounds__(384, 1)
     }
     const bool valid = i < Lq;
     const float inv_l = (LR > 0.f) ? p.v_descale / LR : 0.f;
-    uint16_t* orow;
-    if (p.cu_q != nullptr)
-      orow = reinterpret_cast<uint16_t*>(p.o) + ((size_t)(q_row0 + i) * p.H + h) * D;
-    else
-      orow = reinterpret_cast<uint16_t*>(p.o) + (((size_t)bcoord * p.N + i) * p.H + h) * D;
+    const size_t orow_idx = (p.cu_q != nullptr) ? ((size_t)(q_row0 + i) * p.H + h) * D
+                                                : (((size_t)bcoord * p.N + i) * p.H + h) * D;
+    uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + orow_idx;
     // this half stores O columns [half * D/2, (half + 1) * D/2)
 #pragma unroll 1
     for (int q = half * (D / 64); q < (half + 1) * (D / 64); ++q) {
@@ -447,6 +447,16 @@ __global__ void __launch_bounds__(384, 1)
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      if constexpr (F32O) {
+        if (valid) {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + orow_idx + q * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            dst[v4] = make_float4(__uint_as_float(o[4 * v4]) * inv_l, __uint_as_float(o[4 * v4 + 1]) * inv_l,
+                                  __uint_as_float(o[4 * v4 + 2]) * inv_l, __uint_as_float(o[4 * v4 + 3]) * inv_l);
+        }
+        continue;
       }
       uint32_t pk[16];
 #pragma unroll

@@ -34,7 +34,8 @@ independent of every other row), not an online or tiled reformulation.
 
 Parity status: every function here is pinned — the dense, causal, varlen and backward
 functions by tests/test_oracle_pins.py (closed forms, invariants, brute force, finite
-differences, a hand-worked golden example), the sliding window by
+differences, a hand-worked golden example; the batched [B, N, H, d] forward and backward
+against torch autograd of the naive formula on that layout), the sliding window by
 tests/test_oracle_window_pins.py, the decode step and paged gather by
 tests/test_oracle_decode_pins.py, and the E4M3 decoding and FP8 forward by
 tests/test_oracle_fp8_pins.py.

@@ -3,14 +3,20 @@
 Tolerances are the ones the target fixes for 16-bit inputs with fp32 accumulation:
   max |O - O_ref| <= 1e-2, max |LSE - LSE_ref| <= 1e-3,
   max |dX - dX_ref| <= 2e-2 * max |dX_ref| for dX in dQ, dK, dV.
-For O one documented reading applies: the output is stored in 16 bits, and where |O|
-is large (the peaky Q,K x4 workload reaches |O| ~ 5) a correctly rounded 16-bit value
-can sit up to half a 16-bit ulp from the fp64 value, which alone can exceed 1e-2.  The
-check therefore allows 1e-2 plus half an ulp of the output format at O_ref; the literal
-maximum error is reported next to it.
+O is checked against the literal 1e-2 everywhere except on the peaky workloads (Q and K
+scaled by 4, so that each softmax row is nearly one-hot and |O| reaches ~5): there a
+correctly rounded 16-bit output can sit half a 16-bit ulp (up to 2^-6 at |O| in [4, 8))
+from the fp64 value, which alone exceeds 1e-2, so the stored output is allowed 1e-2 plus
+half an ulp of the output format at O_ref.  For those workloads the literal 1e-2 is
+applied instead to the kernel's fp32 output before rounding (fa_selftest_fwd_f32).
+
+Every check records its maximum error; when FATTN_PARITY_JSON names a file, the whole
+session's records are written there (tests/conftest.py).
 """
 
 from __future__ import annotations
+
+import os
 
 import numpy as np
 import torch
@@ -18,6 +24,15 @@ import torch
 O_TOL = 1e-2
 LSE_TOL = 1e-3
 GRAD_REL_TOL = 2e-2
+
+# (test id, quantity, max error, bound) per check, for the session report
+RECORDS: list = []
+
+
+def _record(what: str, err: float, bound: float, kind: str) -> None:
+    test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+    RECORDS.append({"test": test, "what": what, "kind": kind, "max_err": float(err),
+                    "bound": float(bound)})
 
 
 def half_ulp(x: np.ndarray, dtype: str) -> np.ndarray:
@@ -28,14 +43,19 @@ def half_ulp(x: np.ndarray, dtype: str) -> np.ndarray:
     return 0.5 * 2.0 ** (e - (mant - 1))
 
 
-def check_o(o_gpu: np.ndarray, o_ref: np.ndarray, dtype: str, what: str = "O") -> float:
+def check_o(o_gpu: np.ndarray, o_ref: np.ndarray, dtype: str, what: str = "O",
+            peaky: bool = False) -> float:
+    """max |O - O_ref| <= 1e-2; with peaky=True (Q,K x4 workloads only) the stored 16-bit
+    output may add half a 16-bit ulp at O_ref."""
     err = np.abs(o_gpu.astype(np.float64) - o_ref)
     assert np.all(np.isfinite(o_gpu)), f"{what}: non-finite output"
-    allowed = O_TOL + half_ulp(o_ref, dtype)
+    allowed = O_TOL + half_ulp(o_ref, dtype) if peaky else O_TOL
     bad = err > allowed
+    m = float(err.max()) if err.size else 0.0
+    _record(what, m, O_TOL, "O (peaky: + half ulp)" if peaky else "O")
     assert not bad.any(), (f"{what}: {int(bad.sum())} elements over tolerance; max err "
-                           f"{err.max():.4g}")
-    return float(err.max()) if err.size else 0.0
+                           f"{m:.4g}")
+    return m
 
 
 def check_lse(lse_gpu: np.ndarray, lse_ref: np.ndarray, what: str = "LSE") -> float:
@@ -43,24 +63,54 @@ def check_lse(lse_gpu: np.ndarray, lse_ref: np.ndarray, what: str = "LSE") -> fl
     assert np.array_equal(np.isposinf(lse_gpu), inf_ref), f"{what}: +inf pattern differs"
     fin = ~inf_ref
     if not fin.any():
+        _record(what, 0.0, LSE_TOL, "LSE")
         return 0.0
     err = np.abs(lse_gpu[fin].astype(np.float64) - lse_ref[fin])
     assert np.all(np.isfinite(lse_gpu[fin])), f"{what}: non-finite values"
+    _record(what, err.max(), LSE_TOL, "LSE")
     assert err.max() <= LSE_TOL, f"{what}: max err {err.max():.4g}"
     return float(err.max())
 
 
 def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, scale_ref=None,
                extra=None) -> float:
-    """max |g - g_ref| <= 2e-2 * max|g_ref| (plus an optional per-element `extra`)."""
+    """max |g - g_ref| <= 2e-2 * max|g_ref| (plus an optional per-element `extra`).
+    Returns (and records) the error as a fraction of max|g_ref|."""
     ref_max = np.abs(g_ref).max() if scale_ref is None else scale_ref
     err = np.abs(g_gpu.astype(np.float64) - g_ref)
     assert np.all(np.isfinite(g_gpu)), f"{what}: non-finite gradient"
     tol = GRAD_REL_TOL * max(ref_max, 1e-30)
     allowed = tol if extra is None else tol + extra
     over = err - allowed
+    rel = float(err.max() / max(ref_max, 1e-30)) if err.size else 0.0
+    _record(what, rel, GRAD_REL_TOL, "grad / max|grad_ref|" + ("" if extra is None
+                                                                 else " (+ O16 term)"))
     assert over.max() <= 0, f"{what}: max err {err.max():.4g} > {tol:.4g} (+extra)"
-    return float(err.max() / max(ref_max, 1e-30))
+    return rel
+
+
+def check_grad_segments(got, ref, cu_q, cu_k, what, scale, causal, dtype, q, k, v, do,
+                        window=None, o16_always=False):
+    """Varlen gradients (dQ [total_q,H,d], dK, dV [total_k,H,d]) checked per (segment, head):
+    each slice against 2e-2 x its own max|grad_ref|, so a short segment with small gradients
+    is not judged on its neighbours' scale.  Degenerate slices (a segment with at most two
+    queries or keys, or every slice when o16_always) add the first-order term of D computed
+    from the 16-bit O (o16_term_in_d), where the exact dQ and dK nearly cancel."""
+    H = got[0].shape[1]
+    for s in range(len(cu_q) - 1):
+        a, b, c, e = int(cu_q[s]), int(cu_q[s + 1]), int(cu_k[s]), int(cu_k[s + 1])
+        for h in range(H):
+            bq = bk = None
+            if b > a and e > c and (o16_always or min(b - a, e - c) <= 2):
+                bq, bk = o16_term_in_d(q[a:b, h], k[c:e, h], v[c:e, h], do[a:b, h], scale,
+                                       causal, dtype, window=window)
+            if b > a:
+                check_grad(got[0][a:b, h], ref[0][a:b, h], f"{what} dQ[seg {s}, h {h}]",
+                           extra=bq)
+            if e > c:
+                check_grad(got[1][c:e, h], ref[1][c:e, h], f"{what} dK[seg {s}, h {h}]",
+                           extra=bk)
+                check_grad(got[2][c:e, h], ref[2][c:e, h], f"{what} dV[seg {s}, h {h}]")
 
 
 def o16_term_in_d(q, k, v, do, scale, causal, dtype, window=None):

@@ -96,6 +96,14 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
     st = lib.fa_bwd_noalloc(P, P, P, P, P, P, P, P, P, 8, 16384, 64, 128, 0.1, 1, 0, None)
     assert st == _lib.FA_ERR_UNSUPPORTED
     assert b"scratch capacity" in lib.fa_last_error()
+    # the exact edge: B*H*N = 4194305 (= 5 * 838861) is one element over the capacity ...
+    assert lib.fa_bwd_noalloc(P, P, P, P, P, P, P, P, P, 1, 838861, 5, 128, 0.1, 1, 0,
+                              None) == _lib.FA_ERR_UNSUPPORTED
+    assert b"scratch capacity" in lib.fa_last_error()
+    # ... while B*H*N = 4194304 passes the capacity check (it then fails later, on this
+    # GPU-less host, for a reason that is not the capacity)
+    st = lib.fa_bwd_noalloc(P, P, P, P, P, P, P, P, P, 64, 1024, 64, 128, 0.1, 1, 0, None)
+    assert st != _lib.FA_OK and b"scratch capacity" not in lib.fa_last_error()
 
 
 def test_empty_problems_are_noops(lib):

@@ -10,7 +10,8 @@ import torch
 import oracle
 from exact_tiled_attention_33_b200 import attention as fa
 from exact_tiled_attention_33_b200 import workloads as wl
-from tests.parity import check_grad, f64, guard_intact, guarded_empty, o16_term_in_d
+from tests.parity import (check_grad, check_grad_segments, f64, guard_intact, guarded_empty,
+                          o16_term_in_d)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -154,11 +155,11 @@ def run_varlen_bwd(lens_q, lens_k, H, d, causal, dtype="bf16", seed=3, perturb=N
     o, lse = fa.varlen_fwd(qd, kd, vd, cq, ck, mq, mk, w.softmax_scale, causal)
     dq, dk, dv = fa.varlen_bwd(qd, kd, vd, o, lse, dod, cq, ck, mq, mk, w.softmax_scale, causal)
     assert fa.device_status() == 0
-    ref = oracle.varlen_attention_backward(wl.to_f64(q), wl.to_f64(k), wl.to_f64(v), wl.to_f64(do),
-                                           cu_q, cu_k, w.softmax_scale, causal)
-    for name, got, r in zip(("dQ", "dK", "dV"), (dq, dk, dv), ref):
-        # the tolerance scale is max |grad_ref| over the whole packed tensor
-        check_grad(f64(got), r, name)
+    qf, kf, vf, dof = (wl.to_f64(x) for x in (q, k, v, do))
+    ref = oracle.varlen_attention_backward(qf, kf, vf, dof, cu_q, cu_k, w.softmax_scale, causal)
+    got = [f64(x) for x in (dq, dk, dv)]
+    check_grad_segments(got, ref, cu_q, cu_k, "varlen", w.softmax_scale, causal, dtype,
+                        qf, kf, vf, dof)
     return dq, dk, dv, cu_q, cu_k
 
 

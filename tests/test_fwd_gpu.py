@@ -17,6 +17,11 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
+def is_peaky(w) -> bool:
+    # the Q,K x4 workloads: the only ones whose stored O may add half a 16-bit ulp
+    return getattr(w, "qk_mult", 1.0) != 1.0
+
+
 def run_dense(w, rows_per_head=None, bh_subset=None):
     t = wl.generate(w, with_grad_out=False)
     q, k, v = (t[x].to(DEV) for x in ("q", "k", "v"))
@@ -35,7 +40,8 @@ def run_dense(w, rows_per_head=None, bh_subset=None):
         o_ref, lse_ref = oracle.attention_forward(qf[b, :, h], kf[b, :, h], vf[b, :, h],
                                                   w.softmax_scale, w.causal, rows=rows)
         sel = slice(None) if rows is None else rows
-        eo = max(eo, check_o(og[b, sel, h], o_ref, w.dtype, f"O[b={b},h={h}]"))
+        eo = max(eo, check_o(og[b, sel, h], o_ref, w.dtype, f"O[b={b},h={h}]",
+                             peaky=is_peaky(w)))
         el = max(el, check_lse(lg[b, h, sel], lse_ref, f"LSE[b={b},h={h}]"))
     return eo, el, o, lse
 
@@ -82,6 +88,30 @@ def test_llama_sampled(name):
 def test_long_sampled(name):
     w = wl.get(name)
     run_dense(w, rows_per_head=128)
+
+
+@pytest.mark.parametrize("name", ["long_peaky_causal", "long_peaky_noncausal"])
+def test_long_peaky_fp32_output_literal_bound(name):
+    # The same kernel with O written in fp32 before rounding: the literal |O - O_ref| <= 1e-2
+    # holds on the peaky workloads too, where only the 16-bit rounding of |O| ~ 5 can exceed it.
+    w = wl.get(name)
+    t = wl.generate(w, with_grad_out=False)
+    q, k, v = (t[x].to(DEV) for x in ("q", "k", "v"))
+    o32, lse = fa.fwd_f32out(q, k, v, w.softmax_scale, w.causal)
+    o16, lse16 = fa.fwd(q, k, v, w.softmax_scale, w.causal)
+    assert fa.device_status() == 0
+    # the 16-bit entry point returns exactly this fp32 output rounded to nearest-even
+    assert torch.equal(o32.to(o16.dtype), o16) and torch.equal(lse, lse16)
+    og, lg = f64(o32), f64(lse)
+    qf, kf, vf = (wl.to_f64(t[x]) for x in ("q", "k", "v"))
+    B, N, H, _ = q.shape
+    for b in range(B):
+        for h in range(0, H, 3):
+            rows = wl.sample_rows(N, 128, 1000 + b * H + h)
+            o_ref, lse_ref = oracle.attention_forward(qf[b, :, h], kf[b, :, h], vf[b, :, h],
+                                                      w.softmax_scale, w.causal, rows=rows)
+            check_o(og[b, rows, h], o_ref, "fp32", f"O fp32[b={b},h={h}]")
+            check_lse(lg[b, h, rows], lse_ref, f"LSE[b={b},h={h}]")
 
 
 def test_deterministic():

@@ -12,8 +12,8 @@ import torch
 import oracle
 from exact_tiled_attention_33_b200 import attention as fa
 from exact_tiled_attention_33_b200 import workloads as wl
-from tests.parity import (check_grad, check_lse, check_o, f64, guard_intact, guarded_empty,
-                          o16_term_in_d)
+from tests.parity import (check_grad, check_grad_segments, check_lse, check_o, f64, guard_intact,
+                          guarded_empty, o16_term_in_d)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -194,20 +194,10 @@ def run_varlen(lens_q, lens_k, H, d, window, seed, bwd=True):
     assert fa.device_status() == 0
     gq, gk, gv = oracle.varlen_attention_backward(qf, kf, vf, dof, cq, ck, scale, False,
                                                   window=window)
-    eq = ek = None
-    if tuple(window) == (0, 0):  # one key per row: exact dQ = dK = 0
-        eq, ek = np.zeros_like(qf), np.zeros_like(kf)
-        for s in range(len(lens_q)):
-            a, b, c, e = cq[s], cq[s + 1], ck[s], ck[s + 1]
-            if b == a or e == c:
-                continue
-            for h in range(H):
-                eq[a:b, h], ek[c:e, h] = o16_term_in_d(qf[a:b, h], kf[c:e, h], vf[c:e, h],
-                                                       dof[a:b, h], scale, False, "bf16",
-                                                       window=window)
-    check_grad(f64(dq), gq, f"varlen dQ window {window}", extra=eq)
-    check_grad(f64(dk), gk, f"varlen dK window {window}", extra=ek)
-    check_grad(f64(dv), gv, f"varlen dV window {window}")
+    # per (segment, head) scale; a window of one key per row makes the exact dQ = dK = 0
+    check_grad_segments([f64(dq), f64(dk), f64(dv)], (gq, gk, gv), cq, ck,
+                        f"varlen window {window}", scale, False, "bf16", qf, kf, vf, dof,
+                        window=window, o16_always=tuple(window) == (0, 0))
 
 
 @pytest.mark.parametrize("window", [(1, 0), (100, 0), (128, 3), (20, 20), (-1, 7), (50, -1)])

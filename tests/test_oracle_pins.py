@@ -333,6 +333,28 @@ def test_batched_layout():
     np.testing.assert_allclose(lse[1, 2], l1, atol=1e-15)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_batched_backward_layout(causal):
+    # attention_backward_bhsd on the [batch, seqlen, heads, head_dim] layout against torch
+    # autograd of the naive formula evaluated directly on that layout (a library witness,
+    # independent of the oracle): B != H and unequal sizes make a swapped batch/head or
+    # seqlen/head index, or a gradient written to the wrong slot, fail.
+    B, N, H, d, scale = 2, 7, 3, 4, 0.6
+    q = rnd((B, N, H, d), 97); k = rnd((B, N, H, d), 98); v = rnd((B, N, H, d), 99)
+    do = rnd((B, N, H, d), 100)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    s = scale * torch.einsum("bihc,bjhc->bhij", tq, tk)
+    if causal:
+        s = s.masked_fill(torch.triu(torch.ones(N, N, dtype=torch.bool), 1), float("-inf"))
+    o = torch.einsum("bhij,bjhc->bihc", torch.softmax(s, dim=-1), tv)
+    (o * torch.tensor(do)).sum().backward()
+    dq, dk, dv = oracle.attention_backward_bhsd(q, k, v, do, scale, causal)
+    assert dq.shape == q.shape and dk.shape == k.shape and dv.shape == v.shape
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-12)
+
+
 def test_row_subsets_match_full():
     L, d = 2100, 16  # spans more than two oracle row blocks
     q = rnd((L, d), 93); k = rnd((L, d), 94); v = rnd((L, d), 95); do = rnd((L, d), 96)
