@@ -31,6 +31,11 @@ SIGNATURES = {
     "fa_varlen_bwd_workspace_size": (_sz, [_i, _i, _i]),
     "fa_varlen_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                            _f, _i, _i, _i, _i, _vp, _sz, _i, _vp]),
+    "fa_bwd_deterministic": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                  _f, _i, _i, _vp, _sz, _i, _vp]),
+    "fa_varlen_bwd_deterministic": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                         _i, _i, _i, _i, _f, _i, _i, _i, _i, _i, _vp, _sz, _i,
+                                         _vp]),
     "fa_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                             _i, _vp]),
     "fa_fwd_local": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _i, _vp]),

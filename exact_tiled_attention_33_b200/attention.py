@@ -119,9 +119,32 @@ def varlen_bwd_workspace(total_q, H, d, device) -> torch.Tensor:
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
 
 
+def _bwd_dense(name, q, k, v, o, lse, dout, scale, window, workspace, dq, dk, dv, deterministic):
+    dtype = _check(q, k, v, o, dout)
+    B, N, H, d = q.shape
+    wl, wr = window
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws = bwd_workspace(B, N, H, d, q.device) if workspace is None else workspace
+    lib = _lib.load()
+    fn = lib.fa_bwd_deterministic if deterministic else lib.fa_bwd_local
+    with torch.cuda.device(q.device):
+        st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                _ptr(dv), B, N, H, d, scale, wl, wr, _ptr(ws), ws.numel(), dtype, _stream(q))
+    _lib.check(st, "fa_bwd_deterministic" if deterministic else name)
+    return dq, dk, dv
+
+
 def bwd(q, k, v, o, lse, dout, softmax_scale=None, causal=False, workspace=None,
-        dq=None, dk=None, dv=None):
-    """Dense backward. Returns (dq, dk, dv), each [B, N, H, d]."""
+        dq=None, dk=None, dv=None, deterministic=False):
+    """Dense backward. Returns (dq, dk, dv), each [B, N, H, d].  deterministic=True runs the
+    two-pass backward (fa_bwd_deterministic): bitwise-reproducible dQ."""
+    if deterministic:
+        d = q.shape[-1]
+        scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+        return _bwd_dense("fa_bwd", q, k, v, o, lse, dout, scale, (-1, 0 if causal else -1),
+                          workspace, dq, dk, dv, True)
     dtype = _check(q, k, v, o, dout)
     B, N, H, d = q.shape
     scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
@@ -158,9 +181,38 @@ def bwd_noalloc(q, k, v, o, lse, dout, softmax_scale=None, causal=False, dq=None
     return dq, dk, dv
 
 
+def _bwd_varlen_det(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                    max_seqlen_k, scale, window, workspace, dq, dk, dv):
+    dtype = _check(q, k, v, o, dout)
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    wl, wr = window
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws = varlen_bwd_workspace(total_q, H, d, q.device) if workspace is None else workspace
+    lib = _lib.load()
+    with torch.cuda.device(q.device):
+        st = lib.fa_varlen_bwd_deterministic(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+            _ptr(dv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q),
+            int(max_seqlen_k), H, d, scale, wl, wr, cu_seqlens_q.numel() - 1, total_q, total_k,
+            _ptr(ws), ws.numel(), dtype, _stream(q))
+    _lib.check(st, "fa_varlen_bwd_deterministic")
+    return dq, dk, dv
+
+
 def varlen_bwd(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-               softmax_scale=None, causal=False, workspace=None, dq=None, dk=None, dv=None):
-    """Varlen backward. Returns (dq [total_q,H,d], dk, dv [total_k,H,d])."""
+               softmax_scale=None, causal=False, workspace=None, dq=None, dk=None, dv=None,
+               deterministic=False):
+    """Varlen backward. Returns (dq [total_q,H,d], dk, dv [total_k,H,d]).  deterministic=True
+    runs fa_varlen_bwd_deterministic."""
+    if deterministic:
+        d = q.shape[-1]
+        scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+        return _bwd_varlen_det(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                               max_seqlen_k, scale, (-1, 0 if causal else -1), workspace, dq, dk,
+                               dv)
     dtype = _check(q, k, v, o, dout)
     total_q, H, d = q.shape
     total_k = k.shape[0]
@@ -238,29 +290,25 @@ def varlen_fwd_local(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seql
 
 
 def bwd_local(q, k, v, o, lse, dout, window, softmax_scale=None, workspace=None, dq=None,
-              dk=None, dv=None):
-    """Dense sliding-window backward (fa_bwd_local). Returns (dq, dk, dv)."""
-    dtype = _check(q, k, v, o, dout)
-    B, N, H, d = q.shape
-    wl, wr = _window(window)
+              dk=None, dv=None, deterministic=False):
+    """Dense sliding-window backward (fa_bwd_local, or fa_bwd_deterministic).
+    Returns (dq, dk, dv)."""
+    d = q.shape[-1]
     scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    ws = bwd_workspace(B, N, H, d, q.device) if workspace is None else workspace
-    lib = _lib.load()
-    with torch.cuda.device(q.device):
-        st = lib.fa_bwd_local(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
-                              _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, d, scale, wl, wr, _ptr(ws),
-                              ws.numel(), dtype, _stream(q))
-    _lib.check(st, "fa_bwd_local")
-    return dq, dk, dv
+    return _bwd_dense("fa_bwd_local", q, k, v, o, lse, dout, scale, _window(window), workspace,
+                      dq, dk, dv, deterministic)
 
 
 def varlen_bwd_local(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
                      max_seqlen_k, window, softmax_scale=None, workspace=None, dq=None, dk=None,
-                     dv=None):
-    """Packed sliding-window backward (fa_varlen_bwd_local). Returns (dq, dk, dv)."""
+                     dv=None, deterministic=False):
+    """Packed sliding-window backward (fa_varlen_bwd_local, or
+    fa_varlen_bwd_deterministic). Returns (dq, dk, dv)."""
+    if deterministic:
+        d = q.shape[-1]
+        scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+        return _bwd_varlen_det(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                               max_seqlen_k, scale, _window(window), workspace, dq, dk, dv)
     dtype = _check(q, k, v, o, dout)
     total_q, H, d = q.shape
     total_k = k.shape[0]
@@ -427,60 +475,66 @@ class FlashAttnFunction(torch.autograd.Function):
     window None: the causal flag decides; else the sliding-window calls."""
 
     @staticmethod
-    def forward(ctx, q, k, v, softmax_scale, causal, window):
+    def forward(ctx, q, k, v, softmax_scale, causal, window, deterministic):
         if window is None:
             o, lse = fwd(q, k, v, softmax_scale, causal)
         else:
             o, lse = fwd_local(q, k, v, window, softmax_scale)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.args = (softmax_scale, causal, window)
+        ctx.args = (softmax_scale, causal, window, deterministic)
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse = ctx.saved_tensors
-        scale, causal, window = ctx.args
+        scale, causal, window, det = ctx.args
         if window is None:
-            dq, dk, dv = bwd(q, k, v, o, lse, do.contiguous(), scale, causal)
+            dq, dk, dv = bwd(q, k, v, o, lse, do.contiguous(), scale, causal, deterministic=det)
         else:
-            dq, dk, dv = bwd_local(q, k, v, o, lse, do.contiguous(), window, scale)
-        return dq, dk, dv, None, None, None
+            dq, dk, dv = bwd_local(q, k, v, o, lse, do.contiguous(), window, scale,
+                                   deterministic=det)
+        return dq, dk, dv, None, None, None, None
 
 
 class FlashAttnVarlenFunction(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, cu_q, cu_k, max_q, max_k, softmax_scale, causal, window):
+    def forward(ctx, q, k, v, cu_q, cu_k, max_q, max_k, softmax_scale, causal, window,
+                deterministic):
         if window is None:
             o, lse = varlen_fwd(q, k, v, cu_q, cu_k, max_q, max_k, softmax_scale, causal)
         else:
             o, lse = varlen_fwd_local(q, k, v, cu_q, cu_k, max_q, max_k, window, softmax_scale)
         ctx.save_for_backward(q, k, v, o, lse, cu_q, cu_k)
-        ctx.args = (max_q, max_k, softmax_scale, causal, window)
+        ctx.args = (max_q, max_k, softmax_scale, causal, window, deterministic)
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse, cu_q, cu_k = ctx.saved_tensors
-        max_q, max_k, scale, causal, window = ctx.args
+        max_q, max_k, scale, causal, window, det = ctx.args
         if window is None:
             dq, dk, dv = varlen_bwd(q, k, v, o, lse, do.contiguous(), cu_q, cu_k, max_q, max_k,
-                                    scale, causal)
+                                    scale, causal, deterministic=det)
         else:
             dq, dk, dv = varlen_bwd_local(q, k, v, o, lse, do.contiguous(), cu_q, cu_k, max_q,
-                                          max_k, window, scale)
-        return dq, dk, dv, None, None, None, None, None, None, None
+                                          max_k, window, scale, deterministic=det)
+        return dq, dk, dv, None, None, None, None, None, None, None, None
 
 
-def flash_attn_func(q, k, v, softmax_scale=None, causal=False, window=None):
+def flash_attn_func(q, k, v, softmax_scale=None, causal=False, window=None,
+                    deterministic=False):
     """[batch, seqlen, heads, head_dim] attention with autograd.  window=(left, right)
-    selects sliding-window attention (and overrides causal)."""
+    selects sliding-window attention (and overrides causal); deterministic=True makes the
+    backward bitwise reproducible (the pages' deterministic mode)."""
     return FlashAttnFunction.apply(q, k, v, softmax_scale, causal,
-                                   None if window is None else _window(window))
+                                   None if window is None else _window(window), deterministic)
 
 
 def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                           softmax_scale=None, causal=False, window=None):
-    """Packed variable-length attention with autograd (window as in flash_attn_func)."""
+                           softmax_scale=None, causal=False, window=None, deterministic=False):
+    """Packed variable-length attention with autograd (window and deterministic as in
+    flash_attn_func)."""
     return FlashAttnVarlenFunction.apply(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
                                          max_seqlen_k, softmax_scale, causal,
-                                         None if window is None else _window(window))
+                                         None if window is None else _window(window),
+                                         deterministic)

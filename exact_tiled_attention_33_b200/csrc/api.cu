@@ -441,14 +441,27 @@ int fa_varlen_fwd_fp8(const void* q, const void* k, const void* v, void* o, floa
       launch_fwd_fp8(d, out_dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
 }
 
+namespace {
+
+// Backward workspace: D = rowsum(dO ∘ O) (fp32, one per token row and head), then, for the
+// single-pass backward, the fp32 dQ sums (H x rows rounded up to 32 x d).
+size_t d_vector_bytes(long long rows, long long H) { return align256((size_t)rows * H * 4); }
+long long acc_rows_of(long long rows) { return (rows + 31) / 32 * 32; }
+size_t dq_sum_bytes(long long rows, long long H, long long d) {
+  return align256((size_t)acc_rows_of(rows) * H * d * 4);
+}
+
+}  // namespace
+
 size_t fa_bwd_workspace_size(int B, int N, int H, int d) {
   if (B <= 0 || N <= 0 || H <= 0 || d <= 0) return 0;
-  return align256((size_t)B * H * N * 4);
+  const long long rows = (long long)B * N;
+  return d_vector_bytes(rows, H) + dq_sum_bytes(rows, H, d);
 }
 
 size_t fa_varlen_bwd_workspace_size(int total_q, int H, int d) {
   if (total_q <= 0 || H <= 0 || d <= 0) return 0;
-  return align256((size_t)H * total_q * 4);
+  return d_vector_bytes(total_q, H) + dq_sum_bytes(total_q, H, d);
 }
 
 namespace {
@@ -458,8 +471,9 @@ int bwd_common(const void* q, const void* k, const void* v, const void* o, const
                const float* lse, void* dq, void* dk, void* dv, const int* cu_q, const int* cu_k,
                int H, int d, float scale, int wl, int wr, long long q_rows, long long k_rows,
                int N, int batches, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
-               void* workspace,
-               size_t workspace_bytes, size_t need, int dtype, cudaStream_t stream) {
+               void* workspace, size_t workspace_bytes, bool single_pass, int dtype,
+               cudaStream_t stream) {
+  const size_t need = d_vector_bytes(q_rows, H) + (single_pass ? dq_sum_bytes(q_rows, H, d) : 0);
   if (int e = normalize_window(&wl, &wr, max_seqlen_q, max_seqlen_k)) return e;
   if (int e = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv, workspace})) return e;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -477,6 +491,10 @@ int bwd_common(const void* q, const void* k, const void* v, const void* o, const
   p.q = q; p.k = k; p.v = v; p.o = o; p.dout = dout; p.lse = lse;
   p.dq = dq; p.dk = dk; p.dv = dv;
   p.dvec = static_cast<float*>(workspace);
+  p.dq_acc = single_pass ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                    d_vector_bytes(q_rows, H))
+                         : nullptr;
+  p.acc_rows = acc_rows_of(q_rows);
   p.cu_q = cu_q; p.cu_k = cu_k;
   p.B = cu_q ? 1 : batches; p.N = N; p.H = H;
   p.total_q = total_q; p.total_k = total_k;
@@ -487,6 +505,9 @@ int bwd_common(const void* q, const void* k, const void* v, const void* o, const
   p.reverse_tiles = reverse_tiles(wl, wr);
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
+  if (single_pass)
+    return launch_result(launch_bwd_fused(d, dtype == FA_BF16, mq, mk, mv, mdo, p, q_rows,
+                                          max_seqlen_q, max_seqlen_k, batches, stream));
   return launch_result(launch_bwd(d, dtype == FA_BF16, mq, mk, mv, mdo, p, q_rows, max_seqlen_q,
                                   max_seqlen_k, batches, stream));
 }
@@ -497,8 +518,8 @@ namespace {
 
 int bwd_dense(const void* q, const void* k, const void* v, const void* o, const void* dout,
               const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int d,
-              float scale, int wl, int wr, void* workspace, size_t workspace_bytes, int dtype,
-              void* stream) {
+              float scale, int wl, int wr, void* workspace, size_t workspace_bytes,
+              bool single_pass, int dtype, void* stream) {
   if (int e = check_common(H, d, dtype, scale)) return e;
   if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
   if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
@@ -506,15 +527,15 @@ int bwd_dense(const void* q, const void* k, const void* v, const void* o, const 
   if (int e = check_grid(B, H, N)) return e;
   return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, nullptr, nullptr, H, d, scale, wl, wr,
                     (long long)B * N, (long long)B * N, N, B, N, N, B * N, B * N, workspace,
-                    workspace_bytes, fa_bwd_workspace_size(B, N, H, d), dtype,
-                    (cudaStream_t)stream);
+                    workspace_bytes, single_pass, dtype, (cudaStream_t)stream);
 }
 
 int bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
                const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
                const int* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k, int H, int d,
                float scale, int wl, int wr, int num_seqs, int total_q, int total_k,
-               void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+               void* workspace, size_t workspace_bytes, bool single_pass, int dtype,
+               void* stream) {
   if (int e = check_common(H, d, dtype, scale)) return e;
   if (num_seqs < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
     return fail(FA_ERR_INVALID_ARG, "sizes must be >= 0");
@@ -535,8 +556,8 @@ int bwd_varlen(const void* q, const void* k, const void* v, const void* o, const
   if (int e = check_grid(num_seqs, H, std::max(max_seqlen_q, max_seqlen_k))) return e;
   return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, H, d, scale,
                     wl, wr, total_q, total_k, 0, num_seqs, max_seqlen_q, max_seqlen_k, total_q,
-                    total_k, workspace, workspace_bytes,
-                    fa_varlen_bwd_workspace_size(total_q, H, d), dtype, (cudaStream_t)stream);
+                    total_k, workspace, workspace_bytes, single_pass, dtype,
+                    (cudaStream_t)stream);
 }
 
 }  // namespace
@@ -546,7 +567,16 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            int causal, void* workspace, size_t workspace_bytes, int dtype, void* stream) {
   g_last_error.clear();
   return bwd_dense(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, d, scale, -1, causal ? 0 : -1,
-                   workspace, workspace_bytes, dtype, stream);
+                   workspace, workspace_bytes, true, dtype, stream);
+}
+
+int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int N, int H, int d, float scale, int window_left, int window_right,
+                         void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  g_last_error.clear();
+  return bwd_dense(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, d, scale, window_left,
+                   window_right, workspace, workspace_bytes, false, dtype, stream);
 }
 
 int fa_bwd_local(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -555,7 +585,7 @@ int fa_bwd_local(const void* q, const void* k, const void* v, const void* o, con
                  size_t workspace_bytes, int dtype, void* stream) {
   g_last_error.clear();
   return bwd_dense(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, d, scale, window_left,
-                   window_right, workspace, workspace_bytes, dtype, stream);
+                   window_right, workspace, workspace_bytes, true, dtype, stream);
 }
 
 int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -566,7 +596,20 @@ int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, co
   g_last_error.clear();
   return bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
                     max_seqlen_k, H, d, scale, -1, causal ? 0 : -1, num_seqs, total_q, total_k,
-                    workspace, workspace_bytes, dtype, stream);
+                    workspace, workspace_bytes, true, dtype, stream);
+}
+
+int fa_varlen_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                const int* cu_seqlens_q, const int* cu_seqlens_k,
+                                int max_seqlen_q, int max_seqlen_k, int H, int d, float scale,
+                                int window_left, int window_right, int num_seqs, int total_q,
+                                int total_k, void* workspace, size_t workspace_bytes, int dtype,
+                                void* stream) {
+  g_last_error.clear();
+  return bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                    max_seqlen_k, H, d, scale, window_left, window_right, num_seqs, total_q,
+                    total_k, workspace, workspace_bytes, false, dtype, stream);
 }
 
 int fa_varlen_bwd_local(const void* q, const void* k, const void* v, const void* o,
@@ -578,7 +621,7 @@ int fa_varlen_bwd_local(const void* q, const void* k, const void* v, const void*
   g_last_error.clear();
   return bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
                     max_seqlen_k, H, d, scale, window_left, window_right, num_seqs, total_q,
-                    total_k, workspace, workspace_bytes, dtype, stream);
+                    total_k, workspace, workspace_bytes, true, dtype, stream);
 }
 
 // ------------------------------------------------------------------ allocation-free backward
@@ -620,8 +663,7 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   if (int e = noalloc_scratch(&scratch)) return e;
   return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, nullptr, nullptr, H, d, scale, -1,
                     causal ? 0 : -1, (long long)B * N, (long long)B * N, N, B, N, N, B * N, B * N,
-                    scratch,
-                    sizeof(float) * kNoAllocScratchFloats, fa_bwd_workspace_size(B, N, H, d), dtype,
+                    scratch, sizeof(float) * kNoAllocScratchFloats, false, dtype,
                     (cudaStream_t)stream);
 }
 

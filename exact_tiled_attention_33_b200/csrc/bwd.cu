@@ -1,7 +1,9 @@
 // Backward kernel instantiations and launcher: D preprocess, then the dK/dV pass and the
 // dQ pass, all on the caller's stream.
 #include <algorithm>
+#include <mutex>
 
+#include "bwd_fused_kernel.cuh"
 #include "bwd_kernel.cuh"
 
 namespace fattn {
@@ -36,6 +38,51 @@ static LaunchResult launch_bwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
   dim3 grid_b((max_seqlen_q + C::BM - 1) / C::BM, p.H, batches);
   fa_bwd_dq_kernel<D, BF16><<<grid_b, C::THREADS, C::SMEM_B, stream>>>(tmQ, tmK, tmV, tmDO, p);
   return cudaGetLastError() == cudaSuccess ? LaunchResult::kOk : LaunchResult::kCudaError;
+}
+
+template <int D, bool BF16>
+static LaunchResult launch_bwd_fused_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                       const CUtensorMap& tmV, const CUtensorMap& tmDO,
+                                       const BwdParams& p, long long q_rows, int max_seqlen_k,
+                                       int batches, cudaStream_t stream) {
+  using C = BwdFusedCfg<D>;
+  static std::once_flag once[64];
+  static cudaError_t set_err[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return LaunchResult::kCudaError;
+  std::call_once(once[dev], [&] {
+    set_err[dev] = cudaFuncSetAttribute(fa_bwd_fused_kernel<D, BF16>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  });
+  if (set_err[dev] != cudaSuccess) return LaunchResult::kCudaError;
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // 1) D = rowsum(dO ∘ O) and zeroed dQ sums
+  const long long warps = q_rows * p.H;
+  const long long pre_blocks = std::min<long long>((warps + 7) / 8, (long long)sms * 16);
+  fa_bwd_pre_acc_kernel<D, BF16><<<(unsigned)pre_blocks, 256, 0, stream>>>(p, q_rows);
+  // 2) dK, dV and the dQ partial sums: one CTA per key tile
+  dim3 grid((max_seqlen_k + C::BN - 1) / C::BN, p.H, batches);
+  fa_bwd_fused_kernel<D, BF16><<<grid, C::THREADS, C::SMEM, stream>>>(tmQ, tmK, tmV, tmDO, p);
+  // 3) dQ = scale * sums, rounded to 16 bits
+  const long long groups = (q_rows + 31) / 32 * p.H;
+  const long long cv_blocks = std::min<long long>(groups, (long long)sms * 8);
+  fa_bwd_dq_convert_kernel<D, BF16><<<(unsigned)cv_blocks, 256, 0, stream>>>(p, q_rows);
+  return cudaGetLastError() == cudaSuccess ? LaunchResult::kOk : LaunchResult::kCudaError;
+}
+
+LaunchResult launch_bwd_fused(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                              const CUtensorMap& tmV, const CUtensorMap& tmDO, const BwdParams& p,
+                              long long q_rows, int max_seqlen_q, int max_seqlen_k, int batches,
+                              cudaStream_t stream) {
+  (void)max_seqlen_q;
+  if (d == 128)
+    return bf16 ? launch_bwd_fused_t<128, true>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream)
+                : launch_bwd_fused_t<128, false>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream);
+  if (d == 64)
+    return bf16 ? launch_bwd_fused_t<64, true>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream)
+                : launch_bwd_fused_t<64, false>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream);
+  return LaunchResult::kUnsupported;
 }
 
 LaunchResult launch_bwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,

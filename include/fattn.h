@@ -89,12 +89,20 @@ int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* l
                   int max_seqlen_k, int H, int d, float scale, int causal, int num_seqs,
                   int total_q, int total_k, int dtype, void* stream);
 
-/* Workspace bytes the dense backward needs: D = rowsum(dO ∘ O) [B,H,N] fp32, rounded up
- * to a multiple of 256 bytes (dQ, dK and dV are written directly, with no atomics). */
+/* Workspace bytes the dense backward needs: D = rowsum(dO ∘ O) [B,H,N] fp32 rounded up to
+ * a multiple of 256 bytes, followed by the fp32 sums of dQ (H x B*N rounded up to 32 x d
+ * floats, again rounded to 256 bytes).  Linear in N: no N x N buffer exists. */
 size_t fa_bwd_workspace_size(int B, int N, int H, int d);
 
 /* Dense backward: recomputes P from q, k and lse (as written by fa_fwd with the same
  * scale and causal flag) and writes dq, dk, dv [B,N,H,d].
+ * One pass per 128-key tile computes the five products of every (query tile, key tile)
+ * pair — Sᵀ = K Qᵀ, dPᵀ = V dOᵀ, dV += Pᵀ dO, dK += dSᵀ Q and dQ += dS K — ("global
+ * gradients split into local updates", page "Flash Attention V3：大模型训练加速与显存优化
+ * 技术解析" §3.2); the dQ contributions of the key tiles are added into the workspace's
+ * fp32 sums with atomic adds, then rounded to 16 bits.  dK and dV are bitwise
+ * reproducible; dQ may differ in its last bits from run to run (the order of the fp32
+ * additions varies).  fa_bwd_deterministic gives bitwise-reproducible dQ as well.
  * o and dout are [B,N,H,d]; workspace must hold fa_bwd_workspace_size bytes and be
  * 256-byte aligned; its contents on entry do not matter. */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -102,16 +110,39 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            float scale, int causal, void* workspace, size_t workspace_bytes, int dtype,
            void* stream);
 
-/* Workspace bytes the varlen backward needs: D [H,total_q] fp32, rounded up to a
- * multiple of 256 bytes. */
+/* Workspace bytes the varlen backward needs: D [H,total_q] fp32 and the fp32 dQ sums
+ * (H x total_q rounded up to 32 x d floats), each rounded up to a multiple of 256 bytes. */
 size_t fa_varlen_bwd_workspace_size(int total_q, int H, int d);
 
-/* Varlen backward; arguments as fa_varlen_fwd plus the gradient buffers. */
+/* Varlen backward; arguments as fa_varlen_fwd plus the gradient buffers.  Computed as
+ * fa_bwd (single pass, atomically added dQ). */
 int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                   const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
                   const int* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k, int H, int d,
                   float scale, int causal, int num_seqs, int total_q, int total_k,
                   void* workspace, size_t workspace_bytes, int dtype, void* stream);
+
+/* Deterministic backward (the pages' deterministic=True mode, page
+ * "FlashAttention实战：如何在A100上实现3倍加速的Transformer训练" §4.2): the same results as
+ * fa_bwd / fa_varlen_bwd within rounding, bitwise reproducible from run to run.  Two
+ * passes instead of one: dK and dV per key tile, then dQ per query tile (each recomputes S
+ * and dP: seven products per tile pair instead of five), so that every gradient element is
+ * written exactly once and no fp32 sum depends on timing.  The window arguments are those
+ * of the _local calls ((-1, 0) causal, (-1, -1) full attention).  workspace: only its
+ * first part (D, B*H*N or H*total_q floats rounded up to 256 bytes) is used; a workspace
+ * sized by fa_bwd_workspace_size / fa_varlen_bwd_workspace_size is more than enough. */
+int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int N, int H, int d, float scale, int window_left, int window_right,
+                         void* workspace, size_t workspace_bytes, int dtype, void* stream);
+
+int fa_varlen_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                const int* cu_seqlens_q, const int* cu_seqlens_k,
+                                int max_seqlen_q, int max_seqlen_k, int H, int d, float scale,
+                                int window_left, int window_right, int num_seqs, int total_q,
+                                int total_k, void* workspace, size_t workspace_bytes, int dtype,
+                                void* stream);
 
 /* ---------------------------------------------------------------- local attention
  * Sliding-window (local) attention: the variant listed by the page "FlashAttention技术
@@ -219,7 +250,8 @@ int fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, voi
                     size_t workspace_bytes, int dtype, void* stream);
 
 /* Allocation-free dense backward (no counterpart on the source pages: an interface
- * addition).  Same arguments and results as fa_bwd, without the workspace: the D vector
+ * addition).  Same arguments as fa_bwd without the workspace, and the results of
+ * fa_bwd_deterministic with the causal window (bitwise): the D vector
  * lives in a fixed array inside the library's device memory (16 MiB, held by every GPU
  * that loads the library until the process exits).  For callers that cannot obtain
  * device memory at call time: hosts whose device memory belongs entirely to another
@@ -270,7 +302,7 @@ int fa_selftest_exp2(const float* x, float* y, int n, void* stream);
 
 /* fa_fwd with O written in fp32 before it is rounded to 16 bits (o: float [B,N,H,d]); lse
  * as fa_fwd.  The same kernel as fa_fwd in a test-only instance, so that a parity test can
- * hold the output to |O - O_ref| <= 1e-2 (the benchmark spec's bound, page
+ * hold the output to the accuracy target |O - O_ref| <= 1e-2 (page
  * "FlashAttention-2的核心设计原理", section "FlashAttention-2与标准注意力的计算对比")
  * where the 16-bit rounding of a large |O| alone can exceed it.  Same arguments and
  * conventions as fa_fwd; o must be 16-byte aligned. */

@@ -48,13 +48,14 @@ def run_fwd(w, rows_per_head=None, pairs=None):
     return o, lse
 
 
-def run_bwd(w, dq_rows=None, dkv_rows=None, pairs=None):
+def run_bwd(w, dq_rows=None, dkv_rows=None, pairs=None, deterministic=False):
     t, (q, k, v, do) = dense_inputs(w)
     B, N, H, d = q.shape
     o, lse = fa.fwd_local(q, k, v, w.window, w.softmax_scale)
     grads = [guarded_empty(q.shape, q.dtype, DEV) for _ in range(3)]
     (dq, gq), (dk, gk), (dv, gv) = grads
-    fa.bwd_local(q, k, v, o, lse, do, w.window, w.softmax_scale, dq=dq, dk=dk, dv=dv)
+    fa.bwd_local(q, k, v, o, lse, do, w.window, w.softmax_scale, dq=dq, dk=dk, dv=dv,
+                 deterministic=deterministic)
     assert fa.device_status() == 0
     assert all(guard_intact(g, q.numel()) for g in (gq, gk, gv))
     dqg, dkg, dvg = f64(dq), f64(dk), f64(dv)
@@ -118,9 +119,13 @@ def test_window_matches_causal_and_full_bitwise():
                                 ((5000, 5000), (on, ln))):
         o, l = fa.fwd_local(q, k, v, win)
         assert torch.equal(o, o_ref) and torch.equal(l, l_ref), win
+    gc = fa.bwd(q, k, v, oc, lc, do, None, True, deterministic=True)
+    gl = fa.bwd_local(q, k, v, oc, lc, do, (-1, 0), deterministic=True)
+    assert all(torch.equal(a, b) for a, b in zip(gc, gl))
+    # single pass: dK and dV are written once per key tile, so they agree bitwise too
     gc = fa.bwd(q, k, v, oc, lc, do, None, True)
     gl = fa.bwd_local(q, k, v, oc, lc, do, (-1, 0))
-    assert all(torch.equal(a, b) for a, b in zip(gc, gl))
+    assert torch.equal(gc[1], gl[1]) and torch.equal(gc[2], gl[2])
     assert fa.device_status() == 0
 
 
@@ -135,12 +140,13 @@ def test_long_local_symmetric_sampled():
 
 
 # ------------------------------------------------------------------ dense backward
+@pytest.mark.parametrize("deterministic", [False, True])
 @pytest.mark.parametrize("window", [(0, 0), (1, 0), (127, 0), (128, 0), (3, 5), (64, 64),
                                     (0, 130), (300, -1), (-1, 40)])
 @pytest.mark.parametrize("d", [64, 128])
-def test_bwd_windows(d, window):
+def test_bwd_windows(d, window, deterministic):
     w = wl.custom("local_bwd", B=1, N=520, H=2, d=d, seed=200 + d, window=window)
-    run_bwd(w)
+    run_bwd(w, deterministic=deterministic)
 
 
 def test_bwd_long_local_sampled():
@@ -150,8 +156,8 @@ def test_bwd_long_local_sampled():
 
 def test_bwd_deterministic():
     w = wl.custom("local_det", B=1, N=600, H=2, d=128, seed=12, window=(150, 30))
-    g1 = run_bwd(w)
-    g2 = run_bwd(w)
+    g1 = run_bwd(w, deterministic=True)
+    g2 = run_bwd(w, deterministic=True)
     assert all(torch.equal(a, b) for a, b in zip(g1, g2))
 
 
@@ -159,10 +165,10 @@ def test_autograd_window():
     w = wl.custom("local_autograd", B=1, N=300, H=2, d=64, seed=13, window=(40, 0))
     t, (q, k, v, do) = dense_inputs(w)
     qq, kk, vv = (x.clone().requires_grad_(True) for x in (q, k, v))
-    out = fa.flash_attn_func(qq, kk, vv, None, False, window=(40, 0))
+    out = fa.flash_attn_func(qq, kk, vv, None, False, window=(40, 0), deterministic=True)
     out.backward(do)
     o, lse = fa.fwd_local(q, k, v, (40, 0))
-    dq, dk, dv = fa.bwd_local(q, k, v, o, lse, do, (40, 0))
+    dq, dk, dv = fa.bwd_local(q, k, v, o, lse, do, (40, 0), deterministic=True)
     assert torch.equal(out.detach(), o)
     assert torch.equal(qq.grad, dq) and torch.equal(kk.grad, dk) and torch.equal(vv.grad, dv)
 

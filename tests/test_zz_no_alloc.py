@@ -6,14 +6,14 @@ cudaMalloc and its implicit synchronisation is not acceptable inside their loop.
 fa_bwd_noalloc serves them: it is fa_bwd with its D scratch in a fixed array inside the
 library instead of a caller workspace.
 
-The test calls it through the C ABI twice in a row with different shapes — first a larger
+The test calls it through the C ABI twice in a row with different shapes (first a larger
 non-causal problem, so that the shared array holds stale values, then a smaller causal one
-with another head_dim — and checks each call against fa_bwd (the workspace entry point,
-same kernels: bitwise equal) and the second call against the fp64 oracle's analytic
-gradients on sampled rows, max |dX - dX_ref| <= 2e-2 * max |dX_ref|.  It also checks the
-capacity edge: B*H*N = 4194304 is accepted (and equals fa_bwd), one more is refused.  The
-file sorts last so that a run which stops at its first failure has already run every other
-test.
+with another head_dim) and checks each call against fa_bwd_deterministic, the workspace
+entry point that runs the same kernels (bitwise equal), and the second call against the
+fp64 oracle's analytic gradients on sampled rows, max |dX - dX_ref| <= 2e-2 * max |dX_ref|.
+It also checks the capacity edge: B*H*N = 4194304 is accepted (and equals
+fa_bwd_deterministic), one more is refused.  The file sorts last so that a run which stops
+at its first failure has already run every other test.
 """
 
 import numpy as np
@@ -55,9 +55,9 @@ def test_noalloc_backward_two_calls_against_workspace_backward_and_oracle():
     for call, w in enumerate(shapes):
         t, q, k, v, do, o, lse = _inputs(w)
         got = _noalloc(lib, q, k, v, o, lse, do, w.softmax_scale, w.causal)
-        ref = fa.bwd(q, k, v, o, lse, do, w.softmax_scale, w.causal)
+        ref = fa.bwd(q, k, v, o, lse, do, w.softmax_scale, w.causal, deterministic=True)
         for name, g, r in zip(("dQ", "dK", "dV"), got, ref):
-            assert torch.equal(g, r), f"{name} call {call} differs from fa_bwd"
+            assert torch.equal(g, r), f"{name} call {call} differs from fa_bwd_deterministic"
     # the second call (after the larger one left its values in the shared array) against
     # the oracle on sampled rows of every head
     qf, kf, vf, dof = (wl.to_f64(t[x]) for x in ("q", "k", "v", "do"))
@@ -78,9 +78,9 @@ def test_noalloc_capacity_edge():
     w = wl.custom("noalloc_edge", B=64, N=1024, H=64, d=64, causal=True, seed=33)
     t, q, k, v, do, o, lse = _inputs(w)
     got = _noalloc(lib, q, k, v, o, lse, do, w.softmax_scale, True)
-    ref = fa.bwd(q, k, v, o, lse, do, w.softmax_scale, True)
+    ref = fa.bwd(q, k, v, o, lse, do, w.softmax_scale, True, deterministic=True)
     for name, g, r in zip(("dQ", "dK", "dV"), got, ref):
-        assert torch.equal(g, r), f"{name} at the capacity edge differs from fa_bwd"
+        assert torch.equal(g, r), f"{name} at the capacity edge differs from fa_bwd_deterministic"
     qf, kf, vf, dof = (wl.to_f64(t[x]) for x in ("q", "k", "v", "do"))
     for (b, h) in [(0, 0), (63, 63)]:  # the first and the last D slot of the array
         gq, gk, gv = oracle.attention_backward(qf[b, :, h], kf[b, :, h], vf[b, :, h],
