@@ -405,8 +405,9 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // exponentials bypass the special-function unit.  Method: Cody–Waite range reduction,
 // x = j + f with j = rint(x) obtained by the 1.5·2^23 shift (round to nearest) and
 // f in [-0.5, 0.5]; 2^f by a degree-3 polynomial whose coefficients were fitted for this
-// library (minimax relative error on [-0.5, 0.5] by Lawson-weighted least squares; max
-// relative error 7.5e-5); 2^j by adding j to the exponent field.  Inputs below -126 are
+// library (minimax relative error on [-0.5, 0.5] by the Remez exchange algorithm in
+// exp2_poly_fit.py beside this file, rounded to float32; max relative error 7.5e-5); 2^j by
+// adding j to the exponent field.  Inputs below -126 are
 // clamped to -126; below about -125 results approach the denormal range (~1e-38) and lose
 // relative accuracy, and they are never exactly 0: do not use it where an exact 0 is
 // required (masked keys).
@@ -418,7 +419,7 @@ __device__ __forceinline__ float2 exp2_poly2(float a, float b) {
   const uint64_t j = f2_add(t, f2_pack(-12582912.f, -12582912.f));  // j (exact)
   const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x);             // f = x - j
   uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
-                      f2_pack(0.2426111400127411f, 0.2426111400127411f));
+                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
   p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
   p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
   const float2 pf = f2_unpack(p), tf = f2_unpack(t);

@@ -54,3 +54,16 @@ def test_whole_function_in_float32():
     y = bits.astype(np.uint32).view(np.float32).astype(np.float64)
     rel = np.abs(y / np.exp2(x.astype(np.float64)) - 1.0)
     assert rel.max() <= 1e-4, (rel.max(), x[rel.argmax()])
+
+
+def test_header_constants_are_the_committed_fit():
+    # the four constants in the kernel header are exactly the float32 output of the
+    # committed Remez fit (exp2_poly_fit.py beside the header)
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "exp2_poly_fit", os.path.join(os.path.dirname(HEADER), "exp2_poly_fit.py"))
+    fit = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(fit)
+    assert [float(c) for c in _coefficients()] == fit.float32_coefficients()
+    assert fit.max_rel_error(fit.float32_coefficients()) <= 7.5e-5
+
