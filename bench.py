@@ -71,6 +71,30 @@ def throughput_tflops(flops_per_step_per_rank: float, steps: int, world: int,
     return flops_per_step_per_rank * steps * world / max_seconds / 1e12
 
 
+def head_range(H: int, rank: int, world: int):
+    """Heads [h0, h1) of `rank` in the head split of the pages' tensor-parallel attention
+    (page "FlashAttention-2的核心设计原理", section "FlashAttention-2反向传播与多GPU训练"):
+    H / world consecutive heads per rank, rank r holding heads r*H/world .. (r+1)*H/world - 1."""
+    if world <= 0 or H % world != 0:
+        raise ValueError(f"H = {H} heads do not split evenly over {world} ranks")
+    per = H // world
+    return rank * per, (rank + 1) * per
+
+
+def gather_heads(local, world: int):
+    """All-gather every rank's [B, N, H/world, d] output and join them along the head
+    dimension (rank order = head order): the full [B, N, H, d] result on every rank."""
+    if world == 1:
+        return local
+    import torch
+    import torch.distributed as dist
+    B, N, Hl, d = local.shape
+    parts = torch.empty((world * B, N, Hl, d), dtype=local.dtype, device=local.device)
+    dist.all_gather_into_tensor(parts, local.contiguous())
+    # [world * B, N, Hl, d] -> [world, B, N, Hl, d] -> [B, N, world, Hl, d] -> [B, N, H, d]
+    return parts.view(world, B, N, Hl, d).permute(1, 2, 0, 3, 4).reshape(B, N, world * Hl, d)
+
+
 def sources_sha(paths) -> str:
     """Hash of the kernel sources without their // comments and blank lines, so that the
     recorded DRAM traffic of a kernel stays attached to it until its code changes."""
@@ -422,10 +446,20 @@ def run_fattn(args, w):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     lib = _lib.load()
-    # each rank owns an independent problem of the same size (its own seed)
-    wr = wl.Workload(**{**w.__dict__, "seed": w.seed + rank})
-    host = wl.generate(wr)
-    B, N, H, d = wr.B, wr.N, wr.H, wr.d
+    split_heads = getattr(args, "split", "none") == "heads"
+    if split_heads:
+        # one shared problem (same seed on every rank), its heads split over the ranks; each
+        # step ends with an all-gather of O along the head dimension
+        wr = w
+        h0, h1 = head_range(w.H, rank, world)
+        full = wl.generate(wr)
+        host = {x: full[x][:, :, h0:h1].contiguous() for x in ("q", "k", "v", "do")}
+        del full
+    else:
+        # each rank owns an independent problem of the same size (its own seed)
+        wr = wl.Workload(**{**w.__dict__, "seed": w.seed + rank})
+        host = wl.generate(wr)
+    B, N, H, d = wr.B, wr.N, host["q"].shape[2], wr.d
     scale, causal = wr.softmax_scale, int(wr.causal)
     dtype = _lib.FA_BF16 if wr.dtype == "bf16" else _lib.FA_FP16
     q, k, v, do = (host[x].to(dev) for x in ("q", "k", "v", "do"))
@@ -458,9 +492,13 @@ def run_fattn(args, w):
                                         wr.window[0], wr.window[1], ws.data_ptr(), ws.numel(),
                                         dtype, sh), "fa_bwd_local")
 
+    o_full = [None]
+
     def step():
         launch_fwd()
         launch_bwd()
+        if split_heads:
+            o_full[0] = gather_heads(o, world)
 
     for _ in range(args.warmup):
         step()
@@ -483,6 +521,8 @@ def run_fattn(args, w):
         ev[i][1].record(stream)
         launch_bwd()
         ev[i][2].record(stream)
+        if split_heads:
+            o_full[0] = gather_heads(o, world)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
@@ -494,7 +534,7 @@ def run_fattn(args, w):
     fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
     bwd_ms = [b.elapsed_time(c) for _, b, c in ev]
     max_s = max_over_ranks(total_ms / 1e3, world)
-    f_fwd = wr.fwd_flops()
+    f_fwd = wr.fwd_flops() * H / wr.H   # this rank's share (all of it unless heads are split)
     f_step = 3.5 * f_fwd
     value = throughput_tflops(f_step, args.steps, world, max_s)
     fwd_avg = statistics.mean(fwd_ms)
@@ -525,7 +565,7 @@ def run_fattn(args, w):
     # overlap the compute of the previous / next step (H2D and D2H also run concurrently),
     # as a training loop that feeds a GPU from host memory would.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not split_heads:
         hin = [host[x].pin_memory() for x in ("q", "k", "v", "do")]
         sets = []
         for bset in range(2):
@@ -648,8 +688,11 @@ def run_fattn(args, w):
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": 1e3 * max_s / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": wr.dtype, "data": "synthetic",
-                "config": dict(wr.describe(), seed=w.seed, parallelism=f"dp{world}",
+                "scaling": "strong" if split_heads else "weak", "vs_baseline": None,
+                "dtype": wr.dtype, "data": "synthetic",
+                "config": dict(wr.describe(), seed=w.seed,
+                               parallelism=(f"heads{world} (head split, all-gather of O)"
+                                            if split_heads else f"dp{world}"),
                                l2="inputs larger than L2 (268 MB per tensor), no flush"),
                 "fwd_tflops": f_fwd / (fwd_avg / 1e3) / 1e12,
                 "bwd_tflops": bwd_ach,
@@ -1073,6 +1116,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the small-shape sweep of the default bench line")
+    ap.add_argument("--split", default="none", choices=["none", "heads"],
+                    help="heads: one shared problem with its heads split over the ranks and O "
+                         "all-gathered every step (strong scaling); none: one independent "
+                         "problem per rank (weak scaling)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3) if args.impl == "fattn" else args.warmup
     from exact_tiled_attention_33_b200 import workloads as wl

@@ -49,3 +49,43 @@ def test_two_rank_max_and_throughput():
 def test_single_rank_identity():
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.throughput_tflops(1e12, 10, 1, 2.0) == 5.0
+
+
+# ------------------------------------------------------------------ head split
+def _split_worker(rank, world, port, out):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        B, N, H, d = 2, 5, 8, 3
+        # a stand-in "output" whose every element names its (b, n, h, c) position
+        full = torch.arange(B * N * H * d, dtype=torch.float32).reshape(B, N, H, d)
+        h0, h1 = bench.head_range(H, rank, world)
+        local = full[:, :, h0:h1].contiguous() * 1.0   # what this rank's attention produced
+        out[rank] = (h0, h1, bool(torch.equal(bench.gather_heads(local, world), full)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_head_split_and_gather_order():
+    # the head partition covers every head once, in rank order, and the all-gather of the
+    # ranks' outputs rebuilds the full [B, N, H, d] tensor on every rank
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_split_worker, args=(2, port, out), nprocs=2, join=True,
+                       start_method="spawn")
+    assert [out[r][:2] for r in range(2)] == [(0, 4), (4, 8)]
+    assert out[0][2] and out[1][2]
+
+
+def test_head_range_rejects_uneven_splits():
+    import pytest
+    assert bench.head_range(32, 7, 8) == (28, 32)
+    with pytest.raises(ValueError):
+        bench.head_range(32, 0, 3)
