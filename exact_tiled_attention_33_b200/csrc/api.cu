@@ -221,7 +221,7 @@ int fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.reverse_tiles = reverse_tiles(wl, wr);
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-  const int rows = fwd_rows_per_cta();
+  const int rows = fwd_rows_per_cta(false);
   dim3 grid((N + rows - 1) / rows, H, B);
   return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
 }
@@ -266,7 +266,7 @@ int fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
   p.reverse_tiles = reverse_tiles(wl, wr);
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-  const int rows = fwd_rows_per_cta();
+  const int rows = fwd_rows_per_cta(false);
   dim3 grid((max_seqlen_q + rows - 1) / rows, H, num_seqs);
   return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
 }
@@ -389,7 +389,7 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
   p.reverse_tiles = reverse_tiles(p.win_left, p.win_right);
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-  const int rows = fwd_rows_per_cta();
+  const int rows = fwd_rows_per_cta(true);
   dim3 grid((N + rows - 1) / rows, H, B);
   return launch_result(
       launch_fwd_fp8(d, out_dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
@@ -435,7 +435,7 @@ int fa_varlen_fwd_fp8(const void* q, const void* k, const void* v, void* o, floa
   p.reverse_tiles = reverse_tiles(p.win_left, p.win_right);
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-  const int rows = fwd_rows_per_cta();
+  const int rows = fwd_rows_per_cta(true);
   dim3 grid((max_seqlen_q + rows - 1) / rows, H, num_seqs);
   return launch_result(
       launch_fwd_fp8(d, out_dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
@@ -871,7 +871,7 @@ int fa_selftest_fwd_f32(const void* q, const void* k, const void* v, float* o, f
   p.reverse_tiles = reverse_tiles(p.win_left, p.win_right);
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-  const int rows = fwd_rows_per_cta();
+  const int rows = fwd_rows_per_cta(false);
   dim3 grid((N + rows - 1) / rows, H, B);
   return launch_result(
       launch_fwd_f32out(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));

@@ -141,8 +141,9 @@ LaunchResult launch_fwd_f32out(int d, bool bf16, const CUtensorMap& tmQ, const C
                                const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
                                cudaStream_t stream);
 
-// Forward grid: x = query-tile pairs, y = heads, z = batch (dense) or sequences (varlen).
-int fwd_rows_per_cta();
+// Query rows per forward CTA (grid x = ceil(rows / this), y = heads, z = batch or
+// sequences): two 128-row tiles for 16-bit operands, one for FP8.
+int fwd_rows_per_cta(bool fp8);
 
 // Decode launch: the split kernel and, when p.splits > 1, the merge kernel.
 LaunchResult launch_decode(int d, bool bf16, bool paged, const CUtensorMap& tmK,
