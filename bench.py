@@ -41,6 +41,9 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
 BWD_SOURCES = ["exact_tiled_attention_33_b200/csrc/bwd_fused_kernel.cuh",
                "exact_tiled_attention_33_b200/csrc/sm100.cuh",
                "exact_tiled_attention_33_b200/csrc/fattn_internal.h"]
+FP8_SOURCES = ["exact_tiled_attention_33_b200/csrc/fwd_kernel.cuh",
+               "exact_tiled_attention_33_b200/csrc/sm100.cuh",
+               "exact_tiled_attention_33_b200/csrc/fattn_internal.h"]
 BWD_KERNEL_DESC = ("fa_bwd (D preprocess + single-pass dK/dV/dQ kernel + dQ conversion, timed "
                    "as one call)")
 FWD_SOURCES = ["exact_tiled_attention_33_b200/csrc/fwd2_kernel.cuh",
@@ -900,7 +903,7 @@ def run_fp8(args, w):
     # no measured FP8 peak: the measured bf16 figure times the nominal FP8/BF16 ratio (2)
     peak_b, peak_s = 2 * burst, 2 * sust
     ach = f / per / 1e12
-    sha = sources_sha(FWD_SOURCES)
+    sha = sources_sha(FP8_SOURCES)
     roofline = {"kernel": "fa_fwd_kernel<128, bf16 out, fp8>", "bound": "tensor",
                 "achieved": ach, "peak": peak_s, "unit": "TFLOP/s", "frac": ach / peak_s,
                 "frac_of_burst_peak": ach / peak_b,
