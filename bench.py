@@ -434,6 +434,69 @@ def sweep_small_n(lib, dev):
 
 
 # ------------------------------------------------------------------ GPU arm
+def other_arms(lib, dev, reps=10):
+    """The NEXT rows' workloads timed inside the default bench run, so that its line carries
+    them: the FP8 forward on the long causal shape (TFLOPS), one KV-cache decode step over
+    8 x 16384 cached tokens (GB/s of K/V read), and the causal 4096-key window on the long
+    shape (fwd + bwd TFLOPS).  Each launch alone with CUDA events on the launching stream,
+    L2 flushed before it (a 256 MB write); median of `reps`."""
+    import torch
+    from exact_tiled_attention_33_b200 import _lib
+    from exact_tiled_attention_33_b200 import attention as fa
+    from exact_tiled_attention_33_b200 import workloads as wl
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    # FP8 forward
+    w = wl.get("fp8_long_causal")
+    t = wl.generate(w, with_grad_out=False)
+    q8, k8, v8 = (t[x].to(dev) for x in ("q8", "k8", "v8"))
+    sq, sk, sv = t["q_descale"], t["k_descale"], t["v_descale"]
+    del t
+    o8, l8 = fa.fwd_fp8(q8, k8, v8, sq, sk, sv, w.softmax_scale, w.causal)
+    tf = _timed(lambda: fa.fwd_fp8(q8, k8, v8, sq, sk, sv, w.softmax_scale, w.causal, out=o8,
+                                   lse=l8), stream, dev, flush, reps)
+    out["fp8_long_causal_fwd"] = {"ms": tf["median"], "tflops": w.fwd_flops() / tf["median"] / 1e9,
+                                  "unit": "TFLOPS", "reps": reps}
+    del q8, k8, v8, o8, l8
+    # KV-cache decode, one new token per sequence
+    dw = wl.get_decode("decode_b8_l16k")
+    g = wl.generate_decode(dw)
+    q, kc, vc = g["q"].to(dev), g["k_cache"].to(dev), g["v_cache"].to(dev)
+    lens = g["cache_seqlens"].to(dev)
+    del g
+    max_len = max(dw.cache_lens)
+    od = torch.empty_like(q)
+    ld = torch.empty((q.shape[0], q.shape[2], q.shape[1]), dtype=torch.float32, device=dev)
+    wsd = fa.decode_workspace(q.shape[0], q.shape[1], q.shape[2], q.shape[3], max_len, dev)
+    td = _timed(lambda: fa.decode(q, kc, vc, lens, max_len, dw.softmax_scale, dw.causal, out=od,
+                                  lse=ld, workspace=wsd), stream, dev, flush, 5 * reps)
+    out["decode_b8_l16k"] = {"us": 1e3 * td["median"],
+                             "gbs": dw.bytes_moved() / td["median"] / 1e6, "unit": "GB/s",
+                             "reps": 5 * reps}
+    del q, kc, vc, od, ld, wsd
+    # sliding window (4095, 0) on the long shape
+    w = wl.get("long_local_w4096")
+    t = wl.generate(w)
+    q, k, v, do = (t[x].to(dev) for x in ("q", "k", "v", "do"))
+    del t
+    o, lse = fa.fwd_local(q, k, v, w.window, w.softmax_scale)
+    ws = fa.bwd_workspace(w.B, w.N, w.H, w.d, dev)
+    tf = _timed(lambda: fa.fwd_local(q, k, v, w.window, w.softmax_scale, out=o, lse=lse), stream,
+                dev, flush, reps)
+    tb = _timed(lambda: fa.bwd_local(q, k, v, o, lse, do, w.window, w.softmax_scale,
+                                     workspace=ws), stream, dev, flush, reps)
+    f = w.fwd_flops()
+    out["long_local_w4096"] = {"fwd_ms": tf["median"], "bwd_ms": tb["median"],
+                               "fwd_tflops": f / tf["median"] / 1e9,
+                               "fwd_bwd_tflops": 3.5 * f / (tf["median"] + tb["median"]) / 1e9,
+                               "unit": "TFLOPS", "reps": reps}
+    assert lib.fa_get_device_status(stream.cuda_stream) == 0
+    del q, k, v, do, o, lse, ws, flush
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_fattn(args, w):
     import torch
     import torch.distributed as dist
@@ -670,6 +733,9 @@ def run_fattn(args, w):
     sweep = None
     if rank == 0 and world == 1 and not args.no_sweep:
         sweep = sweep_small_n(lib, dev)
+    arms = None
+    if rank == 0 and world == 1 and not args.no_other_arms:
+        arms = other_arms(lib, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -706,7 +772,8 @@ def run_fattn(args, w):
                 "ms_fwd": fwd_avg, "ms_bwd": bwd_avg,
                 "gpu_launches": 4 * args.steps,
                 "roofline": roofline, "roofline_fwd": fwd_roof, "fwd_only": fwd_only,
-                "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "sweep_small_n": sweep}
+                "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "sweep_small_n": sweep,
+                "other_arms": arms}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -1120,6 +1187,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the small-shape sweep of the default bench line")
+    ap.add_argument("--no-other-arms", action="store_true",
+                    help="skip the FP8, decode and window timings of the default bench line")
     ap.add_argument("--split", default="none", choices=["none", "heads"],
                     help="heads: one shared problem with its heads split over the ranks and O "
                          "all-gathered every step (strong scaling); none: one independent "
