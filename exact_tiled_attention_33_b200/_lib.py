@@ -58,7 +58,7 @@ SIGNATURES = {
     "fa_last_error": (ctypes.c_char_p, []),
     "fa_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "fa_selftest_exp2": (_i, [_vp, _vp, _i, _vp]),
-    "fa_selftest_fwd_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]),
+    "fa_selftest_fwd_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _i, _vp]),
 }
 
 _LIB = None

@@ -64,9 +64,9 @@ def fwd(q, k, v, softmax_scale=None, causal=False, out=None, lse=None):
     return o, lse_t
 
 
-def fwd_f32out(q, k, v, softmax_scale=None, causal=False):
-    """Test hook: fa_fwd with O returned in fp32 before rounding (fa_selftest_fwd_f32).
-    Returns (o [B,N,H,d] fp32, lse [B,H,N] fp32)."""
+def fwd_f32out(q, k, v, softmax_scale=None, causal=False, window=None):
+    """Test hook: fa_fwd (window None) or fa_fwd_local with O returned in fp32 before
+    rounding (fa_selftest_fwd_f32).  Returns (o [B,N,H,d] fp32, lse [B,H,N] fp32)."""
     if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v must all be [B, N, H, d] with equal shapes")
     dtype = _check(q, k, v)
@@ -76,8 +76,9 @@ def fwd_f32out(q, k, v, softmax_scale=None, causal=False):
     lse_t = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
     lib = _lib.load()
     with torch.cuda.device(q.device):
+        wl, wr = (-1, 0 if causal else -1) if window is None else _window(window)
         st = lib.fa_selftest_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, N, H,
-                                     d, scale, int(bool(causal)), dtype, _stream(q))
+                                     d, scale, wl, wr, dtype, _stream(q))
     _lib.check(st, "fa_selftest_fwd_f32")
     return o, lse_t
 

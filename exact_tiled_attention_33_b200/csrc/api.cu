@@ -219,6 +219,7 @@ int fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.win_left = wl;
   p.win_right = wr;
   p.reverse_tiles = reverse_tiles(wl, wr);
+  p.max_seqlen_q = N;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   const int rows = fwd_rows_per_cta(false);
@@ -264,6 +265,7 @@ int fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
   p.win_left = wl;
   p.win_right = wr;
   p.reverse_tiles = reverse_tiles(wl, wr);
+  p.max_seqlen_q = max_seqlen_q;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   const int rows = fwd_rows_per_cta(false);
@@ -387,6 +389,7 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
   p.win_left = -1;
   p.win_right = causal ? 0 : -1;
   p.reverse_tiles = reverse_tiles(p.win_left, p.win_right);
+  p.max_seqlen_q = N;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   const int rows = fwd_rows_per_cta(true);
@@ -433,6 +436,7 @@ int fa_varlen_fwd_fp8(const void* q, const void* k, const void* v, void* o, floa
   p.win_left = -1;
   p.win_right = causal ? 0 : -1;
   p.reverse_tiles = reverse_tiles(p.win_left, p.win_right);
+  p.max_seqlen_q = max_seqlen_q;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   const int rows = fwd_rows_per_cta(true);
@@ -503,6 +507,8 @@ int bwd_common(const void* q, const void* k, const void* v, const void* o, const
   p.win_left = wl;
   p.win_right = wr;
   p.reverse_tiles = reverse_tiles(wl, wr);
+  p.max_seqlen_q = max_seqlen_q;
+  p.max_seqlen_k = max_seqlen_k;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   if (single_pass)
@@ -846,13 +852,16 @@ int fa_selftest_exp2(const float* x, float* y, int n, void* stream) {
 }
 
 int fa_selftest_fwd_f32(const void* q, const void* k, const void* v, float* o, float* lse, int B,
-                        int N, int H, int d, float scale, int causal, int dtype, void* stream) {
+                        int N, int H, int d, float scale, int window_left, int window_right,
+                        int dtype, void* stream) {
   g_last_error.clear();
   if (int e = check_common(H, d, dtype, scale)) return e;
   if (B < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "B and N must be >= 0");
   if ((long long)B * N >= (1LL << 31)) return fail(FA_ERR_UNSUPPORTED, "B*N must be < 2^31");
   if (B == 0 || N == 0 || H == 0) return FA_OK;
   if (int e = check_grid(B, H, N)) return e;
+  int wl = window_left, wr = window_right;
+  if (int e = normalize_window(&wl, &wr, N, N)) return e;
   if (int e = check_ptrs({q, k, v, o, lse})) return e;
   CUtensorMap mq, mk, mv;
   if (int e = make_map(&mq, q, d, H, N, B, 128)) return e;
@@ -866,9 +875,10 @@ int fa_selftest_fwd_f32(const void* q, const void* k, const void* v, float* o, f
   p.total_q = B * N;
   p.scale = scale;
   set_fwd_scale(p, scale);
-  p.win_left = -1;
-  p.win_right = causal ? 0 : -1;
-  p.reverse_tiles = reverse_tiles(p.win_left, p.win_right);
+  p.win_left = wl;
+  p.win_right = wr;
+  p.reverse_tiles = reverse_tiles(wl, wr);
+  p.max_seqlen_q = N;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   const int rows = fwd_rows_per_cta(false);

@@ -163,8 +163,8 @@ __global__ void __launch_bounds__(384, 1)
   const int bz = blockIdx.z;
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
-    if (!varlen_segment_ok(p.cu_q, p.cu_k, bz, p.total_q, p.total_k, -1,
-                           (long long)gridDim.x * BN, p.status))
+    if (!varlen_segment_ok(p.cu_q, p.cu_k, bz, p.total_q, p.total_k, -1, p.max_seqlen_k,
+                           p.status))
       return;
     q_row0 = p.cu_q[bz];
     Lq = p.cu_q[bz + 1] - q_row0;
@@ -489,8 +489,8 @@ __global__ void __launch_bounds__(384, 1)
   const int bz = blockIdx.z;
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
-    if (!varlen_segment_ok(p.cu_q, p.cu_k, bz, p.total_q, p.total_k, (long long)gridDim.x * BM,
-                           -1, p.status))
+    if (!varlen_segment_ok(p.cu_q, p.cu_k, bz, p.total_q, p.total_k, p.max_seqlen_q, -1,
+                           p.status))
       return;
     q_row0 = p.cu_q[bz];
     Lq = p.cu_q[bz + 1] - q_row0;

@@ -27,6 +27,7 @@ struct FwdParams {
   int win_left;     // attention window (see key_tile_range); causal is (-1, 0)
   int win_right;
   int reverse_tiles;// launch the query tiles with the most key tiles first
+  int max_seqlen_q; // varlen: longest allowed segment (longer ones are skipped, reported)
   uint32_t* status; // device status word
 };
 
@@ -53,6 +54,7 @@ struct BwdParams {
   float scale_log2;
   int win_left, win_right;  // attention window (see key_tile_range)
   int reverse_tiles;        // dQ pass: launch the query tiles with the most key tiles first
+  int max_seqlen_q, max_seqlen_k;  // varlen: longest allowed segments (longer: skipped, reported)
   uint32_t* status;
 };
 

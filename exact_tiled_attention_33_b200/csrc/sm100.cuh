@@ -25,8 +25,8 @@ enum : uint32_t {
 
 // Varlen segment bz read from device prefix sums, checked before any use: rows
 // [cu_q[bz], cu_q[bz+1]) must lie in [0, total_q) and keys likewise in [0, total_k), and the
-// segment must fit the rows (q_cover) or keys (k_cover) the grid covers (negative: not
-// checked).  A bad segment is reported in the status word and its CTA does nothing, so a
+// segment may hold at most q_cover rows and k_cover keys (the caller's max_seqlen_q /
+// max_seqlen_k, which size the grid; negative: not checked).  A bad segment is reported in the status word and its CTA does nothing, so a
 // malformed cu_seqlens never leads to an out-of-bounds access.
 __device__ __forceinline__ bool varlen_segment_ok(const int* cu_q, const int* cu_k, int bz,
                                                   int total_q, int total_k, long long q_cover,

@@ -300,15 +300,16 @@ int fa_selftest_wait_timeout(unsigned int limit_us, void* stream);
  * A self-test hook with no counterpart on the pages. */
 int fa_selftest_exp2(const float* x, float* y, int n, void* stream);
 
-/* fa_fwd with O written in fp32 before it is rounded to 16 bits (o: float [B,N,H,d]); lse
- * as fa_fwd.  The same kernel as fa_fwd in a test-only instance, so that a parity test can
- * hold the output to the accuracy target |O - O_ref| <= 1e-2 (page
- * "FlashAttention-2的核心设计原理", section "FlashAttention-2与标准注意力的计算对比")
- * where the 16-bit rounding of a large |O| alone can exceed it.  Same arguments and
- * conventions as fa_fwd; o must be 16-byte aligned. */
+/* fa_fwd_local with O written in fp32 before it is rounded to 16 bits (o: float
+ * [B,N,H,d]); lse as fa_fwd.  The same kernel as fa_fwd / fa_fwd_local in a test-only
+ * instance, so that a parity test can hold the output to the accuracy target
+ * |O - O_ref| <= 1e-2 (page "FlashAttention-2的核心设计原理", section
+ * "FlashAttention-2与标准注意力的计算对比") where the 16-bit rounding of a large |O| alone can
+ * exceed it.  Window (-1, 0) is causal, (-1, -1) full attention; other arguments and
+ * conventions as fa_fwd_local; o must be 16-byte aligned. */
 int fa_selftest_fwd_f32(const void* q, const void* k, const void* v, float* o, float* lse,
-                        int B, int N, int H, int d, float scale, int causal, int dtype,
-                        void* stream);
+                        int B, int N, int H, int d, float scale, int window_left,
+                        int window_right, int dtype, void* stream);
 
 #ifdef __cplusplus
 }

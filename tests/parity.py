@@ -3,12 +3,15 @@
 Tolerances are the ones the target fixes for 16-bit inputs with fp32 accumulation:
   max |O - O_ref| <= 1e-2, max |LSE - LSE_ref| <= 1e-3,
   max |dX - dX_ref| <= 2e-2 * max |dX_ref| for dX in dQ, dK, dV.
-O is checked against the literal 1e-2 everywhere except on the peaky workloads (Q and K
-scaled by 4, so that each softmax row is nearly one-hot and |O| reaches ~5): there a
-correctly rounded 16-bit output can sit half a 16-bit ulp (up to 2^-6 at |O| in [4, 8))
-from the fp64 value, which alone exceeds 1e-2, so the stored output is allowed 1e-2 plus
-half an ulp of the output format at O_ref.  For those workloads the literal 1e-2 is
-applied instead to the kernel's fp32 output before rounding (fa_selftest_fwd_f32).
+The stored 16-bit O is checked against the literal 1e-2 everywhere except where |O| itself
+is large: the peaky workloads (Q and K scaled by 4, each softmax row nearly one-hot, |O| up
+to ~5), rows that see one or two keys (a window of width <= 1: O is one value or the mix of
+two, |O| up to ~4) and inputs shifted to make |O| ~ 2.  A correctly rounded bf16 output can
+sit half an ulp from the fp64 value (2^-8 for |O| in [2, 4), 2^-7 in [4, 8)), which alone
+approaches or exceeds 1e-2, so there the stored output is allowed 1e-2 plus half an ulp of
+the output format at O_ref (rounding_allowance=True), and those tests apply the literal 1e-2
+to the kernel's fp32 output before rounding (fa_selftest_fwd_f32) wherever the call has
+such an instance (dense, causal, windowed).
 
 Every check records its maximum error; when FATTN_PARITY_JSON names a file, the whole
 session's records are written there (tests/conftest.py).
@@ -44,15 +47,15 @@ def half_ulp(x: np.ndarray, dtype: str) -> np.ndarray:
 
 
 def check_o(o_gpu: np.ndarray, o_ref: np.ndarray, dtype: str, what: str = "O",
-            peaky: bool = False) -> float:
-    """max |O - O_ref| <= 1e-2; with peaky=True (Q,K x4 workloads only) the stored 16-bit
-    output may add half a 16-bit ulp at O_ref."""
+            rounding_allowance: bool = False) -> float:
+    """max |O - O_ref| <= 1e-2; with rounding_allowance=True (large-|O| cases only, see the
+    module docstring) the stored 16-bit output may add half a 16-bit ulp at O_ref."""
     err = np.abs(o_gpu.astype(np.float64) - o_ref)
     assert np.all(np.isfinite(o_gpu)), f"{what}: non-finite output"
-    allowed = O_TOL + half_ulp(o_ref, dtype) if peaky else O_TOL
+    allowed = O_TOL + half_ulp(o_ref, dtype) if rounding_allowance else O_TOL
     bad = err > allowed
     m = float(err.max()) if err.size else 0.0
-    _record(what, m, O_TOL, "O (peaky: + half ulp)" if peaky else "O")
+    _record(what, m, O_TOL, "O (+ half ulp of the output)" if rounding_allowance else "O")
     assert not bad.any(), (f"{what}: {int(bad.sum())} elements over tolerance; max err "
                            f"{m:.4g}")
     return m

@@ -41,7 +41,7 @@ def run_dense(w, rows_per_head=None, bh_subset=None):
                                                   w.softmax_scale, w.causal, rows=rows)
         sel = slice(None) if rows is None else rows
         eo = max(eo, check_o(og[b, sel, h], o_ref, w.dtype, f"O[b={b},h={h}]",
-                             peaky=is_peaky(w)))
+                             rounding_allowance=is_peaky(w)))
         el = max(el, check_lse(lg[b, h, sel], lse_ref, f"LSE[b={b},h={h}]"))
     return eo, el, o, lse
 
@@ -153,7 +153,9 @@ def run_varlen(lens_q, lens_k, H, d, causal, dtype="bf16", seed=3, scale=None, p
     assert guard_intact(obuf, o.numel()) and guard_intact(lbuf, lse.numel())
     o_ref, lse_ref = oracle.varlen_attention_forward(wl.to_f64(q), wl.to_f64(k), wl.to_f64(v),
                                                      cu_q, cu_k, w.softmax_scale, causal)
-    check_o(f64(o), o_ref, dtype)
+    # the perturbed inputs of the isolation test shift one segment's V by -2 (|O| ~ 2, where
+    # half a bf16 ulp is 2^-8): the stored output gets the output-rounding allowance there
+    check_o(f64(o), o_ref, dtype, rounding_allowance=perturb is not None)
     check_lse(f64(lse), lse_ref)
     return o, lse, cu_q
 
