@@ -21,7 +21,7 @@ def pytest_sessionfinish(session, exitstatus):
     worst = {}
     for r in parity.RECORDS:
         key = (r["test"], r["kind"])
-        if key not in worst or r["max_err"] > worst[key]["max_err"]:
+        if key not in worst or r["frac_of_bound"] > worst[key]["frac_of_bound"]:
             worst[key] = r
     summary = sorted(worst.values(), key=lambda r: (r["test"], r["kind"]))
     os.makedirs(os.path.dirname(os.path.abspath(path)), exist_ok=True)

@@ -32,10 +32,12 @@ GRAD_REL_TOL = 2e-2
 RECORDS: list = []
 
 
-def _record(what: str, err: float, bound: float, kind: str) -> None:
+def _record(what: str, err: float, bound: float, kind: str, frac: float) -> None:
+    """err: the check's maximum error (gradients: as a fraction of max|ref|); bound: the
+    tolerance it is held to; frac: the largest error / allowed ratio over the elements."""
     test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
     RECORDS.append({"test": test, "what": what, "kind": kind, "max_err": float(err),
-                    "bound": float(bound)})
+                    "bound": float(bound), "frac_of_bound": float(frac)})
 
 
 def half_ulp(x: np.ndarray, dtype: str) -> np.ndarray:
@@ -55,7 +57,8 @@ def check_o(o_gpu: np.ndarray, o_ref: np.ndarray, dtype: str, what: str = "O",
     allowed = O_TOL + half_ulp(o_ref, dtype) if rounding_allowance else O_TOL
     bad = err > allowed
     m = float(err.max()) if err.size else 0.0
-    _record(what, m, O_TOL, "O (+ half ulp of the output)" if rounding_allowance else "O")
+    frac = float((err / allowed).max()) if err.size else 0.0
+    _record(what, m, O_TOL, "O (+ half ulp of the output)" if rounding_allowance else "O", frac)
     assert not bad.any(), (f"{what}: {int(bad.sum())} elements over tolerance; max err "
                            f"{m:.4g}")
     return m
@@ -66,11 +69,11 @@ def check_lse(lse_gpu: np.ndarray, lse_ref: np.ndarray, what: str = "LSE") -> fl
     assert np.array_equal(np.isposinf(lse_gpu), inf_ref), f"{what}: +inf pattern differs"
     fin = ~inf_ref
     if not fin.any():
-        _record(what, 0.0, LSE_TOL, "LSE")
+        _record(what, 0.0, LSE_TOL, "LSE", 0.0)
         return 0.0
     err = np.abs(lse_gpu[fin].astype(np.float64) - lse_ref[fin])
     assert np.all(np.isfinite(lse_gpu[fin])), f"{what}: non-finite values"
-    _record(what, err.max(), LSE_TOL, "LSE")
+    _record(what, err.max(), LSE_TOL, "LSE", err.max() / LSE_TOL)
     assert err.max() <= LSE_TOL, f"{what}: max err {err.max():.4g}"
     return float(err.max())
 
@@ -86,8 +89,9 @@ def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, scale_ref=None,
     allowed = tol if extra is None else tol + extra
     over = err - allowed
     rel = float(err.max() / max(ref_max, 1e-30)) if err.size else 0.0
+    frac = float((err / np.maximum(allowed, 1e-300)).max()) if err.size else 0.0
     _record(what, rel, GRAD_REL_TOL, "grad / max|grad_ref|" + ("" if extra is None
-                                                                 else " (+ O16 term)"))
+                                                                 else " (+ O16 term)"), frac)
     assert over.max() <= 0, f"{what}: max err {err.max():.4g} > {tol:.4g} (+extra)"
     return rel
 
