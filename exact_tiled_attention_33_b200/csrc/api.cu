@@ -16,6 +16,11 @@ namespace fattn {
 // One status word per device (each device that loads the module gets its own copy).
 __device__ uint32_t g_status_word;
 
+cudaError_t& launch_error() {
+  static thread_local cudaError_t e = cudaSuccess;
+  return e;
+}
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -158,7 +163,9 @@ int check_grid(long long batches, long long H, long long max_len) {
 int launch_result(LaunchResult r) {
   if (r == LaunchResult::kOk) return FA_OK;
   if (r == LaunchResult::kUnsupported) return fail(FA_ERR_UNSUPPORTED, "unsupported configuration");
-  return cuda_fail(cudaGetLastError(), "kernel launch");
+  const cudaError_t e = launch_error() != cudaSuccess ? launch_error() : cudaGetLastError();
+  launch_error() = cudaSuccess;
+  return cuda_fail(e, "kernel launch");
 }
 
 constexpr float kLog2e = 1.4426950408889634f;

@@ -37,7 +37,7 @@ static LaunchResult launch_bwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
   // 3) dQ: one CTA per query tile
   dim3 grid_b((max_seqlen_q + C::BM - 1) / C::BM, p.H, batches);
   fa_bwd_dq_kernel<D, BF16><<<grid_b, C::THREADS, C::SMEM_B, stream>>>(tmQ, tmK, tmV, tmDO, p);
-  return cudaGetLastError() == cudaSuccess ? LaunchResult::kOk : LaunchResult::kCudaError;
+  return launch_status(cudaGetLastError());
 }
 
 template <int D, bool BF16>
@@ -54,7 +54,7 @@ static LaunchResult launch_bwd_fused_t(const CUtensorMap& tmQ, const CUtensorMap
     set_err[dev] = cudaFuncSetAttribute(fa_bwd_fused_kernel<D, BF16>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   });
-  if (set_err[dev] != cudaSuccess) return LaunchResult::kCudaError;
+  if (set_err[dev] != cudaSuccess) return launch_status(set_err[dev]);
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // 1) D = rowsum(dO ∘ O) and zeroed dQ sums
@@ -68,7 +68,7 @@ static LaunchResult launch_bwd_fused_t(const CUtensorMap& tmQ, const CUtensorMap
   const long long groups = (q_rows + 31) / 32 * p.H;
   const long long cv_blocks = std::min<long long>(groups, (long long)sms * 8);
   fa_bwd_dq_convert_kernel<D, BF16><<<(unsigned)cv_blocks, 256, 0, stream>>>(p, q_rows);
-  return cudaGetLastError() == cudaSuccess ? LaunchResult::kOk : LaunchResult::kCudaError;
+  return launch_status(cudaGetLastError());
 }
 
 LaunchResult launch_bwd_fused(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,

@@ -22,7 +22,7 @@ static LaunchResult launch_decode_t(const CUtensorMap& tmK, const CUtensorMap& t
     const long long warps = (long long)p.B * p.Nq * p.H;
     fa_decode_combine_kernel<D, BF16><<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(p);
   }
-  return cudaGetLastError() == cudaSuccess ? LaunchResult::kOk : LaunchResult::kCudaError;
+  return launch_status(cudaGetLastError());
 }
 
 template <int D, bool BF16, bool PAGED>

@@ -128,6 +128,16 @@ struct DecParams {
 
 enum class LaunchResult { kOk, kUnsupported, kCudaError };
 
+// The CUDA error behind the calling host thread's last kCudaError (set by the launchers).
+cudaError_t& launch_error();
+
+// kOk, or kCudaError with the error recorded for the caller's message.
+inline LaunchResult launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return LaunchResult::kOk;
+  launch_error() = e;
+  return LaunchResult::kCudaError;
+}
+
 // Forward launch for one problem.  Tensor maps are built by the caller (api.cu).
 LaunchResult launch_fwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                         const CUtensorMap& tmV, const FwdParams& p, dim3 grid,

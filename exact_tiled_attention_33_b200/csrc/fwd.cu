@@ -24,7 +24,7 @@ static LaunchResult launch_fwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
     configured[dev] = true;
   }
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
-  return cudaGetLastError() == cudaSuccess ? LaunchResult::kOk : LaunchResult::kCudaError;
+  return launch_status(cudaGetLastError());
 }
 
 // 16-bit operands: two query tiles per CTA (fwd2_kernel.cuh).
@@ -42,9 +42,9 @@ static LaunchResult launch_fwd2_t(const CUtensorMap& tmQ, const CUtensorMap& tmK
     set_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::SMEM_BYTES);
   });
-  if (set_err[dev] != cudaSuccess) return LaunchResult::kCudaError;
+  if (set_err[dev] != cudaSuccess) return launch_status(set_err[dev]);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
-  return cudaGetLastError() == cudaSuccess ? LaunchResult::kOk : LaunchResult::kCudaError;
+  return launch_status(cudaGetLastError());
 }
 
 LaunchResult launch_fwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,

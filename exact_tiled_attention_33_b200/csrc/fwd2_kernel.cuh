@@ -9,14 +9,16 @@
 // How it maps to B200:
 //   * one CTA owns two 128-row query tiles (rows q0 .. q0 + 255) and walks the union of the
 //     128-key tiles they may see; each K/V tile read from shared memory serves both;
-//   * warp 8 issues TMA loads (Q0 and Q1 once; K through a KST-deep ring, V VST-deep);
-//   * warp 9, one thread, issues every tcgen05.mma, alternating between the tiles:
+//   * warp 0 issues TMA loads (Q0 and Q1 once; K through a KST-deep ring, V VST-deep);
+//   * warp 1, one thread, issues every tcgen05.mma, alternating between the tiles:
 //     S0 = Q0 Kᵀ, S1 = Q1 Kᵀ, then per key tile O0 += P0 V, S0' = Q0 K'ᵀ, O1 += P1 V,
 //     S1' = Q1 K'ᵀ, so the tensor core works on one tile while the other tile's softmax runs;
-//   * warps 0..3 are the softmax warpgroup of tile 0, warps 4..7 that of tile 1: thread r
-//     owns row r (= tensor-memory lane r) and all 128 scores of a key tile, held in
-//     registers (10 warps leave ~200 registers a thread), so no row statistic is exchanged
-//     between warps.  P is written over its own S columns as packed
+//   * warps 4..7 are the softmax warpgroup of tile 0, warps 8..11 that of tile 1: thread r
+//     owns row r (= tensor-memory lane r) and all 128 scores of a key tile, so no row
+//     statistic is exchanged between warps.  A row's scores are read from tensor memory
+//     three times per key tile: all 128 at once for the row maximum, then 64 at a time for
+//     the exponentials (all 128 plus the exponentials' temporaries exceed the 168 registers
+//     a thread has with 12 warps);  P is written over its own S columns as packed
 //     16-bit values and read by the P·V product from tensor memory.  The reference maximum m
 //     is refreshed only when the row maximum grows by more than 2^8 (O and l share it, so
 //     this is exact); O is then rescaled in tensor memory.  The row sum that normalises O is
@@ -55,8 +57,8 @@ struct Fwd2Cfg {
   static constexpr int NBAR = B_ODONE + 2;
   static constexpr int SMEM_BYTES = OFF_BAR + 8 * NBAR + 16 + 1024;  // + alignment slack
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-  static constexpr int THREADS = 320;  // warps 0-3 / 4-7 softmax, 8 loads, 9 MMA
-  static constexpr int W_LOAD = 8, W_MMA = 9;
+  static constexpr int THREADS = 384;  // warps 0 loads, 1 MMA, 2-3 idle, 4-7 / 8-11 softmax
+  static constexpr int W_LOAD = 0, W_MMA = 1;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TM_S = 0;    // + 128 * tile
   static constexpr uint32_t TM_O = 256;  // + D * tile
@@ -72,7 +74,7 @@ struct Fwd2Cfg {
 
 // F32O: O written in fp32 before rounding (test-only instance, fa_selftest_fwd_f32).
 template <int D, bool BF16, bool F32O = false>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(384, 1)
     fa_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = Fwd2Cfg<D>;
@@ -278,9 +280,9 @@ __global__ void __maxnreg__(200)
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 4) {
     // ============================================================ softmax warpgroups
-    const int t = warp >> 2;             // query tile of this warpgroup
+    const int t = (warp - 4) >> 2;       // query tile of this warpgroup
     const int quarter = warp & 3;        // tensor-memory lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const int q0 = qp + t * BM;
@@ -304,30 +306,31 @@ __global__ void __maxnreg__(200)
       // allowed columns: lo <= e < lim (only consulted when need_mask)
       const int lim = wr >= 0 ? min(Lk - kt, i + diag + wr - kt + 1) : Lk - kt;
       const int lo = wl >= 0 ? i + diag - wl - kt : 0;
-      // the row's 128 scores in registers: four loads, one wait
-      uint32_t sr[128];
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * q]));
-      tmem_wait_ld();
-      reg_fence(sr);
-      if (need_mask) {
-#pragma unroll
-        for (int e = 0; e < 128; ++e)
-          if (e >= lim || e < lo) sr[e] = __float_as_uint(-INFINITY);
-      }
-      // row maximum: 3-input maxima, four independent chains of 32
+      // row maximum over all 128 scores: four loads, one wait
       float mq[4];
+      {
+        uint32_t sr[128];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float t1[11];
+        for (int q = 0; q < 4; ++q)
+          tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * q]));
+        tmem_wait_ld();
+        reg_fence(sr);
+        if (need_mask) {
 #pragma unroll
-        for (int e = 0; e < 10; ++e)
-          t1[e] = fmax3(__uint_as_float(sr[32 * q + 3 * e]), __uint_as_float(sr[32 * q + 3 * e + 1]),
-                        __uint_as_float(sr[32 * q + 3 * e + 2]));
-        t1[10] = fmaxf(__uint_as_float(sr[32 * q + 30]), __uint_as_float(sr[32 * q + 31]));
-        mq[q] = fmax3(fmax3(t1[0], t1[1], t1[2]), fmax3(t1[3], t1[4], t1[5]),
-                      fmax3(fmax3(t1[6], t1[7], t1[8]), t1[9], t1[10]));
+          for (int e = 0; e < 128; ++e)
+            if (e >= lim || e < lo) sr[e] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float t1[11];
+#pragma unroll
+          for (int e = 0; e < 10; ++e)
+            t1[e] = fmax3(__uint_as_float(sr[32 * q + 3 * e]), __uint_as_float(sr[32 * q + 3 * e + 1]),
+                          __uint_as_float(sr[32 * q + 3 * e + 2]));
+          t1[10] = fmaxf(__uint_as_float(sr[32 * q + 30]), __uint_as_float(sr[32 * q + 31]));
+          mq[q] = fmax3(fmax3(t1[0], t1[1], t1[2]), fmax3(t1[3], t1[4], t1[5]),
+                        fmax3(fmax3(t1[6], t1[7], t1[8]), t1[9], t1[10]));
+        }
       }
       const float mxs = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
       const float mx = mxs * c;
@@ -351,29 +354,43 @@ __global__ void __maxnreg__(200)
       // masked keys), the rest on the special-function unit
       auto exp_pass = [&](auto use_poly) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          // keys 32q .. 32q+31 -> packed columns 16q .. 16q+15 (all S columns are in registers)
-          uint32_t pk[16];
+        for (int hh = 0; hh < 2; ++hh) {
+          // keys 64hh .. 64hh+63 -> packed columns 32hh .. 32hh+31; those columns belong to
+          // score columns already read (the half before, or this half itself)
+          uint32_t sr[64];
+          tmem_ld32(tS + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(tS + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          tmem_wait_ld();
+          reg_fence(sr);
+          if (!decltype(use_poly)::value) {  // masked tiles
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float2 xx = f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[32 * q + 2 * e]),
-                                                       __uint_as_float(sr[32 * q + 2 * e + 1])),
-                                               c2, nm2));
-            float p0, p1;
-            if (decltype(use_poly)::value && e < C::kPolyPairs) {
-              const float2 pp = exp2_poly2(xx.x, xx.y);
-              p0 = pp.x;
-              p1 = pp.y;
-            } else {
-              p0 = ex2_approx(xx.x);
-              p1 = ex2_approx(xx.y);
-            }
-            pk[e] = pack2<BF16>(p0, p1);
-            ls2 = f2_add(ls2, f2_pack(p0, p1));
-            const float2 pr = unpack2<BF16>(pk[e]);
-            lrs2 = f2_add(lrs2, f2_pack(pr.x, pr.y));
+            for (int e = 0; e < 64; ++e)
+              if (64 * hh + e >= lim || 64 * hh + e < lo) sr[e] = __float_as_uint(-INFINITY);
           }
-          tmem_st16(tS + q * 16, pk);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float2 xx = f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[32 * q + 2 * e]),
+                                                         __uint_as_float(sr[32 * q + 2 * e + 1])),
+                                                 c2, nm2));
+              float p0, p1;
+              if (decltype(use_poly)::value && e < C::kPolyPairs) {
+                const float2 pp = exp2_poly2(xx.x, xx.y);
+                p0 = pp.x;
+                p1 = pp.y;
+              } else {
+                p0 = ex2_approx(xx.x);
+                p1 = ex2_approx(xx.y);
+              }
+              pk[e] = pack2<BF16>(p0, p1);
+              ls2 = f2_add(ls2, f2_pack(p0, p1));
+              const float2 pr = unpack2<BF16>(pk[e]);
+              lrs2 = f2_add(lrs2, f2_pack(pr.x, pr.y));
+            }
+            tmem_st16(tS + 32 * hh + 16 * q, pk);
+          }
         }
       };
       if (need_mask)
