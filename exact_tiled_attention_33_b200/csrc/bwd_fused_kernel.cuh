@@ -138,12 +138,18 @@ struct BwdFusedCfg {
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
   static constexpr int OFF_Q = OFF_V + TILE;             // 2 stages
-  static constexpr int OFF_DO = OFF_Q + 2 * TILE;        // 1 stage
-  static constexpr int OFF_DS = OFF_DO + TILE;
+#ifndef FATTN_BWD_DO_STAGES
+#define FATTN_BWD_DO_STAGES 1
+#endif
+  static constexpr int DO_ST = FATTN_BWD_DO_STAGES;      // dO stages (1 or 2)
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;
+  static constexpr int OFF_DS = OFF_DO + DO_ST * TILE;
   static constexpr int OFF_VEC = OFF_DS + DS_TILE;       // per Q stage: -lse*log2e [128], D [128]
   static constexpr int OFF_BAR = OFF_VEC + 2 * 2 * BM * 4;
   static constexpr int NBAR = 16;
-  static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16 + 1024;
+  // The dynamic shared memory base is 1024-byte aligned on sm_100 (it follows the 1 KB the
+  // driver reserves per CTA); the kernel checks that instead of reserving slack for it.
+  static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16;
   static_assert(SMEM <= 232448, "shared memory per CTA");
   static constexpr int THREADS = 512;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -163,13 +169,16 @@ __global__ void __launch_bounds__(512, 1)
                         const BwdParams p) {
   using C = BwdFusedCfg<D>;
   constexpr int BM = C::BM, BN = C::BN;
-  enum { B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_DOFULL = 5, B_DOEMPTY, B_SFULL, B_DPFULL, B_PFULL,
+  enum { B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_DOFULL = 5, B_DOEMPTY = 7, B_SFULL = 9, B_DPFULL, B_PFULL,
          B_DSFULL, B_DQFULL, B_DQEMPTY, B_DONE };
   static_assert(B_DONE < C::NBAR, "mbarrier slots");
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t sbase = (raw + 1023u) & ~1023u;
-  uint8_t* sgen = smem_raw + (sbase - raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t sbase = smem_u32(smem_raw);
+  if ((sbase & 1023u) != 0u) {  // the 128-byte swizzled tiles need 1024-byte atoms
+    if (threadIdx.x == 0) atomicOr(p.status, kDevSmemAlign);
+    return;
+  }
+  uint8_t* sgen = smem_raw;
   auto BAR = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + C::OFF_BAR + 8 * C::NBAR);
   volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -212,8 +221,10 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(BAR(B_QFULL + s), 32);
       mbar_init(BAR(B_QEMPTY + s), 1);
     }
-    mbar_init(BAR(B_DOFULL), 1);
-    mbar_init(BAR(B_DOEMPTY), 1);
+    for (int s = 0; s < C::DO_ST; ++s) {
+      mbar_init(BAR(B_DOFULL + s), 1);
+      mbar_init(BAR(B_DOEMPTY + s), 1);
+    }
     mbar_init(BAR(B_SFULL), 1);
     mbar_init(BAR(B_DPFULL), 1);
     mbar_init(BAR(B_PFULL), 256);
@@ -273,12 +284,14 @@ __global__ void __launch_bounds__(512, 1)
           for (int c = 0; c < C::KCH; ++c)
             tma_load_4d(&tmQ, BAR(B_QFULL + s), sbase + C::OFF_Q + s * C::TILE + c * C::CHUNK,
                         c * 64, h, q_row0 + q0, bcoord);
-          // dO has one stage: free once the dV product of the previous step has read it
-          mbar_wait(BAR(B_DOEMPTY), ((uint32_t)it & 1u) ^ 1u, abort_flag, p.status);
-          mbar_arrive_expect_tx(BAR(B_DOFULL), C::TILE);
+          // a dO stage is free once the dV product of its previous step has read it
+          const int ds_ = it % C::DO_ST;
+          mbar_wait(BAR(B_DOEMPTY + ds_), ((uint32_t)(it / C::DO_ST) & 1u) ^ 1u, abort_flag,
+                    p.status);
+          mbar_arrive_expect_tx(BAR(B_DOFULL + ds_), C::TILE);
           for (int c = 0; c < C::KCH; ++c)
-            tma_load_4d(&tmDO, BAR(B_DOFULL), sbase + C::OFF_DO + c * C::CHUNK, c * 64, h,
-                        q_row0 + q0, bcoord);
+            tma_load_4d(&tmDO, BAR(B_DOFULL + ds_), sbase + C::OFF_DO + ds_ * C::TILE + c * C::CHUNK,
+                        c * 64, h, q_row0 + q0, bcoord);
         } else {
           mbar_arrive(BAR(B_QFULL + s));
         }
@@ -315,9 +328,10 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
       };
       auto issue_dp = [&](int it) {
-        mbar_wait(BAR(B_DOFULL), (uint32_t)it & 1u, abort_flag, p.status);
+        mbar_wait(BAR(B_DOFULL + it % C::DO_ST), (uint32_t)(it / C::DO_ST) & 1u, abort_flag,
+                  p.status);
         tc_fence_after();
-        issue_kt(C::TM_DP, dV, dDOk);
+        issue_kt(C::TM_DP, dV, sdesc_adv(dDOk, (it % C::DO_ST) * C::TILE));
         mma_commit(BAR(B_DPFULL));
       };
       mbar_wait(BAR(B_KV), 0, abort_flag, p.status);
@@ -333,9 +347,10 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + C::TM_DV, tmem + C::TM_S + C::packed_col(kk), sdesc_adv(dDOm, kk * 2048),
+          mma_ts(tmem + C::TM_DV, tmem + C::TM_S + C::packed_col(kk),
+                 sdesc_adv(dDOm, (it % C::DO_ST) * C::TILE + kk * 2048),
                  ID_DV, (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(BAR(B_DOEMPTY));
+        mma_commit(BAR(B_DOEMPTY + it % C::DO_ST));
         if (it + 1 < n_q) {  // Sᵀ of the next step over Pᵀ (in order after the dV product)
           wait_q(it + 1);
           issue_kt(C::TM_S, dK, sdesc_adv(dQk, (it + 1 & 1) * C::TILE));
