@@ -46,7 +46,7 @@ FP8_SOURCES = ["exact_tiled_attention_33_b200/csrc/fwd_kernel.cuh",
                "exact_tiled_attention_33_b200/csrc/fattn_internal.h"]
 BWD_KERNEL_DESC = ("fa_bwd (D preprocess + single-pass dK/dV/dQ kernel + dQ conversion, timed "
                    "as one call)")
-FWD_SOURCES = ["exact_tiled_attention_33_b200/csrc/fwd2_kernel.cuh",
+FWD_SOURCES = ["exact_tiled_attention_33_b200/csrc/fwd_kernel.cuh",
                "exact_tiled_attention_33_b200/csrc/sm100.cuh",
                "exact_tiled_attention_33_b200/csrc/fattn_internal.h"]
 
@@ -719,11 +719,11 @@ def run_fattn(args, w):
         "frac_of_sustained_peak": bwd_ach / peak_sust,
         "traffic": read_traffic("fa_bwd", wr.name, bwd_sha),
         "flops_per_launch": 2.5 * f_fwd}
-    fwd_roof = {"kernel": "fa_fwd2_kernel", "bound": "tensor", "achieved": fwd_ach,
+    fwd_roof = {"kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": fwd_ach,
                 "peak": peak_burst, "unit": "TFLOP/s", "frac": fwd_ach / peak_burst,
                 "peak_source": f"bf16_tflops burst ({peak_src})",
                 "frac_of_sustained_peak": fwd_ach / peak_sust,
-                "traffic": read_traffic("fa_fwd2_kernel", wr.name, fwd_sha),
+                "traffic": read_traffic("fa_fwd_kernel", wr.name, fwd_sha),
                 "flops_per_launch": f_fwd}
     fwd_only = {"ms": 1e3 * fo_s / args.steps, "tflops": fwd_only_tflops,
                 "frac_of_burst_peak": fwd_only_tflops / world / peak_burst,

@@ -154,7 +154,7 @@ LaunchResult launch_fwd_f32out(int d, bool bf16, const CUtensorMap& tmQ, const C
                                cudaStream_t stream);
 
 // Query rows per forward CTA (grid x = ceil(rows / this), y = heads, z = batch or
-// sequences): two 128-row tiles for 16-bit operands, one for FP8.
+// sequences): one 128-row tile.
 int fwd_rows_per_cta(bool fp8);
 
 // Decode launch: the split kernel and, when p.splits > 1, the merge kernel.

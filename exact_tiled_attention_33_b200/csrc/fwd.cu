@@ -1,12 +1,11 @@
 // Forward kernel instantiations and launchers.
 #include <mutex>
 
-#include "fwd2_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 namespace fattn {
 
-int fwd_rows_per_cta(bool fp8) { return fp8 ? FwdCfg<128, true>::BM : 2 * Fwd2Cfg<128>::BM; }
+int fwd_rows_per_cta(bool fp8) { return fp8 ? FwdCfg<128, true>::BM : FwdCfg<128>::BM; }
 
 template <int D, bool BF16, bool FP8 = false, bool F32O = false>
 static LaunchResult launch_fwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
@@ -27,36 +26,16 @@ static LaunchResult launch_fwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
   return launch_status(cudaGetLastError());
 }
 
-// 16-bit operands: two query tiles per CTA (fwd2_kernel.cuh).
-template <int D, bool BF16, bool F32O = false>
-static LaunchResult launch_fwd2_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                                  const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
-                                  cudaStream_t stream) {
-  using C = Fwd2Cfg<D>;
-  auto kern = fa_fwd2_kernel<D, BF16, F32O>;
-  static std::once_flag once[64];
-  static cudaError_t set_err[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return LaunchResult::kCudaError;
-  std::call_once(once[dev], [&] {
-    set_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        C::SMEM_BYTES);
-  });
-  if (set_err[dev] != cudaSuccess) return launch_status(set_err[dev]);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
-  return launch_status(cudaGetLastError());
-}
-
 LaunchResult launch_fwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                         const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
                         cudaStream_t stream) {
   if (d == 128) {
-    return bf16 ? launch_fwd2_t<128, true>(tmQ, tmK, tmV, p, grid, stream)
-                : launch_fwd2_t<128, false>(tmQ, tmK, tmV, p, grid, stream);
+    return bf16 ? launch_fwd_t<128, true>(tmQ, tmK, tmV, p, grid, stream)
+                : launch_fwd_t<128, false>(tmQ, tmK, tmV, p, grid, stream);
   }
   if (d == 64) {
-    return bf16 ? launch_fwd2_t<64, true>(tmQ, tmK, tmV, p, grid, stream)
-                : launch_fwd2_t<64, false>(tmQ, tmK, tmV, p, grid, stream);
+    return bf16 ? launch_fwd_t<64, true>(tmQ, tmK, tmV, p, grid, stream)
+                : launch_fwd_t<64, false>(tmQ, tmK, tmV, p, grid, stream);
   }
   return LaunchResult::kUnsupported;
 }
@@ -73,11 +52,11 @@ LaunchResult launch_fwd_f32out(int d, bool bf16, const CUtensorMap& tmQ, const C
                                const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
                                cudaStream_t stream) {
   if (d == 128)
-    return bf16 ? launch_fwd2_t<128, true, true>(tmQ, tmK, tmV, p, grid, stream)
-                : launch_fwd2_t<128, false, true>(tmQ, tmK, tmV, p, grid, stream);
+    return bf16 ? launch_fwd_t<128, true, false, true>(tmQ, tmK, tmV, p, grid, stream)
+                : launch_fwd_t<128, false, false, true>(tmQ, tmK, tmV, p, grid, stream);
   if (d == 64)
-    return bf16 ? launch_fwd2_t<64, true, true>(tmQ, tmK, tmV, p, grid, stream)
-                : launch_fwd2_t<64, false, true>(tmQ, tmK, tmV, p, grid, stream);
+    return bf16 ? launch_fwd_t<64, true, false, true>(tmQ, tmK, tmV, p, grid, stream)
+                : launch_fwd_t<64, false, false, true>(tmQ, tmK, tmV, p, grid, stream);
   return LaunchResult::kUnsupported;
 }
 
