@@ -126,6 +126,24 @@ struct PerDeviceSymbol {
   }
 };
 
+// Tensor map over fp32 [rows, H, d] sums for TMA reduce-adds: box 32 columns (128 bytes,
+// one swizzle row) x 1 head x 128 rows, 128-byte swizzle; rows past the end are skipped.
+int make_map_f32_reduce(CUtensorMap* map, float* base, int d, int H, long long rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  if (int e = ensure_context()) return e;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)rows, 1};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)rows * H * d * 4};
+  cuuint32_t box[4] = {32, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled (dQ sums) failed (code " + std::to_string((int)r) + ")");
+  return FA_OK;
+}
+
 uint32_t* status_ptr() {
   static PerDeviceSymbol<uint32_t> cache;
   int dev = 0;
@@ -457,9 +475,8 @@ namespace {
 // Backward workspace: D = rowsum(dO ∘ O) (fp32, one per token row and head), then, for the
 // single-pass backward, the fp32 dQ sums (H x rows rounded up to 32 x d).
 size_t d_vector_bytes(long long rows, long long H) { return align256((size_t)rows * H * 4); }
-long long acc_rows_of(long long rows) { return (rows + 31) / 32 * 32; }
 size_t dq_sum_bytes(long long rows, long long H, long long d) {
-  return align256((size_t)acc_rows_of(rows) * H * d * 4);
+  return align256((size_t)rows * H * d * 4);
 }
 
 }  // namespace
@@ -505,7 +522,6 @@ int bwd_common(const void* q, const void* k, const void* v, const void* o, const
   p.dq_acc = single_pass ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                                     d_vector_bytes(q_rows, H))
                          : nullptr;
-  p.acc_rows = acc_rows_of(q_rows);
   p.cu_q = cu_q; p.cu_k = cu_k;
   p.B = cu_q ? 1 : batches; p.N = N; p.H = H;
   p.total_q = total_q; p.total_k = total_k;
@@ -518,9 +534,14 @@ int bwd_common(const void* q, const void* k, const void* v, const void* o, const
   p.max_seqlen_k = max_seqlen_k;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-  if (single_pass)
-    return launch_result(launch_bwd_fused(d, dtype == FA_BF16, mq, mk, mv, mdo, p, q_rows,
+  if (single_pass) {
+    // the fp32 dQ sums, [q_rows, H, d], reduce-added by the TMA unit 32 columns x 128 rows
+    // at a time
+    CUtensorMap mdq;
+    if (int e = make_map_f32_reduce(&mdq, p.dq_acc, d, H, q_rows)) return e;
+    return launch_result(launch_bwd_fused(d, dtype == FA_BF16, mq, mk, mv, mdo, mdq, p, q_rows,
                                           max_seqlen_q, max_seqlen_k, batches, stream));
+  }
   return launch_result(launch_bwd(d, dtype == FA_BF16, mq, mk, mv, mdo, p, q_rows, max_seqlen_q,
                                   max_seqlen_k, batches, stream));
 }

@@ -43,8 +43,9 @@ static LaunchResult launch_bwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
 template <int D, bool BF16>
 static LaunchResult launch_bwd_fused_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                        const CUtensorMap& tmV, const CUtensorMap& tmDO,
-                                       const BwdParams& p, long long q_rows, int max_seqlen_k,
-                                       int batches, cudaStream_t stream) {
+                                       const CUtensorMap& tmDQ, const BwdParams& p,
+                                       long long q_rows, int max_seqlen_k, int batches,
+                                       cudaStream_t stream) {
   using C = BwdFusedCfg<D>;
   static std::once_flag once[64];
   static cudaError_t set_err[64] = {};
@@ -63,25 +64,26 @@ static LaunchResult launch_bwd_fused_t(const CUtensorMap& tmQ, const CUtensorMap
   fa_bwd_pre_acc_kernel<D, BF16><<<(unsigned)pre_blocks, 256, 0, stream>>>(p, q_rows);
   // 2) dK, dV and the dQ partial sums: one CTA per key tile
   dim3 grid((max_seqlen_k + C::BN - 1) / C::BN, p.H, batches);
-  fa_bwd_fused_kernel<D, BF16><<<grid, C::THREADS, C::SMEM, stream>>>(tmQ, tmK, tmV, tmDO, p);
+  fa_bwd_fused_kernel<D, BF16><<<grid, C::THREADS, C::SMEM, stream>>>(tmQ, tmK, tmV, tmDO, tmDQ, p);
   // 3) dQ = scale * sums, rounded to 16 bits
-  const long long groups = (q_rows + 31) / 32 * p.H;
-  const long long cv_blocks = std::min<long long>(groups, (long long)sms * 8);
-  fa_bwd_dq_convert_kernel<D, BF16><<<(unsigned)cv_blocks, 256, 0, stream>>>(p, q_rows);
+  const long long elems = q_rows * p.H * D;
+  const long long cv_blocks = std::min<long long>((elems / 8 + 255) / 256, (long long)sms * 16);
+  fa_bwd_dq_convert_kernel<BF16><<<(unsigned)cv_blocks, 256, 0, stream>>>(p, elems);
   return launch_status(cudaGetLastError());
 }
 
 LaunchResult launch_bwd_fused(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                              const CUtensorMap& tmV, const CUtensorMap& tmDO, const BwdParams& p,
-                              long long q_rows, int max_seqlen_q, int max_seqlen_k, int batches,
+                              const CUtensorMap& tmV, const CUtensorMap& tmDO,
+                              const CUtensorMap& tmDQ, const BwdParams& p, long long q_rows,
+                              int max_seqlen_q, int max_seqlen_k, int batches,
                               cudaStream_t stream) {
   (void)max_seqlen_q;
   if (d == 128)
-    return bf16 ? launch_bwd_fused_t<128, true>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream)
-                : launch_bwd_fused_t<128, false>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream);
+    return bf16 ? launch_bwd_fused_t<128, true>(tmQ, tmK, tmV, tmDO, tmDQ, p, q_rows, max_seqlen_k, batches, stream)
+                : launch_bwd_fused_t<128, false>(tmQ, tmK, tmV, tmDO, tmDQ, p, q_rows, max_seqlen_k, batches, stream);
   if (d == 64)
-    return bf16 ? launch_bwd_fused_t<64, true>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream)
-                : launch_bwd_fused_t<64, false>(tmQ, tmK, tmV, tmDO, p, q_rows, max_seqlen_k, batches, stream);
+    return bf16 ? launch_bwd_fused_t<64, true>(tmQ, tmK, tmV, tmDO, tmDQ, p, q_rows, max_seqlen_k, batches, stream)
+                : launch_bwd_fused_t<64, false>(tmQ, tmK, tmV, tmDO, tmDQ, p, q_rows, max_seqlen_k, batches, stream);
   return LaunchResult::kUnsupported;
 }
 

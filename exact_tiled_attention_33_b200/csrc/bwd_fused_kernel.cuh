@@ -22,7 +22,9 @@
 // LSE and D; dO one stage), warp 1 issues every tcgen05.mma from one thread, warps 4-11 are
 // two compute warpgroups (thread = key row, one half of the 128 query columns each: Pᵀ into
 // tensor memory, dSᵀ into shared memory), warps 12-15 drain each dQ partial from tensor
-// memory into the fp32 sums (thread = query row) while the compute warps move on.
+// memory into the fp32 sums (thread = query row) while the compute warps move on: 32
+// columns at a time into a swizzled shared-memory staging tile, which one thread hands to the
+// TMA unit as a reduce-add into the sums (two staging tiles alternate).
 // Tensor memory: Sᵀ/Pᵀ [0,128) | dPᵀ [128,256) | dK [256,256+D) | dV [256+D,256+2D); the dQ
 // partial (128 query lanes x D columns) takes the dPᵀ columns at D = 128 (free once the
 // compute warps have loaded dPᵀ; the next dPᵀ waits for the drain) and columns [384,448) at
@@ -83,46 +85,27 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_acc_kernel(const BwdParams p, 
       }
       p.dvec[di] = acc;
     }
-    // zero the row's dQ sums: lane l clears columns 4l..4l+3 (and 4l+128.. for D > 128)
+    // zero the row's dQ sums ([rows, H, D], like dq): lane l clears columns 4l .. 4l+3
 #pragma unroll
     for (int c = lane * 4; c < D; c += 128)
-      *reinterpret_cast<float4*>(p.dq_acc + dq_acc_index(row, h, c, D, p.acc_rows)) =
-          make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(p.dq_acc + (size_t)w * D + c) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
 // ------------------------------------------------------------------ dQ conversion
-// One CTA of 256 threads per (group of 32 token rows, head): the group's fp32 sums (32 x D,
-// contiguous) go through shared memory so that each warp writes whole 16-bit rows.
-template <int D, bool BF16>
-__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const BwdParams p, long long rows_total) {
-  __shared__ float tile[32][D + 4];
-  const long long groups = (rows_total + 31) / 32;
-  for (long long gi = blockIdx.x; gi < groups * p.H; gi += gridDim.x) {
-    const int h = (int)(gi % p.H);
-    const long long g = gi / p.H;
-    const float4* src = reinterpret_cast<const float4*>(p.dq_acc + dq_acc_index(g * 32, h, 0, D, p.acc_rows));
-    // float4 f of the group: columns 4 (f / 32) .. +3 of row f % 32
-    for (int f = threadIdx.x; f < 8 * D; f += blockDim.x) {
-      const float4 v = src[f];
-      const int r = f & 31, c = (f >> 5) * 4;
-      tile[r][c] = v.x;
-      tile[r][c + 1] = v.y;
-      tile[r][c + 2] = v.z;
-      tile[r][c + 3] = v.w;
-    }
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int r = warp; r < 32; r += blockDim.x / 32) {
-      const long long row = g * 32 + r;
-      if (row < rows_total) {
-        uint16_t* dst = reinterpret_cast<uint16_t*>(p.dq) + ((size_t)row * p.H + h) * D;
-#pragma unroll
-        for (int c = lane * 2; c < D; c += 64)
-          *reinterpret_cast<uint32_t*>(dst + c) = pack2<BF16>(tile[r][c] * p.scale, tile[r][c + 1] * p.scale);
-      }
-    }
-    __syncthreads();
+// dQ = scale · sums, rounded to 16 bits; the sums and dq share the [rows, H, D] layout, so
+// each thread converts 8 consecutive elements (two float4 reads, one 16-byte write).
+template <bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const BwdParams p, long long elems) {
+  const long long n8 = elems >> 3;  // D is a multiple of 8
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(p.dq_acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(p.dq_acc)[2 * i + 1];
+    const float sc = p.scale;
+    reinterpret_cast<uint4*>(p.dq)[i] =
+        make_uint4(pack2<BF16>(a.x * sc, a.y * sc), pack2<BF16>(a.z * sc, a.w * sc),
+                   pack2<BF16>(b.x * sc, b.y * sc), pack2<BF16>(b.z * sc, b.w * sc));
   }
 }
 
@@ -144,7 +127,9 @@ struct BwdFusedCfg {
   static constexpr int DO_ST = FATTN_BWD_DO_STAGES;      // dO stages (1 or 2)
   static constexpr int OFF_DO = OFF_Q + 2 * TILE;
   static constexpr int OFF_DS = OFF_DO + DO_ST * TILE;
-  static constexpr int OFF_VEC = OFF_DS + DS_TILE;       // per Q stage: -lse*log2e [128], D [128]
+  static constexpr int STG_TILE = 128 * 128;            // dQ staging: 128 rows x 32 fp32
+  static constexpr int OFF_STG = OFF_DS + DS_TILE;       // 2 staging tiles
+  static constexpr int OFF_VEC = OFF_STG + 2 * STG_TILE; // per Q stage: -lse*log2e [128], D [128]
   static constexpr int OFF_BAR = OFF_VEC + 2 * 2 * BM * 4;
   static constexpr int NBAR = 16;
   // The dynamic shared memory base is 1024-byte aligned on sm_100 (it follows the 1 KB the
@@ -166,7 +151,7 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                        const BwdParams p) {
+                        const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BwdFusedCfg<D>;
   constexpr int BM = C::BM, BN = C::BN;
   enum { B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_DOFULL = 5, B_DOEMPTY = 7, B_SFULL = 9, B_DPFULL, B_PFULL,
@@ -520,34 +505,48 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp >= 12) {
     // ============================================================ dQ drain
-    // thread = query row (tensor-memory lane) of the partial; adds its D columns into the
-    // fp32 sums, four at a time (512 contiguous bytes per warp and instruction).
+    // thread = query row (tensor-memory lane) of the partial.  Per 32 columns: tensor memory
+    // -> registers -> the staging tile (128-byte swizzle, the layout of the tensor map's box)
+    // -> one TMA reduce-add into the fp32 sums.  The TMA unit skips rows past the sums' end;
+    // rows of this tile past the sequence carry zeros (their P is 0).
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const bool leader = threadIdx.x == 12 * 32;  // issues and waits for the reduce-adds
+    uint32_t nchunk = 0;
+    if (leader) tma_prefetch_desc(&tmDQ);
     for (int it = 0; it < n_q; ++it) {
-      const int qg = q_tile(it) * BM + r;
+      const int q0 = q_tile(it) * BM;
       mbar_wait(BAR(B_DQFULL), (uint32_t)it & 1u, abort_flag, p.status);
       tc_fence_after();
-      const long long row = acc_row0 + qg;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
+      for (int c = 0; c < D; c += 32, ++nchunk) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + C::TM_DQ + c, v);
         tmem_wait_ld();
         reg_fence(v);
-        if (qg < Lq) {
-          float* dst = p.dq_acc + dq_acc_index(row, h, c, D, p.acc_rows);
+        if (c + 32 == D) {  // the partial has been read: the next dPᵀ may overwrite it
+          tc_fence_before();
+          mbar_arrive(BAR(B_DQEMPTY));
+        }
+        // staging tile nchunk % 2 was last handed to the TMA unit two chunks ago
+        if (leader && nchunk >= 2) bulk_wait_group_read1();
+        named_barrier_sync(1, 128);
+        uint8_t* row_ptr = sgen + C::OFF_STG + (nchunk & 1u) * C::STG_TILE + r * 128;
 #pragma unroll
-          for (int u = 0; u < 8; ++u)  // columns c + 4u .. c + 4u + 3 are 128 floats apart
-            atomicAdd(reinterpret_cast<float4*>(dst + u * 128),
-                      make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
-                                  __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3])));
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(row_ptr + ((u ^ (r & 7)) << 4)) =
+              make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        fence_proxy_async_smem();
+        named_barrier_sync(1, 128);
+        if (leader) {
+          tma_reduce_add_4d(&tmDQ, sbase + C::OFF_STG + (nchunk & 1u) * C::STG_TILE, c, h,
+                            (int)(acc_row0 + q0), 0);
+          bulk_commit_group();
         }
       }
-      tc_fence_before();
-      mbar_arrive(BAR(B_DQEMPTY));
     }
+    if (leader) bulk_wait_group0();  // every reduce-add has completed before the CTA ends
   }
 
   tc_fence_before();

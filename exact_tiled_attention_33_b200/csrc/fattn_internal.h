@@ -43,9 +43,8 @@ struct BwdParams {
   void* dk;
   void* dv;
   float* dvec;        // D = rowsum(dO ∘ O), same layout as lse (caller's workspace)
-  float* dq_acc;      // single-pass backward: fp32 dQ sums (caller's workspace), laid out
-                      // [H][acc_rows / 32][D / 4][32][4] over token rows (dq_acc_index)
-  long long acc_rows; // token rows of dq_acc per head (B*N or total_q, rounded up to 32)
+  float* dq_acc;      // single-pass backward: fp32 dQ sums (caller's workspace), [rows, H, D]
+                      // like dq itself (rows = B*N or total_q)
   const int* cu_q;
   const int* cu_k;
   int B, N, H;
@@ -57,16 +56,6 @@ struct BwdParams {
   int max_seqlen_q, max_seqlen_k;  // varlen: longest allowed segments (longer: skipped, reported)
   uint32_t* status;
 };
-
-// Position of element (token row, head h, column c) in the single-pass backward's fp32 dQ
-// sums: for every head, groups of 32 consecutive token rows hold their D columns four at a
-// time, so the 32 lanes of a warp that add four columns of 32 consecutive rows touch 512
-// contiguous bytes.
-__host__ __device__ inline size_t dq_acc_index(long long row, int h, int c, int D,
-                                               long long acc_rows) {
-  return (((size_t)h * (size_t)(acc_rows >> 5) + (size_t)(row >> 5)) * (size_t)(D >> 2) +
-          (size_t)(c >> 2)) * 128u + (size_t)(row & 31) * 4u + (size_t)(c & 3);
-}
 
 // Attention window.  Within one sequence of Lq queries and Lk keys (diag = Lk - Lq, the
 // bottom-right alignment), key j is allowed for query i iff
@@ -162,10 +151,13 @@ LaunchResult launch_decode(int d, bool bf16, bool paged, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const DecParams& p, cudaStream_t stream);
 
 // Single-pass backward launch: D preprocess (and zeroing of the dQ sums), the fused
-// dK/dV/dQ pass, the dQ conversion.  Same arguments as launch_bwd; p.dq_acc must be set.
+// dK/dV/dQ pass, the dQ conversion.  As launch_bwd, plus tmDQ: a tensor map over the fp32
+// dQ sums p.dq_acc ([rows, H, D]; box 32 columns x 1 head x 128 rows, 128-byte swizzle)
+// that the pass reduce-adds its dQ partials through.
 LaunchResult launch_bwd_fused(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                              const CUtensorMap& tmV, const CUtensorMap& tmDO, const BwdParams& p,
-                              long long q_rows, int max_seqlen_q, int max_seqlen_k, int batches,
+                              const CUtensorMap& tmV, const CUtensorMap& tmDO,
+                              const CUtensorMap& tmDQ, const BwdParams& p, long long q_rows,
+                              int max_seqlen_q, int max_seqlen_k, int batches,
                               cudaStream_t stream);
 
 // Backward launch: D preprocess, dK/dV pass, dQ pass.  q_rows = B*N (dense) or total_q

@@ -90,8 +90,8 @@ int fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* l
                   int total_q, int total_k, int dtype, void* stream);
 
 /* Workspace bytes the dense backward needs: D = rowsum(dO ∘ O) [B,H,N] fp32 rounded up to
- * a multiple of 256 bytes, followed by the fp32 sums of dQ (H x B*N rounded up to 32 x d
- * floats, again rounded to 256 bytes).  Linear in N: no N x N buffer exists. */
+ * a multiple of 256 bytes, followed by the fp32 sums of dQ ([B,N,H,d], again rounded to 256
+ * bytes).  Linear in N: no N x N buffer exists. */
 size_t fa_bwd_workspace_size(int B, int N, int H, int d);
 
 /* Dense backward: recomputes P from q, k and lse (as written by fa_fwd with the same
@@ -111,7 +111,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            void* stream);
 
 /* Workspace bytes the varlen backward needs: D [H,total_q] fp32 and the fp32 dQ sums
- * (H x total_q rounded up to 32 x d floats), each rounded up to a multiple of 256 bytes. */
+ * ([total_q,H,d]), each rounded up to a multiple of 256 bytes. */
 size_t fa_varlen_bwd_workspace_size(int total_q, int H, int d);
 
 /* Varlen backward; arguments as fa_varlen_fwd plus the gradient buffers.  Computed as

@@ -12,7 +12,3 @@ extern "C" void shim_query_tile_range(int k_first, int k_last, int Lq, int diag,
   fattn::query_tile_range(k_first, k_last, Lq, diag, win_left, win_right, BM, begin, count);
 }
 
-extern "C" unsigned long long shim_dq_acc_index(long long row, int h, int c, int D,
-                                                long long acc_rows) {
-  return (unsigned long long)fattn::dq_acc_index(row, h, c, D, acc_rows);
-}

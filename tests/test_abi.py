@@ -46,16 +46,16 @@ def test_status_strings(lib):
 
 def test_workspace_sizes(lib):
     # the backward workspace holds D = rowsum(dO ∘ O) (fp32 [B, H, N]) and the fp32 dQ sums
-    # (H x rows rounded up to 32 x d), each rounded up to 256 bytes
+    # ([rows, H, d]), each rounded up to 256 bytes
     def r256(x):
         return (x + 255) // 256 * 256
 
     B, N, H, d = 2, 16384, 32, 128
     assert lib.fa_bwd_workspace_size(B, N, H, d) == B * H * N * 4 + B * N * H * d * 4
-    assert lib.fa_bwd_workspace_size(1, 3, 1, 64) == 256 + r256(32 * 64 * 4)
+    assert lib.fa_bwd_workspace_size(1, 3, 1, 64) == 256 + r256(3 * 64 * 4)
     assert lib.fa_bwd_workspace_size(0, 3, 1, 64) == 0
     assert lib.fa_varlen_bwd_workspace_size(896, 32, 128) == 896 * 32 * 4 + 896 * 32 * 128 * 4
-    assert lib.fa_varlen_bwd_workspace_size(33, 2, 64) == r256(33 * 2 * 4) + 64 * 2 * 64 * 4
+    assert lib.fa_varlen_bwd_workspace_size(33, 2, 64) == r256(33 * 2 * 4) + r256(33 * 2 * 64 * 4)
 
 
 P = ctypes.c_void_p(4096)  # a 16-byte aligned fake address; validation fails before any use

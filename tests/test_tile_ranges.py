@@ -96,27 +96,3 @@ def test_tile_ranges_at_kernel_sizes(shim):
             want = {int(i) // T for i in np.nonzero(full[:, k0:k1 + 1].any(axis=1))[0]}
             assert _call(shim.shim_query_tile_range, k0, k1, Lq, diag, *win, T) == want
 
-
-def test_dq_sum_layout_is_a_bijection_with_warp_contiguous_columns(shim):
-    # The single-pass backward's fp32 dQ sums: every (token row, head, column) has its own
-    # slot inside the H x rows(rounded to 32) x D buffer, and the 32 rows of a warp that add
-    # the same four columns touch 512 contiguous bytes.
-    import ctypes
-    f = shim.shim_dq_acc_index
-    f.restype = ctypes.c_ulonglong
-    f.argtypes = [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_longlong]
-    for D, rows, H in ((64, 70, 3), (128, 33, 2)):
-        acc_rows = (rows + 31) // 32 * 32
-        seen = set()
-        for h in range(H):
-            for r in range(rows):
-                for c in range(D):
-                    idx = f(r, h, c, D, acc_rows)
-                    assert idx < H * acc_rows * D
-                    seen.add(idx)
-        assert len(seen) == H * rows * D
-        for c4 in range(0, D, 4):
-            base = f(32, 1 % H, c4, D, acc_rows)
-            got = sorted(f(32 + r, 1 % H, c4 + e, D, acc_rows) for r in range(32) for e in range(4))
-            assert got == list(range(base, base + 128))
-
