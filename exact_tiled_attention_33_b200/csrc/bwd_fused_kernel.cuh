@@ -22,9 +22,10 @@
 // LSE and D; dO one stage), warp 1 issues every tcgen05.mma from one thread, warps 4-11 are
 // two compute warpgroups (thread = key row, one half of the 128 query columns each: Pᵀ into
 // tensor memory, dSᵀ into shared memory), warps 12-15 drain each dQ partial from tensor
-// memory into the fp32 sums (thread = query row) while the compute warps move on: 32
-// columns at a time into a swizzled shared-memory staging tile, which one thread hands to the
-// TMA unit as a reduce-add into the sums (two staging tiles alternate).
+// memory into the fp32 sums (thread = query row) while the compute warps move on: the whole
+// partial goes into swizzled shared-memory staging tiles of 32 columns (at D = 128 two of them
+// lie in the dS tile, free from the dQ product until the next dS), tensor memory is released,
+// and one thread hands the tiles to the TMA unit as reduce-adds into the sums.
 // Tensor memory: Sᵀ/Pᵀ [0,128) | dPᵀ [128,256) | dK [256,256+D) | dV [256+D,256+2D); the dQ
 // partial (128 query lanes x D columns) takes the dPᵀ columns at D = 128 (free once the
 // compute warps have loaded dPᵀ; the next dPᵀ waits for the drain) and columns [384,448) at
@@ -131,7 +132,7 @@ struct BwdFusedCfg {
   static constexpr int OFF_STG = OFF_DS + DS_TILE;       // 2 staging tiles
   static constexpr int OFF_VEC = OFF_STG + 2 * STG_TILE; // per Q stage: -lse*log2e [128], D [128]
   static constexpr int OFF_BAR = OFF_VEC + 2 * 2 * BM * 4;
-  static constexpr int NBAR = 16;
+  static constexpr int NBAR = 18;
   // The dynamic shared memory base is 1024-byte aligned on sm_100 (it follows the 1 KB the
   // driver reserves per CTA); the kernel checks that instead of reserving slack for it.
   static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16;
@@ -155,8 +156,8 @@ __global__ void __launch_bounds__(512, 1)
   using C = BwdFusedCfg<D>;
   constexpr int BM = C::BM, BN = C::BN;
   enum { B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_DOFULL = 5, B_DOEMPTY = 7, B_SFULL = 9, B_DPFULL, B_PFULL,
-         B_DSFULL, B_DQFULL, B_DQEMPTY, B_DONE };
-  static_assert(B_DONE < C::NBAR, "mbarrier slots");
+         B_DSFULL, B_DQFULL, B_DQEMPTY, B_DONE, B_DSFREE };
+  static_assert(B_DSFREE < C::NBAR, "mbarrier slots");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase = smem_u32(smem_raw);
   if ((sbase & 1023u) != 0u) {  // the 128-byte swizzled tiles need 1024-byte atoms
@@ -217,6 +218,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_DQFULL), 1);
     mbar_init(BAR(B_DQEMPTY), 128);
     mbar_init(BAR(B_DONE), 1);
+    mbar_init(BAR(B_DSFREE), 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
@@ -446,6 +448,8 @@ __global__ void __launch_bounds__(512, 1)
       tmem_wait_ld();
       reg_fence(dv);
       const float4* d4 = reinterpret_cast<const float4*>(&vec[BM + cbase]);
+      if (C::DQ_ALIASES_DP && it > 0)  // the previous dQ partial's staging in this tile is read
+        mbar_wait(BAR(B_DSFREE), (uint32_t)(it - 1) & 1u, abort_flag, p.status);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {  // 16-byte unit u = queries cbase + 8u .. + 7
         uint32_t w[4];
@@ -505,44 +509,61 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp >= 12) {
     // ============================================================ dQ drain
-    // thread = query row (tensor-memory lane) of the partial.  Per 32 columns: tensor memory
-    // -> registers -> the staging tile (128-byte swizzle, the layout of the tensor map's box)
-    // -> one TMA reduce-add into the fp32 sums.  The TMA unit skips rows past the sums' end;
-    // rows of this tile past the sequence carry zeros (their P is 0).
+    // thread = query row (tensor-memory lane) of the partial.  The partial is copied, 64
+    // columns at a time, into staging tiles of 32 columns (128-byte swizzle, the layout of the
+    // tensor map's box); tensor memory is released; then one thread issues a TMA reduce-add
+    // per staging tile.  The TMA unit skips rows past the sums' end; rows of this tile past
+    // the sequence carry zeros (their P is 0).  At D = 128 staging tiles 0 and 1 are the dS
+    // tile (the dK and dQ products, its readers, completed before the partial was final); the
+    // next dS waits until those reduce-adds have read them (B_DSFREE).
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const bool leader = threadIdx.x == 12 * 32;  // issues and waits for the reduce-adds
-    uint32_t nchunk = 0;
+    auto stage_off = [&](int c) -> uint32_t {   // staging tile of columns 32c .. 32c+31
+      if constexpr (C::DQ_ALIASES_DP)
+        return c < 2 ? (uint32_t)(C::OFF_DS + c * C::STG_TILE) : (uint32_t)(C::OFF_STG + (c - 2) * C::STG_TILE);
+      else
+        return (uint32_t)(C::OFF_STG + c * C::STG_TILE);
+    };
     if (leader) tma_prefetch_desc(&tmDQ);
     for (int it = 0; it < n_q; ++it) {
       const int q0 = q_tile(it) * BM;
       mbar_wait(BAR(B_DQFULL), (uint32_t)it & 1u, abort_flag, p.status);
       tc_fence_after();
+      if (leader && it > 0) bulk_wait_group_read0();  // the previous partial's tiles are read
+      named_barrier_sync(1, 128);
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32, ++nchunk) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + C::TM_DQ + c, v);
+      for (int c2 = 0; c2 < D / 64; ++c2) {
+        uint32_t v[64];
+        tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * c2, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * c2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_wait_ld();
         reg_fence(v);
-        if (c + 32 == D) {  // the partial has been read: the next dPᵀ may overwrite it
-          tc_fence_before();
-          mbar_arrive(BAR(B_DQEMPTY));
-        }
-        // staging tile nchunk % 2 was last handed to the TMA unit two chunks ago
-        if (leader && nchunk >= 2) bulk_wait_group_read1();
-        named_barrier_sync(1, 128);
-        uint8_t* row_ptr = sgen + C::OFF_STG + (nchunk & 1u) * C::STG_TILE + r * 128;
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<uint4*>(row_ptr + ((u ^ (r & 7)) << 4)) =
-              make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-        fence_proxy_async_smem();
-        named_barrier_sync(1, 128);
-        if (leader) {
-          tma_reduce_add_4d(&tmDQ, sbase + C::OFF_STG + (nchunk & 1u) * C::STG_TILE, c, h,
-                            (int)(acc_row0 + q0), 0);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint8_t* row_ptr = sgen + stage_off(2 * c2 + h2) + r * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(row_ptr + ((u ^ (r & 7)) << 4)) =
+                make_uint4(v[32 * h2 + 4 * u], v[32 * h2 + 4 * u + 1], v[32 * h2 + 4 * u + 2],
+                           v[32 * h2 + 4 * u + 3]);
+        }
+      }
+      // the partial has been read: the next dPᵀ may overwrite its tensor-memory columns
+      tc_fence_before();
+      mbar_arrive(BAR(B_DQEMPTY));
+      fence_proxy_async_smem();
+      named_barrier_sync(1, 128);
+      if (leader) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          tma_reduce_add_4d(&tmDQ, sbase + stage_off(c), 32 * c, h, (int)(acc_row0 + q0), 0);
           bulk_commit_group();
+        }
+        if constexpr (C::DQ_ALIASES_DP) {
+          bulk_wait_group_read2();  // the two reduce-adds from the dS tile have read it
+          mbar_arrive(BAR(B_DSFREE));
         }
       }
     }
