@@ -156,8 +156,8 @@ __global__ void __launch_bounds__(512, 1)
   using C = BwdFusedCfg<D>;
   constexpr int BM = C::BM, BN = C::BN;
   enum { B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_DOFULL = 5, B_DOEMPTY = 7, B_SFULL = 9, B_DPFULL, B_PFULL,
-         B_DSFULL, B_DQFULL, B_DQEMPTY, B_DONE, B_DSFREE };
-  static_assert(B_DSFREE < C::NBAR, "mbarrier slots");
+         B_DSFULL, B_DQFULL, B_DQEMPTY, B_DONE, B_DSFREE, B_DKDONE };
+  static_assert(B_DKDONE < C::NBAR, "mbarrier slots");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase = smem_u32(smem_raw);
   if ((sbase & 1023u) != 0u) {  // the 128-byte swizzled tiles need 1024-byte atoms
@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_DQEMPTY), 128);
     mbar_init(BAR(B_DONE), 1);
     mbar_init(BAR(B_DSFREE), 1);
+    mbar_init(BAR(B_DKDONE), 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
@@ -343,16 +344,11 @@ __global__ void __launch_bounds__(512, 1)
           issue_kt(C::TM_S, dK, sdesc_adv(dQk, (it + 1 & 1) * C::TILE));
           mma_commit(BAR(B_SFULL));
         }
+        // dQ  = dS K   (A = dS [queries][keys], the dSᵀ tile read MN-major; B = K [keys][d]
+        //              MN-major), first, so that its drain overlaps the dK product
         // dK += dSᵀ Q  (A = dSᵀ [keys][queries] K-major; B = Q [queries][d] MN-major)
-        // dQ  = dS K   (A = dS, the same tile read MN-major; B = K [keys][d] MN-major)
         mbar_wait(BAR(B_DSFULL), ph, abort_flag, p.status);
         tc_fence_after();
-        const uint64_t qm = sdesc_adv(dQm, s * C::TILE);
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ss(tmem + C::TM_DK, sdesc_adv(dSk, (kk >> 2) * C::CHUNK + (kk & 3) * 32),
-                 sdesc_adv(qm, kk * 2048), ID_DK, (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(BAR(B_QEMPTY + s));
         if (C::DQ_ALIASES_DP == false && it > 0) {
           // the dQ columns of the previous step must have been drained
           mbar_wait(BAR(B_DQEMPTY), (uint32_t)(it - 1) & 1u, abort_flag, p.status);
@@ -363,6 +359,13 @@ __global__ void __launch_bounds__(512, 1)
           mma_ss(tmem + C::TM_DQ, sdesc_adv(dSm, kk * 2048), sdesc_adv(dKm, kk * 2048), ID_DQ,
                  kk > 0 ? 1u : 0u);
         mma_commit(BAR(B_DQFULL));
+        const uint64_t qm = sdesc_adv(dQm, s * C::TILE);
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ss(tmem + C::TM_DK, sdesc_adv(dSk, (kk >> 2) * C::CHUNK + (kk & 3) * 32),
+                 sdesc_adv(qm, kk * 2048), ID_DK, (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(BAR(B_QEMPTY + s));
+        mma_commit(BAR(B_DKDONE));  // the dS tile is no longer read by this step's products
         if (it + 1 < n_q) {
           if constexpr (C::DQ_ALIASES_DP) {
             // the next dPᵀ overwrites this dQ partial: wait until it has been drained
@@ -533,8 +536,15 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_after();
       if (leader && it > 0) bulk_wait_group_read0();  // the previous partial's tiles are read
       named_barrier_sync(1, 128);
+      // columns 64 .. D-1 first (own staging tiles), then, once the dK product has stopped
+      // reading the dS tile, columns 0 .. 63 into it
 #pragma unroll 1
-      for (int c2 = 0; c2 < D / 64; ++c2) {
+      for (int k2 = 0; k2 < D / 64; ++k2) {
+        const int c2 = (k2 + 1) % (D / 64);
+        if (C::DQ_ALIASES_DP && c2 == 0) {
+          mbar_wait(BAR(B_DKDONE), (uint32_t)it & 1u, abort_flag, p.status);
+          tc_fence_after();
+        }
         uint32_t v[64];
         tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * c2, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
         tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * c2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
