@@ -250,28 +250,33 @@ __global__ void __launch_bounds__(512, 1)
       for (int it = 0; it < n_q; ++it) {
         const int s = it & 1;
         const int q0 = q_tile(it) * BM;
-        mbar_wait(BAR(B_QEMPTY + s), ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag, p.status);
-        // -LSE·log2(e) and D of the 128 query rows; rows past the sequence: -inf, 0.
-        float* vec = reinterpret_cast<float*>(sgen + C::OFF_VEC + s * 2 * BM * 4);
+        // -LSE·log2(e) and D of the 128 query rows (rows past the sequence: -inf, 0), read
+        // before the stage is free so that their latency overlaps the wait
+        float nl2[4], dd[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int qc = lane * 4 + e;
-          const int qg = q0 + qc;
-          float nl2 = -INFINITY, dd = 0.f;
+          const int qg = q0 + lane * 4 + e;
+          nl2[e] = -INFINITY;
+          dd[e] = 0.f;
           if (qg < Lq) {
             const size_t vi = (p.cu_q != nullptr) ? (size_t)h * p.total_q + q_row0 + qg
                                                   : ((size_t)bcoord * p.H + h) * p.N + qg;
-            nl2 = -p.lse[vi] * kLog2e;
-            dd = p.dvec[vi];
+            nl2[e] = -p.lse[vi] * kLog2e;
+            dd[e] = p.dvec[vi];
           }
-          vec[qc] = nl2;
-          vec[BM + qc] = dd;
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(BAR(B_QFULL + s), C::TILE);
+        mbar_wait(BAR(B_QEMPTY + s), ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag, p.status);
+        if (lane == 0) {  // the Q tile first; every lane arrives once its vector entries are written
+          mbar_expect_tx(BAR(B_QFULL + s), C::TILE);
           for (int c = 0; c < C::KCH; ++c)
             tma_load_4d(&tmQ, BAR(B_QFULL + s), sbase + C::OFF_Q + s * C::TILE + c * C::CHUNK,
                         c * 64, h, q_row0 + q0, bcoord);
+        }
+        float* vec = reinterpret_cast<float*>(sgen + C::OFF_VEC + s * 2 * BM * 4);
+        *reinterpret_cast<float4*>(&vec[lane * 4]) = make_float4(nl2[0], nl2[1], nl2[2], nl2[3]);
+        *reinterpret_cast<float4*>(&vec[BM + lane * 4]) = make_float4(dd[0], dd[1], dd[2], dd[3]);
+        mbar_arrive(BAR(B_QFULL + s));
+        if (lane == 0) {
           // a dO stage is free once the dV product of its previous step has read it
           const int ds_ = it % C::DO_ST;
           mbar_wait(BAR(B_DOEMPTY + ds_), ((uint32_t)(it / C::DO_ST) & 1u) ^ 1u, abort_flag,
@@ -280,8 +285,6 @@ __global__ void __launch_bounds__(512, 1)
           for (int c = 0; c < C::KCH; ++c)
             tma_load_4d(&tmDO, BAR(B_DOFULL + ds_), sbase + C::OFF_DO + ds_ * C::TILE + c * C::CHUNK,
                         c * 64, h, q_row0 + q0, bcoord);
-        } else {
-          mbar_arrive(BAR(B_QFULL + s));
         }
       }
     }
