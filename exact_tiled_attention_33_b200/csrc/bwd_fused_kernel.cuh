@@ -132,7 +132,7 @@ struct BwdFusedCfg {
   static constexpr int OFF_STG = OFF_DS + DS_TILE;       // 2 staging tiles
   static constexpr int OFF_VEC = OFF_STG + 2 * STG_TILE; // per Q stage: -lse*log2e [128], D [128]
   static constexpr int OFF_BAR = OFF_VEC + 2 * 2 * BM * 4;
-  static constexpr int NBAR = 18;
+  static constexpr int NBAR = 19;
   // The dynamic shared memory base is 1024-byte aligned on sm_100 (it follows the 1 KB the
   // driver reserves per CTA); the kernel checks that instead of reserving slack for it.
   static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16;
@@ -156,8 +156,8 @@ __global__ void __launch_bounds__(512, 1)
   using C = BwdFusedCfg<D>;
   constexpr int BM = C::BM, BN = C::BN;
   enum { B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_DOFULL = 5, B_DOEMPTY = 7, B_SFULL = 9, B_DPFULL, B_PFULL,
-         B_DSFULL, B_DQFULL, B_DQEMPTY, B_DONE, B_DSFREE, B_DKDONE };
-  static_assert(B_DKDONE < C::NBAR, "mbarrier slots");
+         B_DSFULL, B_DQFULL, B_DQEMPTY, B_DONE, B_DKDONE, B_DSFREE /* one per dS chunk */ };
+  static_assert(B_DSFREE + 1 < C::NBAR, "mbarrier slots");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase = smem_u32(smem_raw);
   if ((sbase & 1023u) != 0u) {  // the 128-byte swizzled tiles need 1024-byte atoms
@@ -171,8 +171,15 @@ __global__ void __launch_bounds__(512, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int h = blockIdx.y;
-  const int bz = blockIdx.z;
+  // grid: x = key tile, y = head, z = batch or sequence, launched in groups of heads that
+  // share L2 (their Q, dO and dQ sums; see grouped_tile_order), key tile 0 (the one that
+  // sees the most query tiles when causal) first
+#ifndef FATTN_BWD_HEAD_GROUP
+#define FATTN_BWD_HEAD_GROUP 4
+#endif
+  const GridItem item = grouped_tile_order(FATTN_BWD_HEAD_GROUP);
+  const int h = item.h;
+  const int bz = item.bz;
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
     if (!varlen_segment_ok(p.cu_q, p.cu_k, bz, p.total_q, p.total_k, p.max_seqlen_q,
@@ -188,7 +195,7 @@ __global__ void __launch_bounds__(512, 1)
     Lq = Lk = p.N;
     bcoord = bz;
   }
-  const int k0 = blockIdx.x * BN;
+  const int k0 = item.tile * BN;
   if (k0 >= Lk) return;
   const int diag = Lk - Lq;
   const int wl = p.win_left, wr = p.win_right;
@@ -196,7 +203,7 @@ __global__ void __launch_bounds__(512, 1)
   query_tile_range(k0, min(k0 + BN - 1, Lk - 1), Lq, diag, wl, wr, BM, &i_begin, &n_q);
   // Without a right bound every key tile starts at the same query tile: rotate the order per
   // key tile so that CTAs running together add into different dQ rows.
-  const int rot = (wr < 0 && n_q > 0) ? (int)(blockIdx.x % (unsigned)n_q) : 0;
+  const int rot = (wr < 0 && n_q > 0) ? item.tile % n_q : 0;
   auto q_tile = [&](int it) { int t = it + rot; if (t >= n_q) t -= n_q; return i_begin + t; };
   // token row of query 0 of this sequence in the dQ sums
   const long long acc_row0 = (p.cu_q != nullptr) ? (long long)q_row0 : (long long)bcoord * p.N;
@@ -219,6 +226,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_DQEMPTY), 128);
     mbar_init(BAR(B_DONE), 1);
     mbar_init(BAR(B_DSFREE), 1);
+    mbar_init(BAR(B_DSFREE + 1), 1);
     mbar_init(BAR(B_DKDONE), 1);
     *abort_flag = 0u;
     fence_barrier_init();
@@ -454,11 +462,9 @@ __global__ void __launch_bounds__(512, 1)
       tmem_wait_ld();
       reg_fence(dv);
       const float4* d4 = reinterpret_cast<const float4*>(&vec[BM + cbase]);
-      if (C::DQ_ALIASES_DP && it > 0)  // the previous dQ partial's staging in this tile is read
-        mbar_wait(BAR(B_DSFREE), (uint32_t)(it - 1) & 1u, abort_flag, p.status);
+      uint32_t w[8][4];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {  // 16-byte unit u = queries cbase + 8u .. + 7
-        uint32_t w[4];
 #pragma unroll
         for (int e2 = 0; e2 < 2; ++e2) {
           const int e4 = 2 * u + e2;
@@ -471,11 +477,18 @@ __global__ void __launch_bounds__(512, 1)
           const float2 db = f2_unpack(f2_mul(f2_add(f2_pack(__uint_as_float(dv[4 * e4 + 2]), __uint_as_float(dv[4 * e4 + 3])),
                                                     f2_pack(-dd.z, -dd.w)),
                                              f2_pack(pb.x, pb.y)));
-          w[2 * e2] = pack2<BF16>(da.x, da.y);
-          w[2 * e2 + 1] = pack2<BF16>(db.x, db.y);
+          w[u][2 * e2] = pack2<BF16>(da.x, da.y);
+          w[u][2 * e2 + 1] = pack2<BF16>(db.x, db.y);
         }
-        *reinterpret_cast<uint4*>(ds_row + ((u ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
+      // this warpgroup's chunk of the tile held the previous dQ partial's staging: wait until
+      // its reduce-add has read it
+      if (C::DQ_ALIASES_DP && it > 0)
+        mbar_wait(BAR(B_DSFREE + half), (uint32_t)(it - 1) & 1u, abort_flag, p.status);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4*>(ds_row + ((u ^ (r & 7)) << 4)) =
+            make_uint4(w[u][0], w[u][1], w[u][2], w[u][3]);
       fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
       tc_fence_before();
       mbar_arrive(BAR(B_DSFULL));
@@ -521,7 +534,8 @@ __global__ void __launch_bounds__(512, 1)
     // per staging tile.  The TMA unit skips rows past the sums' end; rows of this tile past
     // the sequence carry zeros (their P is 0).  At D = 128 staging tiles 0 and 1 are the dS
     // tile (the dK and dQ products, its readers, completed before the partial was final); the
-    // next dS waits until those reduce-adds have read them (B_DSFREE).
+    // next dS waits until those reduce-adds have read them (B_DSFREE, one per 64-query chunk
+    // of the tile, which is one compute warpgroup's).
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -575,8 +589,10 @@ __global__ void __launch_bounds__(512, 1)
           bulk_commit_group();
         }
         if constexpr (C::DQ_ALIASES_DP) {
-          bulk_wait_group_read2();  // the two reduce-adds from the dS tile have read it
+          bulk_wait_group_read3();  // the reduce-add from dS chunk 0 has read it
           mbar_arrive(BAR(B_DSFREE));
+          bulk_wait_group_read2();  // and the one from chunk 1
+          mbar_arrive(BAR(B_DSFREE + 1));
         }
       }
     }

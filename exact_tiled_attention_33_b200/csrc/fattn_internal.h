@@ -96,6 +96,33 @@ __host__ __device__ inline void query_tile_range(int k_first, int k_last, int Lq
   }
 }
 
+// Work item of the CTA with linear launch index L = x + T (y + H z) on a (T tiles, H heads,
+// HB / H batches) grid, in launch order: the (batch, head) pairs are taken `group` at a time,
+// and within a group tile-major (tile 0 of each of its heads, then tile 1, ...).  The hardware
+// starts CTAs roughly in linear order, so the heads of a group share L2 while they run, and
+// the heaviest tiles of the last group start together with the rest of it instead of after
+// every other CTA has been handed out.  A bijection of [0, T * HB) onto (tile, h, bz).
+struct GridItem {
+  int tile, h, bz;
+};
+__host__ __device__ inline GridItem grouped_grid_item(unsigned long long L, unsigned long long T,
+                                                      unsigned long long H,
+                                                      unsigned long long HB,
+                                                      unsigned long long group) {
+  const unsigned long long first = L / (group * T) * group;  // first (batch, head) of the group
+  const unsigned long long gn = group < HB - first ? group : HB - first;  // pairs in the group
+  const unsigned long long i = L - first * T;                 // < gn * T
+  const unsigned long long hb = first + i % gn;
+  return {(int)(i / gn), (int)(hb % H), (int)(hb / H)};
+}
+#ifdef __CUDACC__
+__device__ inline GridItem grouped_tile_order(unsigned group) {
+  const unsigned long long T = gridDim.x, H = gridDim.y;
+  return grouped_grid_item(blockIdx.x + T * (blockIdx.y + H * blockIdx.z), T, H,
+                           H * gridDim.z, group);
+}
+#endif
+
 // KV-cache decode parameters (see decode_kernel.cuh).
 constexpr int kDecodeMaxQueries = 16;  // query rows per sequence in one decode call
 struct DecParams {

@@ -117,12 +117,16 @@ __global__ void __launch_bounds__(384, 1)
   const int lane = threadIdx.x & 31;
 
   // ---------------------------------------------------------------- work item
-  // grid: x = query tile (fastest, so the CTAs running together share one head's K/V in
-  // L2), y = head, z = batch or sequence; when causal the tile with the most key tiles of
-  // each head is launched first.
-  const int h = blockIdx.y;
-  const int bz = blockIdx.z;
-  const int tile = p.reverse_tiles ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  // grid: x = query tile, y = head, z = batch or sequence, launched in groups of heads that
+  // share L2 (see grouped_tile_order); when causal the tile with the most key tiles of each
+  // head comes first.
+#ifndef FATTN_FWD_HEAD_GROUP
+#define FATTN_FWD_HEAD_GROUP 4
+#endif
+  const GridItem item = grouped_tile_order(FATTN_FWD_HEAD_GROUP);
+  const int h = item.h;
+  const int bz = item.bz;
+  const int tile = p.reverse_tiles ? (int)(gridDim.x - 1) - item.tile : item.tile;
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
     if (!varlen_segment_ok(p.cu_q, p.cu_k, bz, p.total_q, p.total_k, p.max_seqlen_q, -1,

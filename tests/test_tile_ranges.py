@@ -96,3 +96,34 @@ def test_tile_ranges_at_kernel_sizes(shim):
             want = {int(i) // T for i in np.nonzero(full[:, k0:k1 + 1].any(axis=1))[0]}
             assert _call(shim.shim_query_tile_range, k0, k1, Lq, diag, *win, T) == want
 
+
+
+def _grid_item(shim, L, T, H, HB, group):
+    f = shim.shim_grouped_grid_item
+    f.argtypes = [ctypes.c_ulonglong] * 5 + [ctypes.POINTER(ctypes.c_int)]
+    f.restype = None
+    out = (ctypes.c_int * 3)(-1, -1, -1)
+    f(L, T, H, HB, group, out)
+    return tuple(out)
+
+
+@pytest.mark.parametrize("T,H,B,group", [(1, 1, 1, 4), (3, 2, 1, 4), (5, 3, 3, 4), (4, 7, 2, 2),
+                                         (2, 5, 1, 1), (128, 32, 2, 4), (8, 16, 8, 4),
+                                         (6, 1, 9, 4)])
+def test_launch_order_is_a_grouped_tile_major_bijection(shim, T, H, B, group):
+    """The forward and the fused backward map a CTA's linear launch index to (tile, head,
+    batch) with `grouped_grid_item`: every work item exactly once; groups of `group`
+    consecutive (batch, head) pairs (the last one possibly smaller) one after the other; and
+    inside a group tile 0 of each of its pairs first, then tile 1, and so on."""
+    HB = H * B
+    items = [_grid_item(shim, L, T, H, HB, group) for L in range(T * HB)]
+    assert sorted(items) == sorted((t, h, b) for t in range(T) for h in range(H)
+                                   for b in range(B))
+    L = 0
+    for first in range(0, HB, group):
+        pairs = list(range(first, min(first + group, HB)))
+        for t in range(T):
+            for hb in pairs:
+                assert items[L] == (t, hb % H, hb // H), (L, items[L])
+                L += 1
+    assert L == T * HB
