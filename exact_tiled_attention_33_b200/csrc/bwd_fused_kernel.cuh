@@ -138,6 +138,11 @@ struct BwdFusedCfg {
   static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16;
   static_assert(SMEM <= 232448, "shared memory per CTA");
   static constexpr int THREADS = 512;
+#ifndef FATTN_BWD_POLY_QUADS
+#define FATTN_BWD_POLY_QUADS 4
+#endif
+  // of the 16 groups of 4 exponentials per thread and step, those taken by exp2_poly2
+  static constexpr int kPolyQuads = FATTN_BWD_POLY_QUADS;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DK = 256, TM_DV = 256 + D;
   // the dQ partial: over dPᵀ at D = 128 (then the next dPᵀ waits for the drain)
@@ -431,10 +436,18 @@ __global__ void __launch_bounds__(512, 1)
                                            c2, f2_pack(nl.x, nl.y)));
         const float2 x1 = f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[4 * e4 + 2]), __uint_as_float(sv[4 * e4 + 3])),
                                            c2, f2_pack(nl.z, nl.w)));
-        pv[4 * e4] = ex2_approx(x0.x);
-        pv[4 * e4 + 1] = ex2_approx(x0.y);
-        pv[4 * e4 + 2] = ex2_approx(x1.x);
-        pv[4 * e4 + 3] = ex2_approx(x1.y);
+        if (e4 < C::kPolyQuads) {  // on the FMA pipe, beside the special-function unit
+          const float2 y0 = exp2_poly2(x0.x, x0.y), y1 = exp2_poly2(x1.x, x1.y);
+          pv[4 * e4] = y0.x;
+          pv[4 * e4 + 1] = y0.y;
+          pv[4 * e4 + 2] = y1.x;
+          pv[4 * e4 + 3] = y1.y;
+        } else {
+          pv[4 * e4] = ex2_approx(x0.x);
+          pv[4 * e4 + 1] = ex2_approx(x0.y);
+          pv[4 * e4 + 2] = ex2_approx(x1.x);
+          pv[4 * e4 + 3] = ex2_approx(x1.y);
+        }
       }
       if (need_mask) {
         const int lo = key_ok ? max(qmin, 0) - cbase : 64;
