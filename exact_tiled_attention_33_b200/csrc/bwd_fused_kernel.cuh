@@ -22,10 +22,10 @@
 // LSE and D; dO one stage), warp 1 issues every tcgen05.mma from one thread, warps 4-11 are
 // two compute warpgroups (thread = key row, one half of the 128 query columns each: Pᵀ into
 // tensor memory, dSᵀ into shared memory), warps 12-15 drain each dQ partial from tensor
-// memory into the fp32 sums (thread = query row) while the compute warps move on: the whole
-// partial goes into swizzled shared-memory staging tiles of 32 columns (at D = 128 two of them
-// lie in the dS tile, free from the dQ product until the next dS), tensor memory is released,
-// and one thread hands the tiles to the TMA unit as reduce-adds into the sums.
+// memory into the fp32 sums (thread = query row) while the compute warps move on: 32 columns
+// at a time go through two swizzled shared-memory staging tiles, which one thread hands to
+// the TMA unit as reduce-adds into the sums; what does not fit in the tiles at once waits in
+// registers, so tensor memory is released after one pass over the partial.
 // Tensor memory: Sᵀ/Pᵀ [0,128) | dPᵀ [128,256) | dK [256,256+D) | dV [256+D,256+2D); the dQ
 // partial (128 query lanes x D columns) takes the dPᵀ columns at D = 128 (free once the
 // compute warps have loaded dPᵀ; the next dPᵀ waits for the drain) and columns [384,448) at
@@ -132,7 +132,7 @@ struct BwdFusedCfg {
   static constexpr int OFF_STG = OFF_DS + DS_TILE;       // 2 staging tiles
   static constexpr int OFF_VEC = OFF_STG + 2 * STG_TILE; // per Q stage: -lse*log2e [128], D [128]
   static constexpr int OFF_BAR = OFF_VEC + 2 * 2 * BM * 4;
-  static constexpr int NBAR = 19;
+  static constexpr int NBAR = 16;
   // The dynamic shared memory base is 1024-byte aligned on sm_100 (it follows the 1 KB the
   // driver reserves per CTA); the kernel checks that instead of reserving slack for it.
   static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16;
@@ -161,8 +161,8 @@ __global__ void __launch_bounds__(512, 1)
   using C = BwdFusedCfg<D>;
   constexpr int BM = C::BM, BN = C::BN;
   enum { B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_DOFULL = 5, B_DOEMPTY = 7, B_SFULL = 9, B_DPFULL, B_PFULL,
-         B_DSFULL, B_DQFULL, B_DQEMPTY, B_DONE, B_DKDONE, B_DSFREE /* one per dS chunk */ };
-  static_assert(B_DSFREE + 1 < C::NBAR, "mbarrier slots");
+         B_DSFULL, B_DQFULL, B_DQEMPTY, B_DONE };
+  static_assert(B_DONE < C::NBAR, "mbarrier slots");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase = smem_u32(smem_raw);
   if ((sbase & 1023u) != 0u) {  // the 128-byte swizzled tiles need 1024-byte atoms
@@ -230,9 +230,6 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_DQFULL), 1);
     mbar_init(BAR(B_DQEMPTY), 128);
     mbar_init(BAR(B_DONE), 1);
-    mbar_init(BAR(B_DSFREE), 1);
-    mbar_init(BAR(B_DSFREE + 1), 1);
-    mbar_init(BAR(B_DKDONE), 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
@@ -381,7 +378,6 @@ __global__ void __launch_bounds__(512, 1)
           mma_ss(tmem + C::TM_DK, sdesc_adv(dSk, (kk >> 2) * C::CHUNK + (kk & 3) * 32),
                  sdesc_adv(qm, kk * 2048), ID_DK, (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(BAR(B_QEMPTY + s));
-        mma_commit(BAR(B_DKDONE));  // the dS tile is no longer read by this step's products
         if (it + 1 < n_q) {
           if constexpr (C::DQ_ALIASES_DP) {
             // the next dPᵀ overwrites this dQ partial: wait until it has been drained
@@ -475,9 +471,9 @@ __global__ void __launch_bounds__(512, 1)
       tmem_wait_ld();
       reg_fence(dv);
       const float4* d4 = reinterpret_cast<const float4*>(&vec[BM + cbase]);
-      uint32_t w[8][4];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {  // 16-byte unit u = queries cbase + 8u .. + 7
+        uint32_t w[4];
 #pragma unroll
         for (int e2 = 0; e2 < 2; ++e2) {
           const int e4 = 2 * u + e2;
@@ -490,18 +486,11 @@ __global__ void __launch_bounds__(512, 1)
           const float2 db = f2_unpack(f2_mul(f2_add(f2_pack(__uint_as_float(dv[4 * e4 + 2]), __uint_as_float(dv[4 * e4 + 3])),
                                                     f2_pack(-dd.z, -dd.w)),
                                              f2_pack(pb.x, pb.y)));
-          w[u][2 * e2] = pack2<BF16>(da.x, da.y);
-          w[u][2 * e2 + 1] = pack2<BF16>(db.x, db.y);
+          w[2 * e2] = pack2<BF16>(da.x, da.y);
+          w[2 * e2 + 1] = pack2<BF16>(db.x, db.y);
         }
+        *reinterpret_cast<uint4*>(ds_row + ((u ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      // this warpgroup's chunk of the tile held the previous dQ partial's staging: wait until
-      // its reduce-add has read it
-      if (C::DQ_ALIASES_DP && it > 0)
-        mbar_wait(BAR(B_DSFREE + half), (uint32_t)(it - 1) & 1u, abort_flag, p.status);
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        *reinterpret_cast<uint4*>(ds_row + ((u ^ (r & 7)) << 4)) =
-            make_uint4(w[u][0], w[u][1], w[u][2], w[u][3]);
       fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
       tc_fence_before();
       mbar_arrive(BAR(B_DSFULL));
@@ -541,71 +530,70 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp >= 12) {
     // ============================================================ dQ drain
-    // thread = query row (tensor-memory lane) of the partial.  The partial is copied, 64
-    // columns at a time, into staging tiles of 32 columns (128-byte swizzle, the layout of the
-    // tensor map's box); tensor memory is released; then one thread issues a TMA reduce-add
-    // per staging tile.  The TMA unit skips rows past the sums' end; rows of this tile past
-    // the sequence carry zeros (their P is 0).  At D = 128 staging tiles 0 and 1 are the dS
-    // tile (the dK and dQ products, its readers, completed before the partial was final); the
-    // next dS waits until those reduce-adds have read them (B_DSFREE, one per 64-query chunk
-    // of the tile, which is one compute warpgroup's).
+    // thread = query row (tensor-memory lane) of the partial; 32 columns at a time go through
+    // two alternating shared-memory staging tiles (128-byte swizzle, the layout of the tensor
+    // map's box) and one thread issues a TMA reduce-add per tile into the fp32 sums.  The
+    // first two column groups are staged straight away (the tiles' previous reduce-adds, a
+    // step ago, have read them by then), the rest is held in registers, so that the tensor
+    // memory is released after one pass over it.  The TMA unit skips rows past the sums'
+    // end; rows of this tile past the sequence carry zeros (their P is 0).
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const bool leader = threadIdx.x == 12 * 32;  // issues and waits for the reduce-adds
-    auto stage_off = [&](int c) -> uint32_t {   // staging tile of columns 32c .. 32c+31
-      if constexpr (C::DQ_ALIASES_DP)
-        return c < 2 ? (uint32_t)(C::OFF_DS + c * C::STG_TILE) : (uint32_t)(C::OFF_STG + (c - 2) * C::STG_TILE);
-      else
-        return (uint32_t)(C::OFF_STG + c * C::STG_TILE);
+    constexpr int NG = D / 32;                   // 32-column groups
+    constexpr int NS = 2;                        // staging tiles = groups staged at once
+    auto stage = [&](int c, const uint32_t (&g)[32]) {  // one group into tile c % NS
+      uint8_t* row_ptr = sgen + C::OFF_STG + (c % NS) * C::STG_TILE + r * 128;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4*>(row_ptr + ((u ^ (r & 7)) << 4)) =
+            make_uint4(g[4 * u], g[4 * u + 1], g[4 * u + 2], g[4 * u + 3]);
+    };
+    auto issue = [&](int c, int q0) {  // after the group's tile is complete
+      fence_proxy_async_smem();
+      named_barrier_sync(1, 128);
+      if (leader) {
+        tma_reduce_add_4d(&tmDQ, sbase + C::OFF_STG + (c % NS) * C::STG_TILE, 32 * c, h,
+                          (int)(acc_row0 + q0), 0);
+        bulk_commit_group();
+      }
     };
     if (leader) tma_prefetch_desc(&tmDQ);
     for (int it = 0; it < n_q; ++it) {
       const int q0 = q_tile(it) * BM;
       mbar_wait(BAR(B_DQFULL), (uint32_t)it & 1u, abort_flag, p.status);
       tc_fence_after();
-      if (leader && it > 0) bulk_wait_group_read0();  // the previous partial's tiles are read
+      if (leader) bulk_wait_group_read0();  // the previous partial's tiles have been read
       named_barrier_sync(1, 128);
-      // columns 64 .. D-1 first (own staging tiles), then, once the dK product has stopped
-      // reading the dS tile, columns 0 .. 63 into it
-#pragma unroll 1
-      for (int k2 = 0; k2 < D / 64; ++k2) {
-        const int c2 = (k2 + 1) % (D / 64);
-        if (C::DQ_ALIASES_DP && c2 == 0) {
-          mbar_wait(BAR(B_DKDONE), (uint32_t)it & 1u, abort_flag, p.status);
-          tc_fence_after();
-        }
-        uint32_t v[64];
-        tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * c2, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * c2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+#pragma unroll
+      for (int c = 0; c < NS; ++c) {  // staged straight away
+        uint32_t g[32];
+        tmem_ld32(tmem + lane_off + C::TM_DQ + 32 * c, g);
         tmem_wait_ld();
-        reg_fence(v);
+        reg_fence(g);
+        stage(c, g);
+      }
+      uint32_t held[NG > NS ? NG - NS : 1][32];  // held in registers until a tile is free
+      if constexpr (NG > NS) {
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint8_t* row_ptr = sgen + stage_off(2 * c2 + h2) + r * 128;
+        for (int c = NS; c < NG; ++c) tmem_ld32(tmem + lane_off + C::TM_DQ + 32 * c, held[c - NS]);
+        tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(row_ptr + ((u ^ (r & 7)) << 4)) =
-                make_uint4(v[32 * h2 + 4 * u], v[32 * h2 + 4 * u + 1], v[32 * h2 + 4 * u + 2],
-                           v[32 * h2 + 4 * u + 3]);
-        }
+        for (int c = NS; c < NG; ++c) reg_fence(held[c - NS]);
       }
       // the partial has been read: the next dPᵀ may overwrite its tensor-memory columns
       tc_fence_before();
       mbar_arrive(BAR(B_DQEMPTY));
-      fence_proxy_async_smem();
-      named_barrier_sync(1, 128);
-      if (leader) {
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          tma_reduce_add_4d(&tmDQ, sbase + stage_off(c), 32 * c, h, (int)(acc_row0 + q0), 0);
-          bulk_commit_group();
-        }
-        if constexpr (C::DQ_ALIASES_DP) {
-          bulk_wait_group_read3();  // the reduce-add from dS chunk 0 has read it
-          mbar_arrive(BAR(B_DSFREE));
-          bulk_wait_group_read2();  // and the one from chunk 1
-          mbar_arrive(BAR(B_DSFREE + 1));
+#pragma unroll
+      for (int c = 0; c < NS; ++c) issue(c, q0);
+      if constexpr (NG > NS) {
+#pragma unroll
+        for (int c = NS; c < NG; ++c) {
+          if (leader) bulk_wait_group_read1();  // tile c % NS: its reduce-add has read it
+          named_barrier_sync(1, 128);
+          stage(c, held[c - NS]);
+          issue(c, q0);
         }
       }
     }

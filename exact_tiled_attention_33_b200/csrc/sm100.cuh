@@ -186,11 +186,8 @@ __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, uint32
       : "memory");
 }
 // Wait until at most two of this thread's bulk groups are still reading shared memory.
-__device__ __forceinline__ void bulk_wait_group_read3() {
-  asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_group_read2() {
-  asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
+__device__ __forceinline__ void bulk_wait_group_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
