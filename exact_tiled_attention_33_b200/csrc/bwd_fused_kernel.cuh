@@ -542,7 +542,13 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const bool leader = threadIdx.x == 12 * 32;  // issues and waits for the reduce-adds
     constexpr int NG = D / 32;                   // 32-column groups
-    constexpr int NS = 2;                        // staging tiles = groups staged at once
+    constexpr int NS = 2;                        // staging tiles
+#ifndef FATTN_BWD_DRAIN_FIRST
+#define FATTN_BWD_DRAIN_FIRST 2
+#endif
+    // groups staged before the tensor memory is released; the others wait in registers
+    constexpr int NF = FATTN_BWD_DRAIN_FIRST < NG ? FATTN_BWD_DRAIN_FIRST : NG;
+    static_assert(NF >= 1 && NF <= NS, "drain staging");
     auto stage = [&](int c, const uint32_t (&g)[32]) {  // one group into tile c % NS
       uint8_t* row_ptr = sgen + C::OFF_STG + (c % NS) * C::STG_TILE + r * 128;
 #pragma unroll
@@ -567,32 +573,33 @@ __global__ void __launch_bounds__(512, 1)
       if (leader) bulk_wait_group_read0();  // the previous partial's tiles have been read
       named_barrier_sync(1, 128);
 #pragma unroll
-      for (int c = 0; c < NS; ++c) {  // staged straight away
+      for (int c = 0; c < NF; ++c) {  // staged straight away
         uint32_t g[32];
         tmem_ld32(tmem + lane_off + C::TM_DQ + 32 * c, g);
         tmem_wait_ld();
         reg_fence(g);
         stage(c, g);
       }
-      uint32_t held[NG > NS ? NG - NS : 1][32];  // held in registers until a tile is free
-      if constexpr (NG > NS) {
+      uint32_t held[NG > NF ? NG - NF : 1][32];  // held in registers until a tile is free
+      if constexpr (NG > NF) {
 #pragma unroll
-        for (int c = NS; c < NG; ++c) tmem_ld32(tmem + lane_off + C::TM_DQ + 32 * c, held[c - NS]);
+        for (int c = NF; c < NG; ++c) tmem_ld32(tmem + lane_off + C::TM_DQ + 32 * c, held[c - NF]);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = NS; c < NG; ++c) reg_fence(held[c - NS]);
+        for (int c = NF; c < NG; ++c) reg_fence(held[c - NF]);
       }
       // the partial has been read: the next dPᵀ may overwrite its tensor-memory columns
       tc_fence_before();
       mbar_arrive(BAR(B_DQEMPTY));
 #pragma unroll
-      for (int c = 0; c < NS; ++c) issue(c, q0);
-      if constexpr (NG > NS) {
+      for (int c = 0; c < NF; ++c) issue(c, q0);
+      if constexpr (NG > NF) {
 #pragma unroll
-        for (int c = NS; c < NG; ++c) {
-          if (leader) bulk_wait_group_read1();  // tile c % NS: its reduce-add has read it
+        for (int c = NF; c < NG; ++c) {
+          // tile c % NS: from the step's start it was free; reused, its reduce-add has read it
+          if (c >= NS && leader) bulk_wait_group_read1();
           named_barrier_sync(1, 128);
-          stage(c, held[c - NS]);
+          stage(c, held[c - NF]);
           issue(c, q0);
         }
       }
