@@ -64,11 +64,28 @@ static LaunchResult launch_bwd_fused_t(const CUtensorMap& tmQ, const CUtensorMap
   fa_bwd_pre_acc_kernel<D, BF16><<<(unsigned)pre_blocks, 256, 0, stream>>>(p, q_rows);
   // 2) dK, dV and the dQ partial sums: one CTA per key tile
   dim3 grid((max_seqlen_k + C::BN - 1) / C::BN, p.H, batches);
-  fa_bwd_fused_kernel<D, BF16><<<grid, C::THREADS, C::SMEM, stream>>>(tmQ, tmK, tmV, tmDO, tmDQ, p);
+  //    (a programmatic dependent of the preprocess: see grid_dependency_wait in the kernel)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, fa_bwd_fused_kernel<D, BF16>, tmQ, tmK, tmV, tmDO, tmDQ, p);
+  if (e != cudaSuccess) return launch_status(e);
   // 3) dQ = scale * sums, rounded to 16 bits
   const long long elems = q_rows * p.H * D;
   const long long cv_blocks = std::min<long long>((elems / 8 + 255) / 256, (long long)sms * 16);
-  fa_bwd_dq_convert_kernel<BF16><<<(unsigned)cv_blocks, 256, 0, stream>>>(p, elems);
+  //    (a programmatic dependent of the fused pass)
+  cfg.gridDim = dim3((unsigned)cv_blocks);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  e = cudaLaunchKernelEx(&cfg, fa_bwd_dq_convert_kernel<BF16>, p, elems);
+  if (e != cudaSuccess) return launch_status(e);
   return launch_status(cudaGetLastError());
 }
 

@@ -47,6 +47,9 @@ namespace fattn {
 // D fp32 dQ sums set to 0.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_pre_acc_kernel(const BwdParams p, long long rows_total) {
+  // the fused pass is launched as a programmatic dependent of this kernel: its CTAs may start
+  // (setup, K and V loads) while this one runs, and wait for its results where they use them
+  grid_dependents_launch();
   constexpr int PER = D / 32;  // elements per lane
   const long long warps = (long long)gridDim.x * (blockDim.x / 32);
   const int lane = threadIdx.x & 31;
@@ -98,6 +101,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_acc_kernel(const BwdParams p, 
 // each thread converts 8 consecutive elements (two float4 reads, one 16-byte write).
 template <bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const BwdParams p, long long elems) {
+  grid_dependency_wait();  // a programmatic dependent of the fused pass: its sums are complete
   const long long n8 = elems >> 3;  // D is a multiple of 8
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
        i += (long long)gridDim.x * blockDim.x) {
@@ -169,6 +173,9 @@ __global__ void __launch_bounds__(512, 1)
     if (threadIdx.x == 0) atomicOr(p.status, kDevSmemAlign);
     return;
   }
+  // the dQ conversion may be scheduled once every CTA of this grid has started (it waits for
+  // this grid's completion before reading the sums)
+  grid_dependents_launch();
   uint8_t* sgen = smem_raw;
   auto BAR = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + C::OFF_BAR + 8 * C::NBAR);
@@ -257,6 +264,7 @@ __global__ void __launch_bounds__(512, 1)
           tma_load_4d(&tmV, BAR(B_KV), sbase + C::OFF_V + c * C::CHUNK, c * 64, h, k_row0 + k0, bcoord);
         }
       }
+      grid_dependency_wait();  // D comes from the preceding preprocess launch
       for (int it = 0; it < n_q; ++it) {
         const int s = it & 1;
         const int q0 = q_tile(it) * BM;
@@ -566,6 +574,7 @@ __global__ void __launch_bounds__(512, 1)
       }
     };
     if (leader) tma_prefetch_desc(&tmDQ);
+    grid_dependency_wait();  // the sums are zeroed by the preceding preprocess launch
     for (int it = 0; it < n_q; ++it) {
       const int q0 = q_tile(it) * BM;
       mbar_wait(BAR(B_DQFULL), (uint32_t)it & 1u, abort_flag, p.status);

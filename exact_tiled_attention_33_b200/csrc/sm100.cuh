@@ -120,6 +120,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   return mbar_wait_limit(bar, parity, abort_flag, status, FATTN_WAIT_LIMIT_NS);
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// In a kernel launched with programmatic stream serialisation: wait until the preceding
+// kernel in the stream has completed and its memory writes are visible (a no-op otherwise).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// In the preceding kernel: allow the dependent launch to begin before this one completes.
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ register reallocation
 // Executed by every warp of a warpgroup.  The sum over warpgroups must stay within the
 // registers the CTA was launched with (threads x registers per thread at launch).
