@@ -73,7 +73,7 @@ struct FwdCfg {
   // a score carries half the tensor work of d = 128 for the same exponential, so a larger
   // share moves to the FMA pipe there.
 #ifndef FATTN_POLY_PAIRS
-#define FATTN_POLY_PAIRS 2
+#define FATTN_POLY_PAIRS 4
 #endif
 #ifndef FATTN_POLY_PAIRS_D64
 #define FATTN_POLY_PAIRS_D64 6
