@@ -360,13 +360,9 @@ __global__ void __launch_bounds__(512, 1)
                  sdesc_adv(dDOm, (it % C::DO_ST) * C::TILE + kk * 2048),
                  ID_DV, (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(BAR(B_DOEMPTY + it % C::DO_ST));
-        if (it + 1 < n_q) {  // Sᵀ of the next step over Pᵀ (in order after the dV product)
-          wait_q(it + 1);
-          issue_kt(C::TM_S, dK, sdesc_adv(dQk, (it + 1 & 1) * C::TILE));
-          mma_commit(BAR(B_SFULL));
-        }
         // dQ  = dS K   (A = dS [queries][keys], the dSᵀ tile read MN-major; B = K [keys][d]
-        //              MN-major), first, so that its drain overlaps the dK product
+        //              MN-major), first, so that its drain overlaps the next Sᵀ and the dK
+        //              product
         // dK += dSᵀ Q  (A = dSᵀ [keys][queries] K-major; B = Q [queries][d] MN-major)
         mbar_wait(BAR(B_DSFULL), ph, abort_flag, p.status);
         tc_fence_after();
@@ -380,6 +376,11 @@ __global__ void __launch_bounds__(512, 1)
           mma_ss(tmem + C::TM_DQ, sdesc_adv(dSm, kk * 2048), sdesc_adv(dKm, kk * 2048), ID_DQ,
                  kk > 0 ? 1u : 0u);
         mma_commit(BAR(B_DQFULL));
+        if (it + 1 < n_q) {  // Sᵀ of the next step over Pᵀ, between the dQ and dK products
+          wait_q(it + 1);
+          issue_kt(C::TM_S, dK, sdesc_adv(dQk, (it + 1 & 1) * C::TILE));
+          mma_commit(BAR(B_SFULL));
+        }
         const uint64_t qm = sdesc_adv(dQm, s * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
