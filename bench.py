@@ -644,7 +644,9 @@ def run_fattn(args, w):
             sets.append((ins, outs, hout, wsb))
         h2d = sum(x.numel() * x.element_size() for x in hin)
         d2h = sum(x.numel() * x.element_size() for x in sets[0][2])
-        e2e_steps = max(4, min(args.steps, 8))
+        # steady-state throughput of the pipeline: enough steps that its fill (the first
+        # step's inputs) and drain (the last step's outputs) are a small share of the region
+        e2e_steps = max(16, min(2 * args.steps, 48))
         s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_cmp = [torch.cuda.Event() for _ in range(2)]
