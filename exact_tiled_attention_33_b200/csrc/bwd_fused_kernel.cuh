@@ -14,6 +14,11 @@
 //                           that row's fp32 dQ sums
 //   fa_bwd_fused_kernel     the pass above
 //   fa_bwd_dq_convert_kernel dQ = scale · sums, rounded to 16 bits
+// launched in that order, each of the last two as a programmatic dependent of the one before
+// (its CTAs may start early and wait for the preceding kernel only where they read its
+// results).  CTAs of the pass run in groups of four (batch, head) pairs, tile-major inside a
+// group (grouped_grid_item), each head's key tile 0 (the one with most query tiles when
+// causal) first.
 // dK and dV are written once per key tile (deterministic); the dQ sums are fp32 atomic adds
 // whose order varies from run to run (the two-pass backward in bwd_kernel.cuh is the
 // bitwise-reproducible alternative).
