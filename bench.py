@@ -251,7 +251,14 @@ def oracle_sample_seconds(w, rows: int, head=(0, 0)):
     if key not in _HEAD_CACHE:
         t = wl.generate(w)
         b, h = head
-        _HEAD_CACHE[key] = tuple(wl.to_f64(t[x][b, :, h].clone()) for x in ("q", "k", "v", "do"))
+        if w.varlen:  # the longest packed sequence stands for the head's problem
+            cu = w.cu_seqlens()
+            seg = int(np.argmax(np.diff(cu)))
+            rs = slice(int(cu[seg]), int(cu[seg + 1]))
+            _HEAD_CACHE[key] = tuple(wl.to_f64(t[x][rs, h].clone()) for x in ("q", "k", "v", "do"))
+        else:
+            _HEAD_CACHE[key] = tuple(wl.to_f64(t[x][b, :, h].clone())
+                                     for x in ("q", "k", "v", "do"))
     q, k, v, do = _HEAD_CACHE[key]
     N = q.shape[0]
     r0 = N - rows
@@ -295,10 +302,11 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     # size the per-step sample so a step takes about a second on this host
-    rows = 64
+    seq = max(w.seqlens) if w.varlen else w.N
+    rows = min(64, seq)
     dt, _, _ = oracle_sample_seconds(w, rows)
-    while dt < 0.5 and rows < w.N:
-        rows = min(w.N, rows * 2)
+    while dt < 0.5 and rows < seq:
+        rows = min(seq, rows * 2)
         dt, _, _ = oracle_sample_seconds(w, rows)
     for _ in range(args.warmup):
         oracle_sample_seconds(w, rows)
@@ -309,8 +317,9 @@ def run_reference(args, w):
         total_t += dt
         total_f += fl
     value = total_f / total_t / 1e12
-    sample = (f"last {rows} query rows of head (b=0,h=0) of {w.name} against all "
-              f"{w.N} keys, fp64 oracle fwd+bwd, per step")
+    where = ("head 0 of the longest packed sequence" if w.varlen else "head (b=0,h=0)")
+    sample = (f"last {rows} query rows of {where} of {w.name} against all "
+              f"{seq} keys, fp64 oracle fwd+bwd, per step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
@@ -514,6 +523,8 @@ def run_fattn(args, w):
                                 device_id=dev)
     lib = _lib.load()
     split_heads = getattr(args, "split", "none") == "heads"
+    if w.varlen and (split_heads or w.window is not None):
+        raise SystemExit("a packed (varlen) workload runs without --split heads or a window")
     if split_heads:
         # one shared problem (same seed on every rank), its heads split over the ranks; each
         # step ends with an all-gather of O along the head dimension
@@ -526,19 +537,43 @@ def run_fattn(args, w):
         # each rank owns an independent problem of the same size (its own seed)
         wr = wl.Workload(**{**w.__dict__, "seed": w.seed + rank})
         host = wl.generate(wr)
-    B, N, H, d = wr.B, wr.N, host["q"].shape[2], wr.d
     scale, causal = wr.softmax_scale, int(wr.causal)
     dtype = _lib.FA_BF16 if wr.dtype == "bf16" else _lib.FA_FP16
     q, k, v, do = (host[x].to(dev) for x in ("q", "k", "v", "do"))
     o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    if wr.varlen:
+        # packed sequences [total, H, d] through fa_varlen_fwd / fa_varlen_bwd
+        H, d = host["q"].shape[1], wr.d
+        T, S, L = wr.total, len(wr.seqlens), max(wr.seqlens)
+        cu = host["cu_seqlens"].to(device=dev, dtype=torch.int32)
+        lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+
+        def new_ws():
+            return fa.varlen_bwd_workspace(T, H, d, dev)
+    else:
+        B, N, H, d = wr.B, wr.N, host["q"].shape[2], wr.d
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+
+        def new_ws():
+            return fa.bwd_workspace(B, N, H, d, dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = fa.bwd_workspace(B, N, H, d, dev)
+    ws = new_ws()
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
 
+    def varlen_fwd(qq, kk, vv, oo, ll, hs):
+        _lib.check(lib.fa_varlen_fwd(qq, kk, vv, oo, ll, cu.data_ptr(), cu.data_ptr(), L, L, H,
+                                     d, scale, causal, S, T, T, dtype, hs), "fa_varlen_fwd")
+
+    def varlen_bwd(qq, kk, vv, oo, dd, ll, gq, gk, gv, wsb, hs):
+        _lib.check(lib.fa_varlen_bwd(qq, kk, vv, oo, dd, ll, gq, gk, gv, cu.data_ptr(),
+                                     cu.data_ptr(), L, L, H, d, scale, causal, S, T, T,
+                                     wsb.data_ptr(), wsb.numel(), dtype, hs), "fa_varlen_bwd")
+
     def launch_fwd():
-        if wr.window is None:
+        if wr.varlen:
+            varlen_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), sh)
+        elif wr.window is None:
             _lib.check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                   lse.data_ptr(), B, N, H, d, scale, causal, dtype, sh), "fa_fwd")
         else:
@@ -547,7 +582,10 @@ def run_fattn(args, w):
                                         wr.window[1], dtype, sh), "fa_fwd_local")
 
     def launch_bwd():
-        if wr.window is None:
+        if wr.varlen:
+            varlen_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                       lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws, sh)
+        elif wr.window is None:
             _lib.check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                   do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
                                   dv.data_ptr(), B, N, H, d, scale, causal, ws.data_ptr(),
@@ -640,7 +678,7 @@ def run_fattn(args, w):
             outs = [o, lse, dq, dk, dv] if bset == 0 else [torch.empty_like(x)
                                                           for x in (o, lse, dq, dk, dv)]
             hout = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in outs]
-            wsb = ws if bset == 0 else fa.bwd_workspace(B, N, H, d, dev)
+            wsb = ws if bset == 0 else new_ws()
             sets.append((ins, outs, hout, wsb))
         h2d = sum(x.numel() * x.element_size() for x in hin)
         d2h = sum(x.numel() * x.element_size() for x in sets[0][2])
@@ -655,7 +693,10 @@ def run_fattn(args, w):
         def compute(ins, outs, wsb, hs):
             qq, kk, vv, dd = (x.data_ptr() for x in ins)
             oo, ll, gq, gk, gv = (x.data_ptr() for x in outs)
-            if wr.window is None:
+            if wr.varlen:
+                varlen_fwd(qq, kk, vv, oo, ll, hs)
+                varlen_bwd(qq, kk, vv, oo, dd, ll, gq, gk, gv, wsb, hs)
+            elif wr.window is None:
                 _lib.check(lib.fa_fwd(qq, kk, vv, oo, ll, B, N, H, d, scale, causal, dtype, hs),
                            "fa_fwd")
                 _lib.check(lib.fa_bwd(qq, kk, vv, oo, dd, ll, gq, gk, gv, B, N, H, d, scale,
@@ -741,21 +782,25 @@ def run_fattn(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows = 512
+        seq = max(wr.seqlens) if wr.varlen else wr.N
+        rows = min(512, seq)
         dt, fl, threads = oracle_sample_seconds(wr, rows)
         # grow the sample toward ~10 s of CPU work
-        while dt < 5.0 and rows < wr.N:
-            rows = min(wr.N, rows * 2)
+        while dt < 5.0 and rows < seq:
+            rows = min(seq, rows * 2)
             dt, fl, threads = oracle_sample_seconds(wr, rows)
+        where = (f"of head 0 of the longest packed sequence against all its {seq} keys"
+                 if wr.varlen else f"of head (b=0,h=0) against all {seq} keys")
         cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, **host_cpus(),
                "kind": "oracle",
-               "sample": f"last {rows} query rows of head (b=0,h=0) against all {wr.N} keys"
+               "sample": f"last {rows} query rows {where}"
                          f"{'' if wr.window is None else ' (window ' + str(list(wr.window)) + ')'}"
                          f", fp64 oracle fwd+bwd ({dt:.1f} s)",
                # one whole step (every head of every batch row) at the sample's rate
                "full_step_seconds_extrapolated": f_step / (fl / dt),
                "full_runs": [oracle_full_seconds(n) for n in ("tiny_causal", "a100table_N1024")]}
 
+    tensor_mb = q.numel() * q.element_size() / 1e6
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
@@ -765,7 +810,10 @@ def run_fattn(args, w):
                 "config": dict(wr.describe(), seed=w.seed,
                                parallelism=(f"heads{world} (head split, all-gather of O)"
                                             if split_heads else f"dp{world}"),
-                               l2="inputs larger than L2 (268 MB per tensor), no flush"),
+                               l2=(f"inputs larger than L2 ({tensor_mb:.0f} MB per tensor), "
+                                   "no flush" if tensor_mb > 126 else
+                                   f"inputs smaller than L2 ({tensor_mb:.1f} MB per tensor), "
+                                   "L2-warm, no flush")),
                 "fwd_tflops": f_fwd / (fwd_avg / 1e3) / 1e12,
                 "bwd_tflops": bwd_ach,
                 "pct_of_bf16_peak": {"fwd_bwd": value / world / peak_burst,
