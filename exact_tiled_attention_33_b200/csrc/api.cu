@@ -219,6 +219,17 @@ int normalize_window(int* wl, int* wr, long long max_q, long long max_k) {
 // those are launched first.
 int reverse_tiles(int wl, int wr) { return (wl < 0 && wr >= 0) ? 1 : 0; }
 
+// Grid of a varlen forward: per sequence (x = query tiles of the longest sequence, z =
+// sequences), or packed (x = the query tiles of all sequences) when that launches far fewer
+// CTAs (use_packed_grid; its tiles are 128 rows, as are the forward's).
+dim3 varlen_fwd_grid(FwdParams& p, int rows, int total_q, int num_seqs, int max_seqlen_q,
+                     int H) {
+  p.num_seqs = num_seqs;
+  p.packed = (rows == 128 && use_packed_grid(total_q, num_seqs, max_seqlen_q)) ? 1 : 0;
+  if (p.packed) return dim3((unsigned)packed_grid_tiles(total_q, num_seqs, max_seqlen_q), H, 1);
+  return dim3((max_seqlen_q + rows - 1) / rows, H, num_seqs);
+}
+
 int fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N,
               int H, int d, float scale, int wl, int wr, int dtype, void* stream) {
   if (int e = check_common(H, d, dtype, scale)) return e;
@@ -232,6 +243,8 @@ int fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, 
   if (int e = make_map(&mq, q, d, H, N, B, 128)) return e;
   if (int e = make_map(&mk, k, d, H, N, B, 128)) return e;
   if (int e = make_map(&mv, v, d, H, N, B, 128)) return e;
+  CUtensorMap mo;  // O leaves through TMA stores
+  if (int e = make_map(&mo, o, d, H, N, B, 128)) return e;
   FwdParams p{};
   p.o = o;
   p.lse = lse;
@@ -249,7 +262,8 @@ int fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, 
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   const int rows = fwd_rows_per_cta(false);
   dim3 grid((N + rows - 1) / rows, H, B);
-  return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+  return launch_result(
+      launch_fwd(d, dtype == FA_BF16, mq, mk, mv, mo, p, grid, (cudaStream_t)stream));
 }
 
 int fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -276,6 +290,8 @@ int fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
   const long long kr = total_k > 0 ? total_k : total_q;
   if (int e = make_map(&mk, kb, d, H, kr, 1, 128)) return e;
   if (int e = make_map(&mv, vb, d, H, kr, 1, 128)) return e;
+  CUtensorMap mo;
+  if (int e = make_map(&mo, o, d, H, total_q, 1, 128)) return e;
   FwdParams p{};
   p.o = o;
   p.lse = lse;
@@ -293,9 +309,10 @@ int fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
   p.max_seqlen_q = max_seqlen_q;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-  const int rows = fwd_rows_per_cta(false);
-  dim3 grid((max_seqlen_q + rows - 1) / rows, H, num_seqs);
-  return launch_result(launch_fwd(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+  const dim3 grid =
+      varlen_fwd_grid(p, fwd_rows_per_cta(false), total_q, num_seqs, max_seqlen_q, H);
+  return launch_result(
+      launch_fwd(d, dtype == FA_BF16, mq, mk, mv, mo, p, grid, (cudaStream_t)stream));
 }
 
 }  // namespace
@@ -403,6 +420,8 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
   if (int e = make_map(&mq, q, d, H, N, B, 128, 1)) return e;
   if (int e = make_map(&mk, k, d, H, N, B, 128, 1)) return e;
   if (int e = make_map(&mv, v, d, H, N, B, 128, 1)) return e;
+  CUtensorMap mo;  // 16-bit O
+  if (int e = make_map(&mo, o, d, H, N, B, 128)) return e;
   FwdParams p{};
   p.o = o;
   p.lse = lse;
@@ -420,7 +439,7 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
   const int rows = fwd_rows_per_cta(true);
   dim3 grid((N + rows - 1) / rows, H, B);
   return launch_result(
-      launch_fwd_fp8(d, out_dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+      launch_fwd_fp8(d, out_dtype == FA_BF16, mq, mk, mv, mo, p, grid, (cudaStream_t)stream));
 }
 
 int fa_varlen_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -448,6 +467,8 @@ int fa_varlen_fwd_fp8(const void* q, const void* k, const void* v, void* o, floa
   const long long kr = total_k > 0 ? total_k : total_q;
   if (int e = make_map(&mk, kb, d, H, kr, 1, 128, 1)) return e;
   if (int e = make_map(&mv, vb, d, H, kr, 1, 128, 1)) return e;
+  CUtensorMap mo;  // 16-bit O
+  if (int e = make_map(&mo, o, d, H, total_q, 1, 128)) return e;
   FwdParams p{};
   p.o = o;
   p.lse = lse;
@@ -464,10 +485,10 @@ int fa_varlen_fwd_fp8(const void* q, const void* k, const void* v, void* o, floa
   p.max_seqlen_q = max_seqlen_q;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
-  const int rows = fwd_rows_per_cta(true);
-  dim3 grid((max_seqlen_q + rows - 1) / rows, H, num_seqs);
+  const dim3 grid =
+      varlen_fwd_grid(p, fwd_rows_per_cta(true), total_q, num_seqs, max_seqlen_q, H);
   return launch_result(
-      launch_fwd_fp8(d, out_dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+      launch_fwd_fp8(d, out_dtype == FA_BF16, mq, mk, mv, mo, p, grid, (cudaStream_t)stream));
 }
 
 namespace {
@@ -532,15 +553,21 @@ int bwd_common(const void* q, const void* k, const void* v, const void* o, const
   p.reverse_tiles = reverse_tiles(wl, wr);
   p.max_seqlen_q = max_seqlen_q;
   p.max_seqlen_k = max_seqlen_k;
+  p.num_seqs = cu_q ? batches : 0;
+  // the single-pass kernel may take the packed grid over key tiles (use_packed_grid)
+  p.packed = (cu_q && single_pass && use_packed_grid(total_k, batches, max_seqlen_k)) ? 1 : 0;
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail(cudaGetLastError(), "status word");
   if (single_pass) {
+    BwdFusedMaps m;
+    m.q = mq; m.k = mk; m.v = mv; m.dout = mdo;
     // the fp32 dQ sums, [q_rows, H, d], reduce-added by the TMA unit 32 columns x 128 rows
     // at a time
-    CUtensorMap mdq;
-    if (int e = make_map_f32_reduce(&mdq, p.dq_acc, d, H, q_rows)) return e;
-    return launch_result(launch_bwd_fused(d, dtype == FA_BF16, mq, mk, mv, mdo, mdq, p, q_rows,
-                                          max_seqlen_q, max_seqlen_k, batches, stream));
+    if (int e = make_map_f32_reduce(&m.dq, p.dq_acc, d, H, q_rows)) return e;
+    if (int e = make_map(&m.dk, dk, d, H, kr, kb, 128)) return e;
+    if (int e = make_map(&m.dv, dv, d, H, kr, kb, 128)) return e;
+    return launch_result(
+        launch_bwd_fused(d, dtype == FA_BF16, m, p, q_rows, max_seqlen_k, batches, stream));
   }
   return launch_result(launch_bwd(d, dtype == FA_BF16, mq, mk, mv, mdo, p, q_rows, max_seqlen_q,
                                   max_seqlen_k, batches, stream));
@@ -912,7 +939,8 @@ int fa_selftest_fwd_f32(const void* q, const void* k, const void* v, float* o, f
   const int rows = fwd_rows_per_cta(false);
   dim3 grid((N + rows - 1) / rows, H, B);
   return launch_result(
-      launch_fwd_f32out(d, dtype == FA_BF16, mq, mk, mv, p, grid, (cudaStream_t)stream));
+      launch_fwd_f32out(d, dtype == FA_BF16, mq, mk, mv, /*unused*/ mq, p, grid,
+                        (cudaStream_t)stream));
 }
 
 int fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {

@@ -40,10 +40,8 @@ static LaunchResult launch_bwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
   return launch_status(cudaGetLastError());
 }
 
-template <int D, bool BF16>
-static LaunchResult launch_bwd_fused_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                                       const CUtensorMap& tmV, const CUtensorMap& tmDO,
-                                       const CUtensorMap& tmDQ, const BwdParams& p,
+template <int D, bool BF16, bool PACKED>
+static LaunchResult launch_bwd_fused_t(const BwdFusedMaps& m, const BwdParams& p,
                                        long long q_rows, int max_seqlen_k, int batches,
                                        cudaStream_t stream) {
   using C = BwdFusedCfg<D>;
@@ -52,7 +50,7 @@ static LaunchResult launch_bwd_fused_t(const CUtensorMap& tmQ, const CUtensorMap
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return LaunchResult::kCudaError;
   std::call_once(once[dev], [&] {
-    set_err[dev] = cudaFuncSetAttribute(fa_bwd_fused_kernel<D, BF16>,
+    set_err[dev] = cudaFuncSetAttribute(fa_bwd_fused_kernel<D, BF16, PACKED>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   });
   if (set_err[dev] != cudaSuccess) return launch_status(set_err[dev]);
@@ -63,7 +61,11 @@ static LaunchResult launch_bwd_fused_t(const CUtensorMap& tmQ, const CUtensorMap
   const long long pre_blocks = std::min<long long>((warps + 7) / 8, (long long)sms * 16);
   fa_bwd_pre_acc_kernel<D, BF16><<<(unsigned)pre_blocks, 256, 0, stream>>>(p, q_rows);
   // 2) dK, dV and the dQ partial sums: one CTA per key tile
-  dim3 grid((max_seqlen_k + C::BN - 1) / C::BN, p.H, batches);
+  //    (a packed varlen grid numbers the key tiles of all sequences: see packed_tile_lookup)
+  static_assert(C::BN == 128, "the packed grid's tiles are 128 keys");
+  const dim3 grid =
+      PACKED ? dim3((unsigned)packed_grid_tiles(p.total_k, batches, max_seqlen_k), p.H, 1)
+             : dim3((max_seqlen_k + C::BN - 1) / C::BN, p.H, batches);
   //    (a programmatic dependent of the preprocess: see grid_dependency_wait in the kernel)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -75,7 +77,8 @@ static LaunchResult launch_bwd_fused_t(const CUtensorMap& tmQ, const CUtensorMap
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, fa_bwd_fused_kernel<D, BF16>, tmQ, tmK, tmV, tmDO, tmDQ, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, fa_bwd_fused_kernel<D, BF16, PACKED>, m.q, m.k, m.v,
+                                     m.dout, m.dq, m.dk, m.dv, p);
   if (e != cudaSuccess) return launch_status(e);
   // 3) dQ = scale * sums, rounded to 16 bits
   const long long elems = q_rows * p.H * D;
@@ -89,18 +92,25 @@ static LaunchResult launch_bwd_fused_t(const CUtensorMap& tmQ, const CUtensorMap
   return launch_status(cudaGetLastError());
 }
 
-LaunchResult launch_bwd_fused(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                              const CUtensorMap& tmV, const CUtensorMap& tmDO,
-                              const CUtensorMap& tmDQ, const BwdParams& p, long long q_rows,
-                              int max_seqlen_q, int max_seqlen_k, int batches,
+// the packed varlen grid takes its own kernel instance
+template <int D, bool BF16>
+static LaunchResult launch_bwd_fused_grid(const BwdFusedMaps& m, const BwdParams& p,
+                                          long long q_rows, int max_seqlen_k, int batches,
+                                          cudaStream_t stream) {
+  return p.packed
+             ? launch_bwd_fused_t<D, BF16, true>(m, p, q_rows, max_seqlen_k, batches, stream)
+             : launch_bwd_fused_t<D, BF16, false>(m, p, q_rows, max_seqlen_k, batches, stream);
+}
+
+LaunchResult launch_bwd_fused(int d, bool bf16, const BwdFusedMaps& m, const BwdParams& p,
+                              long long q_rows, int max_seqlen_k, int batches,
                               cudaStream_t stream) {
-  (void)max_seqlen_q;
   if (d == 128)
-    return bf16 ? launch_bwd_fused_t<128, true>(tmQ, tmK, tmV, tmDO, tmDQ, p, q_rows, max_seqlen_k, batches, stream)
-                : launch_bwd_fused_t<128, false>(tmQ, tmK, tmV, tmDO, tmDQ, p, q_rows, max_seqlen_k, batches, stream);
+    return bf16 ? launch_bwd_fused_grid<128, true>(m, p, q_rows, max_seqlen_k, batches, stream)
+                : launch_bwd_fused_grid<128, false>(m, p, q_rows, max_seqlen_k, batches, stream);
   if (d == 64)
-    return bf16 ? launch_bwd_fused_t<64, true>(tmQ, tmK, tmV, tmDO, tmDQ, p, q_rows, max_seqlen_k, batches, stream)
-                : launch_bwd_fused_t<64, false>(tmQ, tmK, tmV, tmDO, tmDQ, p, q_rows, max_seqlen_k, batches, stream);
+    return bf16 ? launch_bwd_fused_grid<64, true>(m, p, q_rows, max_seqlen_k, batches, stream)
+                : launch_bwd_fused_grid<64, false>(m, p, q_rows, max_seqlen_k, batches, stream);
   return LaunchResult::kUnsupported;
 }
 

@@ -162,11 +162,14 @@ struct BwdFusedCfg {
   }
 };
 
-template <int D, bool BF16>
+// PACKED: the packed varlen grid (packed_tile_lookup), in an instance of its own so that the
+// lookup's code stays out of the other launches' kernels.
+template <int D, bool BF16, bool PACKED = false>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                        const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
+                        const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
+                        const __grid_constant__ CUtensorMap tmDV, const BwdParams p) {
   using C = BwdFusedCfg<D>;
   constexpr int BM = C::BM, BN = C::BN;
   enum { B_KV = 0, B_QFULL = 1, B_QEMPTY = 3, B_DOFULL = 5, B_DOEMPTY = 7, B_SFULL = 9, B_DPFULL, B_PFULL,
@@ -188,17 +191,25 @@ __global__ void __launch_bounds__(512, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // grid: x = key tile, y = head, z = batch or sequence, launched in groups of heads that
-  // share L2 (their Q, dO and dQ sums; see grouped_tile_order), key tile 0 (the one that
-  // sees the most query tiles when causal) first
+  // grid: x = key tile, y = head, z = batch or sequence (a packed varlen grid: x = the key
+  // tiles of all sequences, z = 1), launched in groups of heads that share L2 (their Q, dO
+  // and dQ sums; see grouped_tile_order), key tile 0 (the one that sees the most query tiles
+  // when causal) first
 #ifndef FATTN_BWD_HEAD_GROUP
 #define FATTN_BWD_HEAD_GROUP 4
 #endif
   const GridItem item = grouped_tile_order(FATTN_BWD_HEAD_GROUP);
   const int h = item.h;
-  const int bz = item.bz;
+  int bz = item.bz;
+  int ktile = item.tile;  // key tile within the batch or sequence
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
+    if constexpr (PACKED) {  // x numbers the key tiles of all segments, one after another
+      if (blockIdx.x == 0 && blockIdx.y == 0)
+        varlen_check_all(p.cu_q, p.cu_k, p.num_seqs, p.total_q, p.total_k, p.max_seqlen_q,
+                         p.max_seqlen_k, p.status);
+      if (!packed_tile_lookup(p.cu_k, p.num_seqs, p.total_k, item.tile, &bz, &ktile)) return;
+    }
     if (!varlen_segment_ok(p.cu_q, p.cu_k, bz, p.total_q, p.total_k, p.max_seqlen_q,
                            p.max_seqlen_k, p.status))
       return;
@@ -212,7 +223,7 @@ __global__ void __launch_bounds__(512, 1)
     Lq = Lk = p.N;
     bcoord = bz;
   }
-  const int k0 = item.tile * BN;
+  const int k0 = ktile * BN;
   if (k0 >= Lk) return;
   const int diag = Lk - Lq;
   const int wl = p.win_left, wr = p.win_right;
@@ -220,7 +231,7 @@ __global__ void __launch_bounds__(512, 1)
   query_tile_range(k0, min(k0 + BN - 1, Lk - 1), Lq, diag, wl, wr, BM, &i_begin, &n_q);
   // Without a right bound every key tile starts at the same query tile: rotate the order per
   // key tile so that CTAs running together add into different dQ rows.
-  const int rot = (wr < 0 && n_q > 0) ? item.tile % n_q : 0;
+  const int rot = (wr < 0 && n_q > 0) ? ktile % n_q : 0;
   auto q_tile = [&](int it) { int t = it + rot; if (t >= n_q) t -= n_q; return i_begin + t; };
   // token row of query 0 of this sequence in the dQ sums
   const long long acc_row0 = (p.cu_q != nullptr) ? (long long)q_row0 : (long long)bcoord * p.N;
@@ -510,7 +521,12 @@ __global__ void __launch_bounds__(512, 1)
       mbar_arrive(BAR(B_DSFULL));
     }
     // ---------------------------------------------------------------- epilogue
-    // half 0 stores dV, half 1 stores dK = scale · Σ dSᵀ Q
+    // half 0 stores dV, half 1 stores dK = scale · Σ dSᵀ Q.  Whole key tiles (and every dense
+    // tile: rows past N lie outside the tensor maps) leave through shared memory: each
+    // thread writes its row into the V (dV) or K (dK) tile, free once the last product
+    // completed, in the 128-byte swizzled layout, and one TMA store per 64-column chunk
+    // writes whole rows.  The last, partial tile of a packed sequence is stored row by row,
+    // so that it leaves the next sequence's rows alone.
     if (n_q > 0) {
       mbar_wait(BAR(B_DONE), 0, abort_flag, p.status);
       tc_fence_after();
@@ -520,6 +536,8 @@ __global__ void __launch_bounds__(512, 1)
                                         : (((size_t)bcoord * p.N + kg) * p.H + h) * D);
     const float sc = half == 0 ? 1.f : p.scale;
     const uint32_t tsrc = tmem + lane_off + (half == 0 ? C::TM_DV : C::TM_DK);
+    const bool via_tma = p.cu_q == nullptr || k0 + BN <= Lk;
+    const int stage_off = half == 0 ? C::OFF_V : C::OFF_K;
 #pragma unroll 1
     for (int q = 0; q < D / 32; ++q) {
       uint32_t v[32];
@@ -531,15 +549,36 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0u;
       }
-      if (key_ok) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+      uint4 w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        w[u] = make_uint4(
+            pack2<BF16>(__uint_as_float(v[8 * u]) * sc, __uint_as_float(v[8 * u + 1]) * sc),
+            pack2<BF16>(__uint_as_float(v[8 * u + 2]) * sc, __uint_as_float(v[8 * u + 3]) * sc),
+            pack2<BF16>(__uint_as_float(v[8 * u + 4]) * sc, __uint_as_float(v[8 * u + 5]) * sc),
+            pack2<BF16>(__uint_as_float(v[8 * u + 6]) * sc, __uint_as_float(v[8 * u + 7]) * sc));
+      if (via_tma) {
+        // 16-byte unit u of row r of a chunk sits at r * 128 + ((u ^ (r % 8)) * 16)
+        uint8_t* srow = sgen + stage_off + (q >> 1) * C::CHUNK + r * 128;
+        const int u0 = (q & 1) * 4;
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          dst[u] = make_uint4(
-              pack2<BF16>(__uint_as_float(v[8 * u]) * sc, __uint_as_float(v[8 * u + 1]) * sc),
-              pack2<BF16>(__uint_as_float(v[8 * u + 2]) * sc, __uint_as_float(v[8 * u + 3]) * sc),
-              pack2<BF16>(__uint_as_float(v[8 * u + 4]) * sc, __uint_as_float(v[8 * u + 5]) * sc),
-              pack2<BF16>(__uint_as_float(v[8 * u + 6]) * sc, __uint_as_float(v[8 * u + 7]) * sc));
+          *reinterpret_cast<uint4*>(srow + (((u0 + u) ^ (r & 7)) << 4)) = w[u];
+      } else if (key_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dst[u] = w[u];
+      }
+    }
+    if (via_tma) {  // uniform over the CTA
+      fence_proxy_async_smem();  // the rows above, visible to the TMA unit
+      named_barrier_sync(2 + half, 128);
+      if (quarter == 0 && lane == 0) {
+        const CUtensorMap* map = half == 0 ? &tmDV : &tmDK;
+        for (int c = 0; c < D / 64; ++c)
+          tma_store_4d(map, sbase + stage_off + c * C::CHUNK, c * 64, h, k_row0 + k0, bcoord);
+        bulk_commit_group();
+        bulk_wait_group_read0();  // shared memory stays allocated until the TMA has read it
       }
     }
   } else if (warp >= 12) {

@@ -28,6 +28,8 @@ struct FwdParams {
   int win_right;
   int reverse_tiles;// launch the query tiles with the most key tiles first
   int max_seqlen_q; // varlen: longest allowed segment (longer ones are skipped, reported)
+  int num_seqs;     // varlen: segments
+  int packed;       // varlen: grid x numbers the tiles of all segments (packed_tile_lookup)
   uint32_t* status; // device status word
 };
 
@@ -54,6 +56,8 @@ struct BwdParams {
   int win_left, win_right;  // attention window (see key_tile_range)
   int reverse_tiles;        // dQ pass: launch the query tiles with the most key tiles first
   int max_seqlen_q, max_seqlen_k;  // varlen: longest allowed segments (longer: skipped, reported)
+  int num_seqs;  // varlen: segments
+  int packed;    // varlen, single pass: grid x numbers the key tiles of all segments
   uint32_t* status;
 };
 
@@ -105,16 +109,45 @@ __host__ __device__ inline void query_tile_range(int k_first, int k_last, int Lq
 struct GridItem {
   int tile, h, bz;
 };
+// U: the unsigned type the arithmetic runs in (32 bits when the grid fits, which keeps the
+// divisions short on the device; 64 bits otherwise).
+template <typename U>
+__host__ __device__ inline GridItem grouped_grid_item_t(U L, U T, U H, U HB, U group) {
+  const U first = L / (group * T) * group;               // first (batch, head) of the group
+  const U gn = group < HB - first ? group : HB - first;  // pairs in the group
+  const U i = L - first * T;                             // < gn * T
+  const U hb = first + i % gn;
+  return {(int)(i / gn), (int)(hb % H), (int)(hb / H)};
+}
 __host__ __device__ inline GridItem grouped_grid_item(unsigned long long L, unsigned long long T,
                                                       unsigned long long H,
                                                       unsigned long long HB,
                                                       unsigned long long group) {
-  const unsigned long long first = L / (group * T) * group;  // first (batch, head) of the group
-  const unsigned long long gn = group < HB - first ? group : HB - first;  // pairs in the group
-  const unsigned long long i = L - first * T;                 // < gn * T
-  const unsigned long long hb = first + i % gn;
-  return {(int)(i / gn), (int)(hb % H), (int)(hb / H)};
+  if (T * HB <= 0xffffffffull && group * T <= 0xffffffffull)
+    return grouped_grid_item_t<unsigned>((unsigned)L, (unsigned)T, (unsigned)H, (unsigned)HB,
+                                         (unsigned)group);
+  return grouped_grid_item_t<unsigned long long>(L, T, H, HB, group);
 }
+
+// Packed varlen grid (the device side is packed_tile_lookup): a packing of `total` rows into
+// nseg segments has at most (total + 127 nseg) / 128 tiles of 128 rows, and never more than
+// the per-segment grid's nseg * ceil(max_len / 128).  The packed grid is used when the
+// per-segment grid would launch at least a quarter more CTAs (the surplus ones exit at
+// once, after the SM has paid for starting them) and the segments are few enough for the
+// per-warp prefix sum.
+constexpr long long kPackedMaxSeqs = 1024;
+__host__ __device__ inline long long packed_grid_tiles(long long total, long long nseg,
+                                                       long long max_len) {
+  const long long per_segment = nseg * ((max_len + 127) / 128);
+  const long long packed = (total + 127 * nseg) / 128;
+  return packed < per_segment ? packed : per_segment;
+}
+__host__ __device__ inline bool use_packed_grid(long long total, long long nseg,
+                                                long long max_len) {
+  return nseg <= kPackedMaxSeqs &&
+         4 * nseg * ((max_len + 127) / 128) >= 5 * packed_grid_tiles(total, nseg, max_len);
+}
+
 #ifdef __CUDACC__
 __device__ inline GridItem grouped_tile_order(unsigned group) {
   const unsigned long long T = gridDim.x, H = gridDim.y;
@@ -156,18 +189,18 @@ inline LaunchResult launch_status(cudaError_t e) {
 
 // Forward launch for one problem.  Tensor maps are built by the caller (api.cu).
 LaunchResult launch_fwd(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                        const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
-                        cudaStream_t stream);
+                        const CUtensorMap& tmV, const CUtensorMap& tmO, const FwdParams& p,
+                        dim3 grid, cudaStream_t stream);
 // FP8 (E4M3) operands, d = 128; bf16 selects the output format.
 LaunchResult launch_fwd_fp8(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                            const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
-                            cudaStream_t stream);
+                            const CUtensorMap& tmV, const CUtensorMap& tmO, const FwdParams& p,
+                            dim3 grid, cudaStream_t stream);
 
 // Test-only instance of the forward kernel that writes O in fp32 before rounding (p.o is
 // then a float buffer of the same shape).
 LaunchResult launch_fwd_f32out(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                               const CUtensorMap& tmV, const FwdParams& p, dim3 grid,
-                               cudaStream_t stream);
+                               const CUtensorMap& tmV, const CUtensorMap& tmO, const FwdParams& p,
+                               dim3 grid, cudaStream_t stream);
 
 // Query rows per forward CTA (grid x = ceil(rows / this), y = heads, z = batch or
 // sequences): one 128-row tile.
@@ -177,14 +210,18 @@ int fwd_rows_per_cta(bool fp8);
 LaunchResult launch_decode(int d, bool bf16, bool paged, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const DecParams& p, cudaStream_t stream);
 
+// Tensor maps of the single-pass backward: q, k, v, dout as for launch_bwd; dq over the
+// fp32 dQ sums p.dq_acc ([rows, H, D]; box 32 columns x 1 head x 128 rows, 128-byte
+// swizzle) that the pass reduce-adds its dQ partials through; dk, dv over the 16-bit
+// gradients (layout and box of k, v) that whole key tiles are stored through.
+struct BwdFusedMaps {
+  CUtensorMap q, k, v, dout, dq, dk, dv;
+};
+
 // Single-pass backward launch: D preprocess (and zeroing of the dQ sums), the fused
-// dK/dV/dQ pass, the dQ conversion.  As launch_bwd, plus tmDQ: a tensor map over the fp32
-// dQ sums p.dq_acc ([rows, H, D]; box 32 columns x 1 head x 128 rows, 128-byte swizzle)
-// that the pass reduce-adds its dQ partials through.
-LaunchResult launch_bwd_fused(int d, bool bf16, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                              const CUtensorMap& tmV, const CUtensorMap& tmDO,
-                              const CUtensorMap& tmDQ, const BwdParams& p, long long q_rows,
-                              int max_seqlen_q, int max_seqlen_k, int batches,
+// dK/dV/dQ pass, the dQ conversion.  q_rows and batches as for launch_bwd.
+LaunchResult launch_bwd_fused(int d, bool bf16, const BwdFusedMaps& m, const BwdParams& p,
+                              long long q_rows, int max_seqlen_k, int batches,
                               cudaStream_t stream);
 
 // Backward launch: D preprocess, dK/dV pass, dQ pass.  q_rows = B*N (dense) or total_q

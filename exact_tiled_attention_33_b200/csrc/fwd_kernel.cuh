@@ -91,10 +91,13 @@ struct FwdCfg {
 // BF16: 16-bit format of the output (and of the operands unless FP8).  F32O: the output is
 // written in fp32 before any rounding (a test-only instance: the library's entry points
 // all write 16-bit O; fa_selftest_fwd_f32 exposes this one to the parity tests).
-template <int D, bool BF16, bool FP8 = false, bool F32O = false>
+// PACKED: the packed varlen grid (packed_tile_lookup).  A separate instance, because the
+// lookup's code in the kernel body slowed the main loop of every launch by about 10%.
+template <int D, bool BF16, bool FP8 = false, bool F32O = false, bool PACKED = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const FwdParams p) {
   using C = FwdCfg<D, FP8>;
   constexpr int EL = 128 / C::EB;  // elements per 128-byte chunk (TMA x step)
   // 8-bit P is scaled by 2^6 (p = 2^(x - m + 6)) so that it spans the normal E4M3 range,
@@ -117,23 +120,32 @@ __global__ void __launch_bounds__(384, 1)
   const int lane = threadIdx.x & 31;
 
   // ---------------------------------------------------------------- work item
-  // grid: x = query tile, y = head, z = batch or sequence, launched in groups of heads that
-  // share L2 (see grouped_tile_order); when causal the tile with the most key tiles of each
-  // head comes first.
+  // grid: x = query tile, y = head, z = batch or sequence (a packed varlen grid: x = the
+  // query tiles of all sequences, z = 1), launched in groups of heads that share L2 (see
+  // grouped_tile_order); when causal the tile with the most key tiles of each head (or of
+  // each sequence) comes first.
 #ifndef FATTN_FWD_HEAD_GROUP
 #define FATTN_FWD_HEAD_GROUP 4
 #endif
   const GridItem item = grouped_tile_order(FATTN_FWD_HEAD_GROUP);
   const int h = item.h;
-  const int bz = item.bz;
-  const int tile = p.reverse_tiles ? (int)(gridDim.x - 1) - item.tile : item.tile;
+  int bz = item.bz;
+  int tile = p.reverse_tiles ? (int)(gridDim.x - 1) - item.tile : item.tile;
   int Lq, Lk, q_row0, k_row0, bcoord;
   if (p.cu_q != nullptr) {
+    if constexpr (PACKED) {  // x numbers the query tiles of all segments, one after another
+      if (blockIdx.x == 0 && blockIdx.y == 0)
+        varlen_check_all(p.cu_q, p.cu_k, p.num_seqs, p.total_q, p.total_k, p.max_seqlen_q, -1,
+                         p.status);
+      if (!packed_tile_lookup(p.cu_q, p.num_seqs, p.total_q, item.tile, &bz, &tile)) return;
+    }
     if (!varlen_segment_ok(p.cu_q, p.cu_k, bz, p.total_q, p.total_k, p.max_seqlen_q, -1,
                            p.status))
       return;
     q_row0 = p.cu_q[bz];
     Lq = p.cu_q[bz + 1] - q_row0;
+    if constexpr (PACKED)
+      if (p.reverse_tiles) tile = (Lq + BM - 1) / BM - 1 - tile;
     k_row0 = p.cu_k[bz];
     Lk = p.cu_k[bz + 1] - k_row0;
     bcoord = 0;
@@ -165,6 +177,26 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(BAR(C::B_ODONE), 1);
     *abort_flag = 0u;
     fence_barrier_init();
+    // Thread 0 is the TMA producer's lane: Q and the first K/V stages are requested right
+    // away, so their DRAM latency overlaps the tensor-memory allocation and the setup
+    // barrier (fresh stages need no EMPTY wait; the ones chunk written below lies outside
+    // the V tile's chunks).
+    if (n_kv > 0) {
+      mbar_arrive_expect_tx(BAR(C::B_QFULL), C::TILE);
+      for (int c = 0; c < C::KCH; ++c)
+        tma_load_4d(&tmQ, BAR(C::B_QFULL), sbase + C::OFF_Q + c * C::CHUNK, c * EL, h, q_row0 + q0,
+                    bcoord);
+      for (int j = 0; j < min(ST, n_kv); ++j) {
+        mbar_arrive_expect_tx(BAR(C::B_KFULL + j), C::TILE);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_4d(&tmK, BAR(C::B_KFULL + j), sbase + C::OFF_K + j * C::TILE + c * C::CHUNK,
+                      c * EL, h, k_row0 + (j0 + j) * BN, bcoord);
+        mbar_arrive_expect_tx(BAR(C::B_VFULL + j), C::TILE);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_4d(&tmV, BAR(C::B_VFULL + j), sbase + C::OFF_V + j * C::VSTAGE + c * C::CHUNK,
+                      c * EL, h, k_row0 + (j0 + j) * BN, bcoord);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -188,14 +220,8 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 0) {
     // ============================================================ TMA producer
     if (lane == 0 && n_kv > 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(BAR(C::B_QFULL), C::TILE);
-      for (int c = 0; c < C::KCH; ++c)
-        tma_load_4d(&tmQ, BAR(C::B_QFULL), sbase + C::OFF_Q + c * C::CHUNK, c * EL, h, q_row0 + q0,
-                    bcoord);
-      for (int j = 0; j < n_kv; ++j) {
+      // Q and key tiles 0 .. ST-1 were requested during setup
+      for (int j = ST; j < n_kv; ++j) {
         const int s = j % ST;
         const uint32_t ph = (uint32_t)(j / ST) & 1u;
         mbar_wait(BAR(C::B_KEMPTY + s), ph ^ 1u, abort_flag, p.status);
@@ -440,6 +466,13 @@ __global__ void __launch_bounds__(384, 1)
     const size_t orow_idx = (p.cu_q != nullptr) ? ((size_t)(q_row0 + i) * p.H + h) * D
                                                 : (((size_t)bcoord * p.N + i) * p.H + h) * D;
     uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + orow_idx;
+    // Whole query tiles (and every dense tile: rows past N lie outside the tensor map) leave
+    // through shared memory: each thread writes its row into the K stages, free once the
+    // last P·V product completed (every S product before it has), in the 128-byte swizzled
+    // layout, and one TMA store per 64-column chunk writes whole rows.  The last, partial
+    // tile of a packed sequence is stored row by row instead, so that it leaves the next
+    // sequence's rows alone.
+    const bool via_tma = !F32O && (p.cu_q == nullptr || q0 + BM <= Lq);
     // this half stores O columns [half * D/2, (half + 1) * D/2)
 #pragma unroll 1
     for (int q = half * (D / 64); q < (half + 1) * (D / 64); ++q) {
@@ -466,11 +499,29 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int e = 0; e < 16; ++e)
         pk[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-      if (valid) {
+      if (via_tma) {
+        // 16-byte unit u of row r of a chunk sits at r * 128 + ((u ^ (r % 8)) * 16)
+        uint8_t* srow = sgen + C::OFF_K + (q >> 1) * C::CHUNK + row * 128;
+        const int u0 = (q & 1) * 4;
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          *reinterpret_cast<uint4*>(srow + (((u0 + v4) ^ (row & 7)) << 4)) =
+              make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      } else if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4)
           dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      }
+    }
+    if (via_tma) {  // uniform over the CTA
+      fence_proxy_async_smem();  // the rows above, visible to the TMA unit
+      named_barrier_sync(1, 256);
+      if (warp == 4 && lane == 0) {
+        for (int c = 0; c < D / 64; ++c)
+          tma_store_4d(&tmO, sbase + C::OFF_K + c * C::CHUNK, c * 64, h, q_row0 + q0, bcoord);
+        bulk_commit_group();
+        bulk_wait_group_read0();  // shared memory stays allocated until the TMA has read it
       }
     }
     if (valid && half == 0) {

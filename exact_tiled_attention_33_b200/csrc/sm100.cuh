@@ -26,17 +26,65 @@ enum : uint32_t {
 // Varlen segment bz read from device prefix sums, checked before any use: rows
 // [cu_q[bz], cu_q[bz+1]) must lie in [0, total_q) and keys likewise in [0, total_k), and the
 // segment may hold at most q_cover rows and k_cover keys (the caller's max_seqlen_q /
-// max_seqlen_k, which size the grid; negative: not checked).  A bad segment is reported in the status word and its CTA does nothing, so a
-// malformed cu_seqlens never leads to an out-of-bounds access.
+// max_seqlen_k; negative: not checked).  A bad segment is reported in the status word and
+// its CTA does nothing, so a malformed cu_seqlens never leads to an out-of-bounds access.
+__device__ __forceinline__ bool varlen_bounds_ok(const int* cu_q, const int* cu_k, int bz,
+                                                 int total_q, int total_k, long long q_cover,
+                                                 long long k_cover) {
+  const int q0 = cu_q[bz], q1 = cu_q[bz + 1], k0 = cu_k[bz], k1 = cu_k[bz + 1];
+  return 0 <= q0 && q0 <= q1 && q1 <= total_q && 0 <= k0 && k0 <= k1 && k1 <= total_k &&
+         (q_cover < 0 || q1 - q0 <= q_cover) && (k_cover < 0 || k1 - k0 <= k_cover);
+}
 __device__ __forceinline__ bool varlen_segment_ok(const int* cu_q, const int* cu_k, int bz,
                                                   int total_q, int total_k, long long q_cover,
                                                   long long k_cover, uint32_t* status) {
-  const int q0 = cu_q[bz], q1 = cu_q[bz + 1], k0 = cu_k[bz], k1 = cu_k[bz + 1];
-  const bool ok = 0 <= q0 && q0 <= q1 && q1 <= total_q && 0 <= k0 && k0 <= k1 &&
-                  k1 <= total_k && (q_cover < 0 || q1 - q0 <= q_cover) &&
-                  (k_cover < 0 || k1 - k0 <= k_cover);
+  const bool ok = varlen_bounds_ok(cu_q, cu_k, bz, total_q, total_k, q_cover, k_cover);
   if (!ok && threadIdx.x == 0) atomicOr(status, kDevBadSeqlens);
   return ok;
+}
+// Every segment checked by one CTA (its threads stride over them): with the packed grid
+// below a segment without tiles has no CTA of its own to report it.
+__device__ __forceinline__ void varlen_check_all(const int* cu_q, const int* cu_k, int nseg,
+                                                 int total_q, int total_k, long long q_cover,
+                                                 long long k_cover, uint32_t* status) {
+  for (int s = threadIdx.x; s < nseg; s += blockDim.x)
+    if (!varlen_bounds_ok(cu_q, cu_k, s, total_q, total_k, q_cover, k_cover))
+      atomicOr(status, kDevBadSeqlens);
+}
+
+// Packed grid of a varlen launch: x numbers the 128-row tiles of all segments one segment
+// after another (ceil(L_s / 128) tiles for segment s, L_s = cu[s+1] - cu[s]), so no CTA is
+// launched for the tiles a short segment lacks.  Each warp finds the segment holding tile t
+// with a running prefix sum over cu[], 32 segments per step (lengths clamped to
+// [0, total] here; the CTA checks its own segment afterwards).  Returns false when t lies
+// past the last tile.  Called by whole warps.
+__device__ __forceinline__ bool packed_tile_lookup(const int* cu, int nseg, int total, int t,
+                                                   int* seg, int* tile) {
+  const int lane = threadIdx.x & 31;
+  long long base = 0;  // tiles of segments 0 .. s0-1
+  for (int s0 = 0; s0 < nseg; s0 += 32) {
+    const int s = s0 + lane;
+    int n = 0;
+    if (s < nseg) {
+      const long long len = (long long)cu[s + 1] - cu[s];
+      n = (int)((min(max(len, 0ll), (long long)total) + 127) >> 7);
+    }
+    int incl = n;  // inclusive prefix sum over the lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int step = __shfl_sync(0xffffffffu, incl, 31);
+    if (t < base + step) {
+      const int ls = __ffs(__ballot_sync(0xffffffffu, t < base + incl)) - 1;
+      *seg = s0 + ls;
+      *tile = (int)(t - base) - __shfl_sync(0xffffffffu, incl - n, ls);
+      return true;
+    }
+    base += step;
+  }
+  return false;
 }
 
 // Upper bound on a single mbarrier wait, in nanoseconds of %globaltimer.  A wait that

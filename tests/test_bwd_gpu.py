@@ -161,7 +161,7 @@ def test_autograd_sum_loss():
 
 # ------------------------------------------------------------------------------ varlen
 def run_varlen_bwd(lens_q, lens_k, H, d, causal, dtype="bf16", seed=3, perturb=None,
-                   deterministic=False):
+                   deterministic=False, nan_fill=False):
     cu_q = np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int32)
     cu_k = np.concatenate([[0], np.cumsum(lens_k)]).astype(np.int32)
     w = wl.custom("varlen_bwd", seqlens=lens_q, H=H, d=d, dtype=dtype, causal=causal, seed=seed)
@@ -177,8 +177,11 @@ def run_varlen_bwd(lens_q, lens_k, H, d, causal, dtype="bf16", seed=3, perturb=N
     cq, ck = torch.from_numpy(cu_q).to(DEV), torch.from_numpy(cu_k).to(DEV)
     mq, mk = max(lens_q), max(lens_k)
     o, lse = fa.varlen_fwd(qd, kd, vd, cq, ck, mq, mk, w.softmax_scale, causal)
+    # nan_fill: gradients start as NaN, so a key tile that no CTA covers cannot pass
+    pre = ([torch.full_like(x, float("nan")) for x in (qd, kd, vd)] if nan_fill
+           else [None, None, None])
     dq, dk, dv = fa.varlen_bwd(qd, kd, vd, o, lse, dod, cq, ck, mq, mk, w.softmax_scale, causal,
-                               deterministic=deterministic)
+                               deterministic=deterministic, dq=pre[0], dk=pre[1], dv=pre[2])
     assert fa.device_status() == 0
     qf, kf, vf, dof = (wl.to_f64(x) for x in (q, k, v, do))
     ref = oracle.varlen_attention_backward(qf, kf, vf, dof, cu_q, cu_k, w.softmax_scale, causal)
@@ -199,6 +202,26 @@ def test_varlen_pages_example():
 def test_varlen_ragged(d, causal, deterministic):
     lens = [1, 300, 0, 129, 77, 256, 2]
     run_varlen_bwd(lens, lens, 2, d, causal, seed=14, deterministic=deterministic)
+
+
+def _many_lengths(n, hi, long_len, seed):
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, hi + 1, size=n).tolist()
+    lens[n // 3] = long_len
+    return lens
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_many_segments_packed_grid(causal):
+    # 200 segments (lengths 0..100, one of 1000, some empty): the single-pass kernel's packed
+    # grid over key tiles, found by a seven-step prefix sum over cu_seqlens_k
+    lens = _many_lengths(200, 100, 1000, 43)
+    run_varlen_bwd(lens, lens, 2, 64, causal, seed=43, nan_fill=True)
+
+
+def test_varlen_over_1024_segments_per_segment_grid():
+    lens = _many_lengths(1100, 40, 300, 44)
+    run_varlen_bwd(lens, lens, 2, 64, True, seed=44, nan_fill=True)
 
 
 @pytest.mark.parametrize("causal", [False, True])

@@ -174,6 +174,27 @@ def test_varlen_ragged(d, causal):
     run_varlen(lens, lens, 3, d, causal, seed=11)
 
 
+def _many_lengths(n, hi, long_len, seed):
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, hi + 1, size=n).tolist()
+    lens[n // 3] = long_len
+    return lens
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_many_segments_packed_grid(causal):
+    # 200 segments (lengths 0..100, one of 1000, some empty): the packed grid, whose
+    # per-warp prefix sum over cu_seqlens then takes seven 32-segment steps
+    lens = _many_lengths(200, 100, 1000, 41)
+    run_varlen(lens, lens, 2, 64, causal, seed=41)
+
+
+def test_varlen_over_1024_segments_per_segment_grid():
+    # more segments than the packed grid's prefix sum takes: the per-segment grid, ragged
+    lens = _many_lengths(1100, 40, 300, 42)
+    run_varlen(lens, lens, 2, 64, True, seed=42)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_varlen_unequal_q_k(causal):
     # Lq != Lk per sequence: bottom-right causal alignment, including fully masked rows

@@ -15,6 +15,7 @@ import numpy as np
 import pytest
 
 import oracle
+from exact_tiled_attention_33_b200 import workloads as wl
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 CSRC = os.path.join(ROOT, "exact_tiled_attention_33_b200", "csrc")
@@ -117,6 +118,14 @@ def test_launch_order_is_a_grouped_tile_major_bijection(shim, T, H, B, group):
     inside a group tile 0 of each of its pairs first, then tile 1, and so on."""
     HB = H * B
     items = [_grid_item(shim, L, T, H, HB, group) for L in range(T * HB)]
+    # the 32-bit arithmetic the kernels take for grids below 2^32 CTAs agrees with 64 bits
+    f = shim.shim_grouped_grid_item_u64
+    f.argtypes = [ctypes.c_ulonglong] * 5 + [ctypes.POINTER(ctypes.c_int)]
+    f.restype = None
+    for L in range(T * HB):
+        out = (ctypes.c_int * 3)(-1, -1, -1)
+        f(L, T, H, HB, group, out)
+        assert tuple(out) == items[L]
     assert sorted(items) == sorted((t, h, b) for t in range(T) for h in range(H)
                                    for b in range(B))
     L = 0
@@ -127,3 +136,52 @@ def test_launch_order_is_a_grouped_tile_major_bijection(shim, T, H, B, group):
                 assert items[L] == (t, hb % H, hb // H), (L, items[L])
                 L += 1
     assert L == T * HB
+
+
+def _packed(shim):
+    for f in (shim.shim_packed_grid_tiles, shim.shim_use_packed_grid):
+        f.argtypes = [ctypes.c_longlong] * 3
+    shim.shim_packed_grid_tiles.restype = ctypes.c_longlong
+    shim.shim_use_packed_grid.restype = ctypes.c_int
+    return shim.shim_packed_grid_tiles, shim.shim_use_packed_grid
+
+
+def test_launch_order_beyond_32_bits(shim):
+    # a grid of more than 2^32 CTAs takes the 64-bit arithmetic: spot-check the bijection's
+    # formula there against the Python model
+    T, H, B, group = 2**20, 64, 2**13, 4
+    HB = H * B
+    for L in (0, 1, 2**32 - 1, 2**32, 2**32 + 12345, T * HB - 1):
+        first = L // (group * T) * group
+        gn = min(group, HB - first)
+        i = L - first * T
+        hb = first + i % gn
+        assert _grid_item(shim, L, T, H, HB, group) == (i // gn, hb % H, hb // H)
+
+
+def test_packed_grid_covers_every_tile(shim):
+    # The packed varlen grid numbers the 128-row tiles of all segments one after another; its
+    # size must cover sum(ceil(L_s / 128)) for every packing of `total` rows into segments
+    # no longer than max_len, and never exceed the per-segment grid.
+    tiles, _ = _packed(shim)
+    rng = np.random.default_rng(5)
+    for _ in range(2000):
+        nseg = int(rng.integers(1, 300))
+        hi = int(rng.choice([1, 60, 128, 129, 700, 5000]))
+        lens = rng.integers(0, hi + 1, size=nseg)
+        total, mx = int(lens.sum()), int(lens.max())
+        need = int(((lens + 127) // 128).sum())
+        got = tiles(total, nseg, mx)
+        assert need <= got <= nseg * ((mx + 127) // 128), (lens.tolist(), got)
+    # tight when every segment is a multiple of 128 rows long and as long as max_len
+    assert tiles(64 * 4096, 64, 4096) == 64 * 32
+
+
+def test_packed_grid_choice(shim):
+    _, use = _packed(shim)
+    seqlens = wl.varlen_lengths_64(3)
+    assert use(sum(seqlens), 64, max(seqlens)) == 1       # the 64-sequence mix: packed
+    assert use(64 * 4096, 64, 4096) == 0                   # equal lengths: per segment
+    assert use(3 * 1024, 3, 1024) == 0
+    assert use(128 + 256 + 512, 3, 512) == 1               # 12 per-segment CTAs for 9 tiles
+    assert use(1025 * 10, 1025, 3000) == 0                 # more segments than the scan takes
