@@ -255,6 +255,17 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(BAR(B_DONE), 1);
     *abort_flag = 0u;
     fence_barrier_init();
+    // Thread 0 is the loads warp's lane: this key tile's K and V are requested right away,
+    // so that their DRAM latency overlaps the tensor-memory allocation and the setup barrier.
+    if (n_q > 0) {
+      mbar_arrive_expect_tx(BAR(B_KV), 2 * C::TILE);
+      for (int c = 0; c < C::KCH; ++c) {
+        tma_load_4d(&tmK, BAR(B_KV), sbase + C::OFF_K + c * C::CHUNK, c * 64, h, k_row0 + k0,
+                    bcoord);
+        tma_load_4d(&tmV, BAR(B_KV), sbase + C::OFF_V + c * C::CHUNK, c * 64, h, k_row0 + k0,
+                    bcoord);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -269,16 +280,9 @@ __global__ void __launch_bounds__(512, 1)
   if (warp == 0) {
     // ============================================================ loads
     if (n_q > 0) {
-      if (lane == 0) {
+      if (lane == 0) {  // K and V were requested during setup
         tma_prefetch_desc(&tmQ);
-        tma_prefetch_desc(&tmK);
-        tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmDO);
-        mbar_arrive_expect_tx(BAR(B_KV), 2 * C::TILE);
-        for (int c = 0; c < C::KCH; ++c) {
-          tma_load_4d(&tmK, BAR(B_KV), sbase + C::OFF_K + c * C::CHUNK, c * 64, h, k_row0 + k0, bcoord);
-          tma_load_4d(&tmV, BAR(B_KV), sbase + C::OFF_V + c * C::CHUNK, c * 64, h, k_row0 + k0, bcoord);
-        }
       }
       grid_dependency_wait();  // D comes from the preceding preprocess launch
       for (int it = 0; it < n_q; ++it) {
@@ -658,7 +662,10 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-    if (leader) bulk_wait_group0();  // every reduce-add has completed before the CTA ends
+    // The staging tiles must stay allocated until the TMA unit has read them.  Completion of
+    // the reduce-adds themselves is not waited for here: the dQ conversion, a programmatic
+    // dependent, waits for this grid's completion and the visibility of its memory operations.
+    if (leader) bulk_wait_group_read0();
   }
 
   tc_fence_before();

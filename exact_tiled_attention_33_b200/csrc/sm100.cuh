@@ -244,7 +244,7 @@ __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, uint32
       "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
-// Wait until at most two of this thread's bulk groups are still reading shared memory.
+// Wait until at most one of this thread's bulk groups is still reading shared memory.
 __device__ __forceinline__ void bulk_wait_group_read1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
