@@ -216,7 +216,7 @@ def run_varlen(lens_q, lens_k, H, d, window, seed, bwd=True):
     # per (segment, head) scale; a window of one key per row makes the exact dQ = dK = 0
     check_grad_segments([f64(dq), f64(dk), f64(dv)], (gq, gk, gv), cq, ck,
                         f"varlen window {window}", scale, False, "bf16", qf, kf, vf, dof,
-                        window=window, o16_always=tuple(window) == (0, 0))
+                        window=window)
 
 
 @pytest.mark.parametrize("window", [(1, 0), (100, 0), (128, 3), (20, 20), (-1, 7), (50, -1)])
