@@ -14,19 +14,21 @@ static LaunchResult launch_bwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                  const BwdParams& p, long long q_rows, int max_seqlen_q,
                                  int max_seqlen_k, int batches, cudaStream_t stream) {
   using C = BwdCfg<D>;
-  static bool configured[64] = {};
+  static std::once_flag once[64];
+  static cudaError_t set_err[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LaunchResult::kCudaError;
+  if (dev < 0 || dev >= 64) return launch_status(cudaErrorInvalidDevice);
+  std::call_once(once[dev], [&] {
+    set_err[dev] = cudaFuncSetAttribute(fa_bwd_dkdv_kernel<D, BF16>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_A);
+    if (set_err[dev] == cudaSuccess)
+      set_err[dev] = cudaFuncSetAttribute(fa_bwd_dq_kernel<D, BF16>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B);
+  });
+  if (set_err[dev] != cudaSuccess) return launch_status(set_err[dev]);
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(fa_bwd_dkdv_kernel<D, BF16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_A) != cudaSuccess ||
-        cudaFuncSetAttribute(fa_bwd_dq_kernel<D, BF16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_B) != cudaSuccess)
-      return LaunchResult::kCudaError;
-    configured[dev] = true;
-  }
   // 1) D = rowsum(dO ∘ O)
   const long long warps = q_rows * p.H;
   const long long pre_blocks = std::min<long long>((warps + 7) / 8, (long long)sms * 16);
@@ -48,7 +50,8 @@ static LaunchResult launch_bwd_fused_t(const BwdFusedMaps& m, const BwdParams& p
   static std::once_flag once[64];
   static cudaError_t set_err[64] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return LaunchResult::kCudaError;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LaunchResult::kCudaError;
+  if (dev < 0 || dev >= 64) return launch_status(cudaErrorInvalidDevice);
   std::call_once(once[dev], [&] {
     set_err[dev] = cudaFuncSetAttribute(fa_bwd_fused_kernel<D, BF16, PACKED>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);

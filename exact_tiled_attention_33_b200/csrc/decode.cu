@@ -1,4 +1,6 @@
 // KV-cache decode kernel instantiations and launcher.
+#include <mutex>
+
 #include "decode_kernel.cuh"
 
 namespace fattn {
@@ -8,15 +10,16 @@ static LaunchResult launch_decode_t(const CUtensorMap& tmK, const CUtensorMap& t
                                     const DecParams& p, cudaStream_t stream) {
   using C = DecCfg<D, NQ>;
   auto kern = fa_decode_kernel<D, BF16, PAGED, NQ>;
-  static bool configured[64] = {};
+  static std::once_flag once[64];
+  static cudaError_t set_err[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LaunchResult::kCudaError;
-  if (dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
-      return LaunchResult::kCudaError;
-    configured[dev] = true;
-  }
+  if (dev < 0 || dev >= 64) return launch_status(cudaErrorInvalidDevice);
+  std::call_once(once[dev], [&] {
+    set_err[dev] =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  });
+  if (set_err[dev] != cudaSuccess) return launch_status(set_err[dev]);
   kern<<<dim3(p.splits, p.H, p.B), C::THREADS, C::SMEM_BYTES, stream>>>(tmK, tmV, p);
   if (p.splits > 1) {
     const long long warps = (long long)p.B * p.Nq * p.H;
