@@ -91,6 +91,16 @@ struct FwdCfg {
 // BF16: 16-bit format of the output (and of the operands unless FP8).  F32O: the output is
 // written in fp32 before any rounding (a test-only instance: the library's entry points
 // all write 16-bit O; fa_selftest_fwd_f32 exposes this one to the parity tests).
+// The check of every segment that the packed grid's first CTA makes, kept out of line: inlined
+// into the kernel body it slowed the main loop of the instance that contains it by about 10%.
+static __device__ __noinline__ void varlen_check_all_out_of_line(const int* cu_q,
+                                                                 const int* cu_k, int nseg,
+                                                                 int total_q, int total_k,
+                                                                 long long q_cover,
+                                                                 uint32_t* status) {
+  varlen_check_all(cu_q, cu_k, nseg, total_q, total_k, q_cover, -1, status);
+}
+
 // PACKED: the packed varlen grid (packed_tile_lookup).  A separate instance, because the
 // lookup's code in the kernel body slowed the main loop of every launch by about 10%.
 template <int D, bool BF16, bool FP8 = false, bool F32O = false, bool PACKED = false>
@@ -135,8 +145,8 @@ __global__ void __launch_bounds__(384, 1)
   if (p.cu_q != nullptr) {
     if constexpr (PACKED) {  // x numbers the query tiles of all segments, one after another
       if (blockIdx.x == 0 && blockIdx.y == 0)
-        varlen_check_all(p.cu_q, p.cu_k, p.num_seqs, p.total_q, p.total_k, p.max_seqlen_q, -1,
-                         p.status);
+        varlen_check_all_out_of_line(p.cu_q, p.cu_k, p.num_seqs, p.total_q, p.total_k,
+                                     p.max_seqlen_q, p.status);
       if (!packed_tile_lookup(p.cu_q, p.num_seqs, p.total_q, item.tile, &bz, &tile)) return;
     }
     if (!varlen_segment_ok(p.cu_q, p.cu_k, bz, p.total_q, p.total_k, p.max_seqlen_q, -1,
