@@ -77,9 +77,12 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 
 /* Varlen forward over packed sequences (flash_attn_varlen_func semantics).
  * Writes o [total_q,H,d] and lse [H,total_q].
- * max_seqlen_q / max_seqlen_k must be >= every sequence's length (they size the grid);
- * num_seqs, total_q, total_k are the host-side counts matching cu_seqlens (the host
- * cannot read device cu_seqlens without a synchronisation).  num_seqs <= 65535.
+ * max_seqlen_q / max_seqlen_k must be >= every sequence's length; num_seqs, total_q,
+ * total_k are the host-side counts matching cu_seqlens (the host cannot read device
+ * cu_seqlens without a synchronisation).  num_seqs <= 65535.  Together they size the grid:
+ * one CTA per 128-row tile of all sequences ((total + 127 num_seqs) / 128 at most) when
+ * that is well below one slot per tile of the longest sequence for every sequence and
+ * num_seqs <= 1024, otherwise the latter.
  * The kernels check every segment before using it: a segment outside [0, total_q) or
  * [0, total_k), or longer than max_seqlen_q (forward, dQ) or max_seqlen_k (dK/dV), is
  * skipped (its outputs are left unwritten) and fa_get_device_status then returns
