@@ -49,6 +49,15 @@ def test_reference_arm_windowed():
     _check_line(d, "long_local_sym512")
 
 
+def test_reference_arm_varlen():
+    # packed sequences: the sample is drawn from the longest sequence, the config names the
+    # packing
+    d = _run(["--impl", "reference", "--workload", "varlen3", "--steps", "1", "--warmup", "0"])
+    _check_line(d, "varlen3")
+    assert d["config"]["num_seqs"] == 3 and d["config"]["total_tokens"] == 896
+    assert d["config"]["max_seqlen"] == 512
+
+
 def test_reference_arm_decode():
     d = _run(["--impl", "reference", "--workload", "decode_q4_l8k", "--steps", "1",
               "--warmup", "0"])
